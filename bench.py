@@ -1,0 +1,364 @@
+"""Throughput benchmark of the fused MoE expert layer on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl {b200,reference}]
+
+One step = one whole layer (route, gather, FC1 + SwiGLU + FP8 requant, FC2,
+combine) over one batch of seeded synthetic inputs already resident in HBM.
+The default workload is the decode-size layer (T=128, H=7168, I=2048, E=32,
+top-8, skewed routing).  With N > 1 (launched by torch.distributed.run) every
+rank runs its own replica of the layer on its own GPU: the path has no exchange
+step, so there is no collective on the data path (weak scaling); the elapsed
+device time is the maximum over ranks.
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
+on the launching stream; L2 is flushed (a 256 MiB buffer is overwritten)
+before every timed step, outside the events.  `e2e` times the same layer
+through the C ABI's host-buffer entry point (pinned host inputs copied in,
+output copied back, all inside the events).
+
+`--impl reference` times the float64 CPU oracle on the host cores instead (a
+bounded sample of the workload's tokens per step) and prints the same line.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s and achieved TFLOPS or HBM GB/s vs roofline, 1×B200"
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), \
+            "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def _dist():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+class Clocks:
+    """Samples SM clocks and throttle reasons with nvidia-smi during timing."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+
+    def start(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def algorithmic_bytes(wl, d):
+    """Bytes the layer must move at minimum: the weights and scales of the
+    experts that receive tokens, x and its scales, the routing, the output."""
+    import torch
+    counts = torch.bincount(d["topk_idx"].reshape(-1).long(), minlength=wl.E)[:wl.E]
+    active = int((counts > 0).sum())
+    per_expert_w = sum(d[k][0].numel() for k in ("w1", "w1_scales", "w2", "w2_scales"))
+    fc1_w = d["w1"][0].numel() + d["w1_scales"][0].numel()
+    act_bytes = (d["x"].numel() + d["x_scales"].numel() + d["topk_idx"].numel() * 4 +
+                 d["topk_w"].numel() * 4 + wl.T * wl.H * 2)
+    return active * per_expert_w + act_bytes, active * fc1_w, active
+
+
+def run_b200(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    import moe_expert_ffn_permute_b200 as moe
+    from moe_expert_ffn_permute_b200.build import build
+    from moe_expert_ffn_permute_b200.synth import make_inputs
+
+    rank, world, local = _dist()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    if rank == 0:
+        build()
+    if world > 1:
+        dist.barrier()
+    lib = moe.lib()
+    dev = torch.device("cuda", local)
+    d = make_inputs(wl, device=dev)
+    lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype=wl.w_dtype, act=wl.act,
+                       alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit, device=dev)
+    out = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    args_dev = (d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], d["w1"], d["w1_scales"],
+                d["w2"], d["w2_scales"])
+
+    def fwd():
+        moe.moe_forward(lay.plan, *args_dev, out, lay.workspace, stream)
+
+    steps = [("route", lambda: moe.moe_route(lay.plan, d["topk_idx"], lay.workspace, stream)),
+             ("gather", lambda: moe.moe_gather(lay.plan, d["x"], d["x_scales"], lay.workspace,
+                                               stream)),
+             ("fc1", lambda: moe.moe_fc1(lay.plan, d["w1"], d["w1_scales"], lay.workspace,
+                                         stream)),
+             ("fc2", lambda: moe.moe_fc2(lay.plan, d["w2"], d["w2_scales"], lay.workspace,
+                                         stream)),
+             ("combine", lambda: moe.moe_combine(lay.plan, d["topk_w"], out, lay.workspace,
+                                                 stream))]
+
+    for _ in range(args.warmup):
+        fwd()
+    torch.cuda.synchronize()
+    if lay.check() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    # ---- timed: whole layer, device-resident inputs
+    clocks = Clocks(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        fwd()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = sum(step_ms)
+
+    # ---- per-kernel split (same launch sequence, one event per step boundary)
+    split = {name: [] for name, _ in steps}
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(steps) + 1)]
+        evs[0].record(stream)
+        for j, (_, fn) in enumerate(steps):
+            fn()
+            evs[j + 1].record(stream)
+        torch.cuda.synchronize()
+        for j, (name, _) in enumerate(steps):
+            split[name].append(evs[j].elapsed_time(evs[j + 1]))
+
+    # ---- e2e through the host-buffer entry point
+    host = {k: d[k].cpu().pin_memory() for k in ("x", "x_scales", "topk_idx", "topk_w")}
+    out_h = torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory()
+    for _ in range(args.warmup):
+        moe.moe_forward_hostio(lay.plan, host["x"], host["x_scales"], host["topk_idx"],
+                               host["topk_w"], d["w1"], d["w1_scales"], d["w2"], d["w2_scales"],
+                               out_h, lay.workspace, stream)
+    torch.cuda.synchronize()
+    e2e_ms = []
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        moe.moe_forward_hostio(lay.plan, host["x"], host["x_scales"], host["topk_idx"],
+                               host["topk_w"], d["w1"], d["w1_scales"], d["w2"], d["w2_scales"],
+                               out_h, lay.workspace, stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms.append(a.elapsed_time(b))
+    if lay.check() != 0:
+        raise RuntimeError("device error during timing")
+
+    # ---- max over ranks
+    vals = torch.tensor([total_ms, sum(e2e_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    total_ms, e2e_total = float(vals[0]), float(vals[1])
+
+    alg_bytes, fc1_bytes, active = algorithmic_bytes(wl, d)
+    hbm, bf16, bf16_sus, peak_src = _peaks()
+    flops = 6.0 * wl.S * wl.H * wl.I
+    fc1_flops = 4.0 * wl.S * wl.H * wl.I
+    fc1_ms = statistics.mean(split["fc1"])
+    hbm_bound = alg_bytes / (hbm * 1e9) > flops / (2 * bf16 * 1e12)
+    if hbm_bound:
+        roof = {"bound": "hbm", "achieved": round(fc1_bytes / (fc1_ms * 1e-3) / 1e9, 1),
+                "peak": hbm, "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": round(fc1_flops / (fc1_ms * 1e-3) / 1e12, 1),
+                "peak": round(2 * bf16, 1), "unit": "TFLOP/s"}
+    roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
+    roof["traffic"] = None
+    roof["kernel"] = "fc1 (grouped GEMM + SwiGLU + FP8 requant)"
+    roof["peak_source"] = f"{peak_src}" + ("" if roof["unit"] == "GB/s" else
+                                           " bf16 burst x2 (FP8 = 2x bf16 nominal)")
+
+    tokens = wl.T * world
+    ms_per_step = total_ms / args.steps
+    res = {
+        "metric": METRIC, "value": round(tokens / (total_ms * 1e-3 / args.steps), 1),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8_e4m3" if wl.w_dtype == "e4m3" else "fp8_e4m3xe2m1",
+        "data": "synthetic (seeded; random-init weights)",
+        "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
+                   "w_dtype": wl.w_dtype, "routing": wl.routing, "act": wl.act,
+                   "active_experts": active, "l2": "flushed (256 MiB write) before each step",
+                   "parallelism": f"replicas x{world}"},
+        "achieved": {"tflops": round(flops / (ms_per_step * 1e-3) / 1e12, 2),
+                     "hbm_gbs": round(alg_bytes / (ms_per_step * 1e-3) / 1e9, 1),
+                     "alg_bytes": alg_bytes, "flops": flops},
+        "kernels_ms": {k: round(statistics.mean(v), 4) for k, v in split.items()},
+        "roofline": roof,
+        "e2e": {"value": round(tokens / (e2e_total * 1e-3 / args.steps), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(sum(v.numel() * v.element_size() for v in host.values())),
+                "d2h_bytes_per_step": int(out_h.numel() * 2)},
+        "gpu_launches": moe.moe_forward_launch_count(lay.plan) * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(wl, d, args)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res))
+
+
+def _oracle_sample(wl, dn, tokens):
+    from oracle import layer as L
+    sub = dict(dn)
+    for key in ("x", "x_scales", "topk_idx", "topk_w"):
+        sub[key] = dn[key][tokens]
+    return L.layer(sub["x"], sub["x_scales"], sub["topk_idx"], sub["topk_w"], dn["w1"],
+                   dn["w1_scales"], dn["w2"], dn["w2_scales"], w_dtype=wl.w_dtype,
+                   alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit)
+
+
+def _cores():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = max((i.get("num_threads", 1) for i in info), default=os.cpu_count())
+        return int(n)
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(wl, d, args, ntok=None):
+    """The float64 oracle, as it stands, on a bounded sample of the workload's
+    tokens (the oracle's cost is dominated by dequantising the touched experts'
+    weights, so a few tokens already take seconds)."""
+    dn = {k: v.cpu().numpy() for k, v in d.items()}
+    ntok = ntok or args.cpu_tokens
+    t0 = time.perf_counter()
+    _oracle_sample(wl, dn, list(range(ntok)))
+    dt = time.perf_counter() - t0
+    return {"value": round(ntok / dt, 4), "unit": "tokens/s", "cores": _cores(),
+            "kind": "oracle", "sample": f"first {ntok} of {wl.T} tokens of {wl.name}, "
+                                        f"float64 NumPy, {dt:.1f} s"}
+
+
+def run_reference(args, wl):
+    rank, world, _ = _dist()
+    if rank != 0:
+        return
+    import torch
+    from moe_expert_ffn_permute_b200.synth import make_inputs
+    d = make_inputs(wl, device="cuda" if torch.cuda.is_available() else "cpu")
+    dn = {k: v.cpu().numpy() for k, v in d.items()}
+    ntok = args.cpu_tokens
+    for i in range(args.warmup):
+        _oracle_sample(wl, dn, [i % wl.T])
+    times = []
+    for i in range(args.steps):
+        t0 = time.perf_counter()
+        _oracle_sample(wl, dn, [(j + i * ntok) % wl.T for j in range(ntok)])
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    val = ntok * args.steps / total
+    res = {"metric": METRIC, "value": round(val, 4), "unit": "tokens/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(1e3 * total / args.steps, 2), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "impl": "reference",
+           "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E,
+                      "k": wl.k, "w_dtype": wl.w_dtype},
+           "cpu_baseline": {"value": round(val, 4), "unit": "tokens/s", "cores": _cores(),
+                            "kind": "oracle",
+                            "sample": f"{ntok} token(s) of {wl.name} per step"},
+           "e2e": {"value": round(val, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(res))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode")
+    ap.add_argument("--tokens", type=int, default=None, help="override T (mxfp4 sweep)")
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--cpu-tokens", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    from moe_expert_ffn_permute_b200.synth import WORKLOADS
+    wl = WORKLOADS[args.workload]
+    if args.tokens:
+        wl = wl.with_tokens(args.tokens)
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_b200(args, wl)
+
+
+if __name__ == "__main__":
+    main()

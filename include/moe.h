@@ -1,0 +1,222 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) fused MoE expert layer.
+ *
+ * What the layer computes (per token t, top-k slots j = 0..k-1, e = topk_idx[t,j]):
+ *
+ *   xh      = E4M3(x[t]) * UE8M0(x_scales[t, c/128])                  (1x128 blocks)
+ *   h       = xh @ W1[e]^T,  W1[e] = [2I, H]: rows [0,I) gate, [I,2I) up
+ *   a       = min(g,L) * sigmoid(alpha*min(g,L)) * (clamp(u,-L,L) + up_bias)
+ *   q, sq   = FP8 E4M3 requantisation of a with one UE8M0 scale per 1x128 block
+ *   y[t,j]  = (q * sq) @ W2[e]^T,  W2[e] = [H, I]
+ *   out[t]  = bf16( sum_j topk_w[t,j] * y[t,j] )     (fp32 sum, j ascending)
+ *
+ * Sources (web pages, by title and section):
+ *   - DeepGEMM PR #445 "fix(sm90): support parameterized SwiGLU in FP8 MegaMoE",
+ *     Summary / Compatibility: the activation and its parameters (defaults
+ *     alpha = 1, up_bias = 0 give SiLU(gate) * up; the clamp is optional).
+ *   - DeepGEMM PR #386 "Optimize sm100 version with token-aware BM240 tiling,
+ *     native UE8M0, and direct combine", title / Description: UE8M0 block
+ *     scales consumed natively and the direct weighted combine to token order.
+ *   - fw-ai/DeepGEMM PR #16 "Sync upstream through PR #441: fix Mega MoE
+ *     scheduler ordering", Overview: the persistent tile scheduler's task-info
+ *     slots and their release ordering (used inside moe_fc1 / moe_fc2).
+ *   - TensorRT-LLM PR #16346 "DSV4 o_proj: fuse fp8/UE8M0 quantize ...",
+ *     Description: BF16/FP32 -> FP8 + 1x128 UE8M0 quantisation fused into a
+ *     GEMM epilogue (the FC1 epilogue here).
+ *
+ * Conventions for every entry point:
+ *   - All tensors are row-major and contiguous; all device pointers must be
+ *     16-byte aligned (MXFP4 weight pointers 32-byte aligned).
+ *   - Ownership: the caller owns every buffer, host or device.  The library
+ *     never allocates or frees device memory; a plan is a small host object.
+ *   - Errors are returned as moe_status; nothing is thrown across the ABI.
+ *     Argument validation happens before anything is enqueued: a call that
+ *     returns an error has launched nothing.
+ *   - Device-side problems (an expert id outside [0,E), a bounded wait that ran
+ *     out) are recorded in an error word inside the workspace; read it with
+ *     moe_check_device_error().  A slot with an out-of-range expert id is not
+ *     routed: it contributes nothing to its token's output.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) unless stated otherwise.  Calls with different plans or
+ *     different workspaces may run concurrently; two calls sharing one
+ *     workspace must be ordered on one stream.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *moe_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,    /* null pointer, bad size, k > E, ...           */
+  MOE_ERR_UNSUPPORTED = 2,    /* shape the kernels do not handle (H % 128 ...) */
+  MOE_ERR_ALIGNMENT = 3,      /* pointer not 16 B (MXFP4 weights: 32 B) aligned */
+  MOE_ERR_CUDA = 4,           /* a CUDA runtime call failed                     */
+  MOE_ERR_DEVICE_TIMEOUT = 5, /* a bounded device wait ran out (see error word) */
+  MOE_ERR_BAD_ROUTING = 6     /* a topk_idx entry was outside [0, E)            */
+} moe_status;
+
+/* Weight formats.  Activations x are always E4M3 with one UE8M0 per 1x128. */
+typedef enum {
+  MOE_W_E4M3_UE8M0_128x128 = 0, /* W1 u8 [E,2I,H], scales u8 [E,2I/128,H/128]  */
+  MOE_W_E2M1_UE8M0_1x32 = 1     /* W1 u8 [E,2I,H/2] (two E2M1 codes per byte,
+                                   element 2i in the low nibble),
+                                   scales u8 [E,2I,H/32]; W2 likewise [E,H,I/2],
+                                   [E,H,I/32]                                   */
+} moe_wdtype;
+
+typedef struct {
+  int w_dtype; /* a moe_wdtype */
+} moe_dtypes;
+
+typedef enum { MOE_ACT_SWIGLU = 0, MOE_ACT_SWIGLU_OAI = 1 } moe_act_kind;
+
+/* Activation parameters (DeepGEMM PR #445, Summary).  For MOE_ACT_SWIGLU the
+ * other fields are ignored (alpha = 1, up_bias = 0, no clamp).  For
+ * MOE_ACT_SWIGLU_OAI, limit > 0 (+INFINITY = no clamp).                      */
+typedef struct {
+  int kind; /* a moe_act_kind */
+  float alpha;
+  float up_bias;
+  float limit;
+} moe_act_params;
+
+typedef struct moe_plan_s *moe_plan_t;
+
+/* Build a plan for T tokens, hidden size H, expert intermediate size I, E
+ * experts and top-k.  Host only; enqueues nothing and allocates no device
+ * memory.  Requirements: T >= 1; H % 128 == 0; I % 128 == 0; 1 <= k <= E <= 256;
+ * T*k < 2^31.  Returns MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED otherwise.  */
+moe_status moe_plan(int T, int H, int I, int E, int k, moe_dtypes dtypes,
+                    moe_act_params act, moe_plan_t *out);
+
+/* Release a plan (NULL is allowed). */
+void moe_plan_destroy(moe_plan_t plan);
+
+/* Size in bytes of the device workspace moe_forward and the step calls need
+ * (256-byte aligned pointer required).  0 for a NULL plan.                   */
+size_t moe_workspace_bytes(moe_plan_t plan);
+
+/* The whole layer: route -> gather -> FC1 (+ activation + FP8 requant) -> FC2
+ * -> combine, enqueued on `stream`.
+ *   x          u8 [T,H]      E4M3 codes of the activations
+ *   x_scales   u8 [T,H/128]  UE8M0 scale bytes
+ *   topk_idx   i32 [T,k]     expert ids
+ *   topk_w     f32 [T,k]     combine weights
+ *   w1, w1_scales, w2, w2_scales   weights in the plan's moe_wdtype layout
+ *   out        bf16 [T,H]    written entirely
+ *   workspace  moe_workspace_bytes(plan) bytes, device, 256-B aligned.
+ * All pointers are device pointers.                                          */
+moe_status moe_forward(moe_plan_t plan, const void *x, const uint8_t *x_scales,
+                       const int32_t *topk_idx, const float *topk_w,
+                       const void *w1, const uint8_t *w1_scales, const void *w2,
+                       const uint8_t *w2_scales, void *out, void *workspace,
+                       moe_stream_t stream);
+
+/* moe_forward with the per-step activations on the HOST: x, x_scales,
+ * topk_idx and topk_w are host pointers (pinned memory gives asynchronous
+ * copies), the weights and the workspace are device pointers, and out_host is
+ * a host bf16 [T,H] buffer.  The host-to-device copies, the layer and the
+ * device-to-host copy of the output are enqueued on `stream`; the output is
+ * valid after the stream has been synchronised.                             */
+moe_status moe_forward_hostio(moe_plan_t plan, const void *x_host,
+                              const uint8_t *x_scales_host,
+                              const int32_t *topk_idx_host,
+                              const float *topk_w_host, const void *w1,
+                              const uint8_t *w1_scales, const void *w2,
+                              const uint8_t *w2_scales, void *out_host,
+                              void *workspace, moe_stream_t stream);
+
+/* ---- The steps of moe_forward, callable one by one (same workspace). ---- */
+
+/* Step 1, routing: per-expert histogram, exclusive scan and stable scatter of
+ * the T*k slots (slot s = t*k + j).  Results live in the workspace and are
+ * exposed by moe_workspace_view(): counts i32[E], offsets i32[E+1], perm i32[S]
+ * (position -> slot, ascending slot order within an expert, -1 past the
+ * routed slots) and inv i32[S] (slot -> position, -1 for an unrouted slot).
+ * Sources: DeepGEMM PR #386 Description (tokens grouped per expert).        */
+moe_status moe_route(moe_plan_t plan, const int32_t *topk_idx, void *workspace,
+                     moe_stream_t stream);
+
+/* Step 2, gather: copies the x rows (and their scale bytes) of every routed
+ * slot into expert order inside the workspace, each expert's block starting
+ * at a multiple of 128 rows.  Needs moe_route() first.                      */
+moe_status moe_gather(moe_plan_t plan, const void *x, const uint8_t *x_scales,
+                      void *workspace, moe_stream_t stream);
+
+/* Step 3, FC1: the FC1 grouped GEMM on the 5th-generation tensor cores with
+ * the block scales applied in hardware, the fused (OAI-)SwiGLU, and the FP8
+ * E4M3 + UE8M0 1x128 requantisation of the activation, all in one kernel.
+ * Needs moe_gather() first.                                                 */
+moe_status moe_fc1(moe_plan_t plan, const void *w1, const uint8_t *w1_scales,
+                   void *workspace, moe_stream_t stream);
+
+/* Step 4, FC2: grouped GEMM of the requantised activation with W2; bf16 rows
+ * written in slot order (y[s], s = t*k + j).  Needs moe_fc1() first.         */
+moe_status moe_fc2(moe_plan_t plan, const void *w2, const uint8_t *w2_scales,
+                   void *workspace, moe_stream_t stream);
+
+/* Step 5, combine: out[t] = bf16(sum_j topk_w[t,j] * y[t*k+j]) in fp32, j
+ * ascending; unrouted slots are skipped.  Needs moe_fc2() first.
+ * Sources: DeepGEMM PR #386 title ("direct combine").                        */
+moe_status moe_combine(moe_plan_t plan, const float *topk_w, void *out,
+                       void *workspace, moe_stream_t stream);
+
+/* Device pointers (inside `workspace`) of the intermediate results, for
+ * inspection.  Rows of act / act_f32 are in expert order with every expert's
+ * block starting at a multiple of 128 rows: expert e's rows are
+ * pad_offsets[e] .. pad_offsets[e]+counts[e]-1.                              */
+typedef struct {
+  int32_t *counts;      /* [E]                                        */
+  int32_t *offsets;     /* [E+1]                                      */
+  int32_t *perm;        /* [S]                                        */
+  int32_t *inv;         /* [S]                                        */
+  int32_t *pad_offsets; /* [E+1]  row offsets, multiples of 128       */
+  uint8_t *act;         /* [rows, I]  FP8 E4M3 activation (FC1 output) */
+  float *act_f32;       /* [rows, I]  the activation before requant,
+                           written only when debug capture is on      */
+  uint16_t *y;          /* [S, H] bf16, slot order (FC2 output)       */
+  uint32_t *error_word; /* bit set = moe_status code seen on device   */
+  int64_t rows;         /* capacity of the padded row space           */
+} moe_workspace_view_t;
+
+moe_status moe_workspace_view(moe_plan_t plan, void *workspace,
+                              moe_workspace_view_t *view);
+
+/* FP8 scale bytes of the activation (FC1 output) for padded row r and block
+ * b = column / 128 are stored inside the workspace in the layout the FC2
+ * tensor cores read; this copies them out as a plain u8 [rows, I/128] array
+ * (device pointer `dst`), enqueued on `stream`.                              */
+moe_status moe_copy_act_scales(moe_plan_t plan, const void *workspace,
+                               uint8_t *dst, moe_stream_t stream);
+
+/* Debug capture: when on, moe_fc1 also writes the fp32 activation before
+ * requantisation to act_f32 (costs bandwidth; off by default).              */
+moe_status moe_plan_set_debug(moe_plan_t plan, int capture_act_f32);
+
+/* Zero the workspace's device error word (enqueued on `stream`). */
+moe_status moe_clear_device_error(moe_plan_t plan, void *workspace,
+                                  moe_stream_t stream);
+
+/* Synchronises `stream`, reads the device error word and returns MOE_OK or
+ * the most severe recorded status (timeout before bad routing).            */
+moe_status moe_check_device_error(moe_plan_t plan, const void *workspace,
+                                  moe_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char *moe_status_str(moe_status status);
+
+/* Kernel launches one moe_forward enqueues for this plan. */
+int moe_forward_launch_count(moe_plan_t plan);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

@@ -1,0 +1,243 @@
+"""Python binding of the B200 fused MoE expert layer (libmoe_b200.so).
+
+Argument marshalling only: every step of the layer runs in the CUDA library.
+The functions carry the C ABI's names (include/moe.h) and accept either
+integers (raw device/host addresses) or torch tensors (their data_ptr() is
+passed).  Errors come back as MoEError carrying the moe_status code.
+
+If the compiled library is missing this module raises ImportError when a
+function is first called: there is no fallback implementation.
+"""
+import ctypes
+import math
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+MOE_OK = 0
+STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
+                3: "MOE_ERR_ALIGNMENT", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_TIMEOUT",
+                6: "MOE_ERR_BAD_ROUTING"}
+W_DTYPES = {"e4m3": 0, "e2m1": 1}
+ACT_KINDS = {"swiglu": 0, "swiglu_oai": 1}
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status, what=""):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+
+
+class _Dtypes(ctypes.Structure):
+    _fields_ = [("w_dtype", ctypes.c_int)]
+
+
+class _Act(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int), ("alpha", ctypes.c_float),
+                ("up_bias", ctypes.c_float), ("limit", ctypes.c_float)]
+
+
+class WorkspaceView(ctypes.Structure):
+    _fields_ = [("counts", ctypes.c_void_p), ("offsets", ctypes.c_void_p),
+                ("perm", ctypes.c_void_p), ("inv", ctypes.c_void_p),
+                ("pad_offsets", ctypes.c_void_p), ("act", ctypes.c_void_p),
+                ("act_f32", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("error_word", ctypes.c_void_p), ("rows", ctypes.c_int64)]
+
+
+_P = ctypes.c_void_p
+_SIGS = {
+    "moe_plan": (ctypes.c_int, [ctypes.c_int] * 5 + [_Dtypes, _Act, ctypes.POINTER(_P)]),
+    "moe_plan_destroy": (None, [_P]),
+    "moe_workspace_bytes": (ctypes.c_size_t, [_P]),
+    "moe_forward": (ctypes.c_int, [_P] * 12),
+    "moe_forward_hostio": (ctypes.c_int, [_P] * 12),
+    "moe_route": (ctypes.c_int, [_P] * 4),
+    "moe_gather": (ctypes.c_int, [_P] * 5),
+    "moe_fc1": (ctypes.c_int, [_P] * 5),
+    "moe_fc2": (ctypes.c_int, [_P] * 5),
+    "moe_combine": (ctypes.c_int, [_P] * 5),
+    "moe_workspace_view": (ctypes.c_int, [_P, _P, ctypes.POINTER(WorkspaceView)]),
+    "moe_copy_act_scales": (ctypes.c_int, [_P] * 4),
+    "moe_plan_set_debug": (ctypes.c_int, [_P, ctypes.c_int]),
+    "moe_clear_device_error": (ctypes.c_int, [_P] * 3),
+    "moe_check_device_error": (ctypes.c_int, [_P] * 3),
+    "moe_status_str": (ctypes.c_char_p, [ctypes.c_int]),
+    "moe_forward_launch_count": (ctypes.c_int, [_P]),
+}
+
+_lib = None
+
+
+def lib():
+    """The loaded CUDA library (ImportError if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m moe_expert_ffn_permute_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _ptr(v):
+    if v is None:
+        return None
+    if isinstance(v, int):
+        return v
+    if hasattr(v, "data_ptr"):
+        return v.data_ptr()
+    raise TypeError(f"expected an address or a tensor, got {type(v)}")
+
+
+def _stream(s):
+    if s is None:
+        try:
+            import torch
+            if torch.cuda.is_available():
+                return torch.cuda.current_stream().cuda_stream
+        except ImportError:  # pragma: no cover
+            pass
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(status, what):
+    if status != MOE_OK:
+        raise MoEError(status, what)
+
+
+def moe_plan(T, H, I, E, k, w_dtype="e4m3", act="swiglu", alpha=1.0, up_bias=0.0,
+             limit=math.inf):
+    """Build a plan (host object).  Returns an opaque handle."""
+    h = _P()
+    st = lib().moe_plan(T, H, I, E, k, _Dtypes(W_DTYPES[w_dtype]),
+                        _Act(ACT_KINDS[act], alpha, up_bias, limit), ctypes.byref(h))
+    _check(st, "moe_plan")
+    return h.value
+
+
+def moe_plan_destroy(plan):
+    lib().moe_plan_destroy(plan)
+
+
+def moe_workspace_bytes(plan):
+    return lib().moe_workspace_bytes(plan)
+
+
+def moe_plan_set_debug(plan, capture_act_f32):
+    _check(lib().moe_plan_set_debug(plan, int(bool(capture_act_f32))), "moe_plan_set_debug")
+
+
+def moe_forward(plan, x, x_scales, topk_idx, topk_w, w1, w1_scales, w2, w2_scales, out,
+                workspace, stream=None):
+    _check(lib().moe_forward(plan, *map(_ptr, (x, x_scales, topk_idx, topk_w, w1, w1_scales,
+                                               w2, w2_scales, out, workspace)),
+                             _stream(stream)), "moe_forward")
+
+
+def moe_forward_hostio(plan, x_host, x_scales_host, topk_idx_host, topk_w_host, w1, w1_scales,
+                       w2, w2_scales, out_host, workspace, stream=None):
+    _check(lib().moe_forward_hostio(plan, *map(_ptr, (x_host, x_scales_host, topk_idx_host,
+                                                      topk_w_host, w1, w1_scales, w2, w2_scales,
+                                                      out_host, workspace)),
+                                    _stream(stream)), "moe_forward_hostio")
+
+
+def moe_route(plan, topk_idx, workspace, stream=None):
+    _check(lib().moe_route(plan, _ptr(topk_idx), _ptr(workspace), _stream(stream)), "moe_route")
+
+
+def moe_gather(plan, x, x_scales, workspace, stream=None):
+    _check(lib().moe_gather(plan, *map(_ptr, (x, x_scales, workspace)), _stream(stream)),
+           "moe_gather")
+
+
+def moe_fc1(plan, w1, w1_scales, workspace, stream=None):
+    _check(lib().moe_fc1(plan, *map(_ptr, (w1, w1_scales, workspace)), _stream(stream)),
+           "moe_fc1")
+
+
+def moe_fc2(plan, w2, w2_scales, workspace, stream=None):
+    _check(lib().moe_fc2(plan, *map(_ptr, (w2, w2_scales, workspace)), _stream(stream)),
+           "moe_fc2")
+
+
+def moe_combine(plan, topk_w, out, workspace, stream=None):
+    _check(lib().moe_combine(plan, *map(_ptr, (topk_w, out, workspace)), _stream(stream)),
+           "moe_combine")
+
+
+def moe_workspace_view(plan, workspace):
+    v = WorkspaceView()
+    _check(lib().moe_workspace_view(plan, _ptr(workspace), ctypes.byref(v)), "moe_workspace_view")
+    return v
+
+
+def moe_copy_act_scales(plan, workspace, dst, stream=None):
+    _check(lib().moe_copy_act_scales(plan, _ptr(workspace), _ptr(dst), _stream(stream)),
+           "moe_copy_act_scales")
+
+
+def moe_clear_device_error(plan, workspace, stream=None):
+    _check(lib().moe_clear_device_error(plan, _ptr(workspace), _stream(stream)),
+           "moe_clear_device_error")
+
+
+def moe_check_device_error(plan, workspace, stream=None):
+    """Synchronises the stream; returns the moe_status code (0 = no device error)."""
+    return lib().moe_check_device_error(plan, _ptr(workspace), _stream(stream))
+
+
+def moe_status_str(status):
+    return lib().moe_status_str(status).decode()
+
+
+def moe_forward_launch_count(plan):
+    return lib().moe_forward_launch_count(plan)
+
+
+class MoELayer:
+    """Convenience owner of a plan and its torch-allocated workspace."""
+
+    def __init__(self, T, H, I, E, k, w_dtype="e4m3", act="swiglu", alpha=1.0, up_bias=0.0,
+                 limit=math.inf, device="cuda", debug=False):
+        import torch
+        self.T, self.H, self.I, self.E, self.k = T, H, I, E, k
+        self.plan = moe_plan(T, H, I, E, k, w_dtype, act, alpha, up_bias, limit)
+        if debug:
+            moe_plan_set_debug(self.plan, True)
+        nbytes = moe_workspace_bytes(self.plan)
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        moe_clear_device_error(self.plan, self.workspace)
+
+    def forward(self, x, x_scales, topk_idx, topk_w, w1, w1_scales, w2, w2_scales, out=None,
+                stream=None):
+        import torch
+        if out is None:
+            out = torch.empty(self.T, self.H, dtype=torch.bfloat16, device=self.workspace.device)
+        moe_forward(self.plan, x, x_scales, topk_idx, topk_w, w1, w1_scales, w2, w2_scales, out,
+                    self.workspace, stream)
+        return out
+
+    def view(self):
+        return moe_workspace_view(self.plan, self.workspace)
+
+    def check(self, stream=None):
+        return moe_check_device_error(self.plan, self.workspace, stream)
+
+    def __del__(self):
+        try:
+            if getattr(self, "plan", None):
+                moe_plan_destroy(self.plan)
+                self.plan = None
+        except Exception:
+            pass

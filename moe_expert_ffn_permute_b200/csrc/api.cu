@@ -1,0 +1,296 @@
+// api.cu -- the C ABI (include/moe.h): plan construction and validation,
+// workspace layout, and the stream-ordered launch sequence of the layer.
+#include <cmath>
+#include <cstring>
+#include <new>
+
+#include "internal.h"
+
+namespace moe {
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+void compute_layout(moe_plan_s* p) {
+  WorkspaceLayout& L = p->ws;
+  const size_t S = static_cast<size_t>(p->S);
+  const size_t E = static_cast<size_t>(p->E);
+  const size_t rows = static_cast<size_t>(p->rows_cap);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  L.err = take(256);
+  L.counts = take(E * 4);
+  L.offsets = take((E + 1) * 4);
+  L.pad_off = take((E + 1) * 4);
+  L.tile_off = take((E + 1) * 4);
+  L.block_hist = take(static_cast<size_t>(p->route_blocks) * E * 4);
+  L.perm = take(S * 4);
+  L.inv = take(S * 4);
+  L.xg = take(rows * p->H);
+  L.xg_sf = take(rows / kTileM * (p->H / 128) * 512);
+  L.act = take(rows * p->I);
+  L.act_sf = take(rows / kTileM * (p->I / 128) * 512);
+  L.act_f32 = take(p->debug_act_f32 ? rows * p->I * 4 : 0);
+  L.y = take(S * p->H * 2);
+  L.in_x = take(static_cast<size_t>(p->T) * p->H);
+  L.in_xs = take(static_cast<size_t>(p->T) * (p->H / 128));
+  L.in_idx = take(S * 4);
+  L.in_w = take(S * 4);
+  L.out_stage = take(static_cast<size_t>(p->T) * p->H * 2);
+  L.total = off;
+}
+
+}  // namespace moe
+
+using moe::kTileM;
+
+static bool aligned(const void* p, size_t a) {
+  return p != nullptr && (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+static moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+extern "C" {
+
+moe_status moe_plan(int T, int H, int I, int E, int k, moe_dtypes dtypes, moe_act_params act,
+                    moe_plan_t* out) {
+  if (out == nullptr) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (T < 1 || H < 1 || I < 1 || k < 1 || E < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (E > 256) return MOE_ERR_UNSUPPORTED;
+  if (H % 128 != 0 || I % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (H % 256 != 0) return MOE_ERR_UNSUPPORTED;   // FC2 tiles are 256 columns wide
+  if (static_cast<long long>(T) * k >= (1ll << 31)) return MOE_ERR_INVALID_ARG;
+  if (dtypes.w_dtype != MOE_W_E4M3_UE8M0_128x128 && dtypes.w_dtype != MOE_W_E2M1_UE8M0_1x32)
+    return MOE_ERR_INVALID_ARG;
+  if (act.kind != MOE_ACT_SWIGLU && act.kind != MOE_ACT_SWIGLU_OAI) return MOE_ERR_INVALID_ARG;
+  if (act.kind == MOE_ACT_SWIGLU_OAI) {
+    if (!(act.limit > 0.0f) || std::isnan(act.alpha) || std::isnan(act.up_bias) ||
+        std::isinf(act.alpha) || std::isinf(act.up_bias))
+      return MOE_ERR_INVALID_ARG;
+  } else {
+    act.alpha = 1.0f;
+    act.up_bias = 0.0f;
+    act.limit = INFINITY;
+  }
+  moe_plan_s* p = new (std::nothrow) moe_plan_s();
+  if (p == nullptr) return MOE_ERR_INVALID_ARG;
+  p->T = T;
+  p->H = H;
+  p->I = I;
+  p->E = E;
+  p->k = k;
+  p->w_dtype = dtypes.w_dtype;
+  p->act = act;
+  p->debug_act_f32 = 0;
+  p->S = static_cast<long long>(T) * k;
+  // Sum over experts of ceil(n_e / 128) <= floor((S + 127 E) / 128).
+  p->rows_cap = ((p->S + 127ll * E) / kTileM) * kTileM;
+  if (p->rows_cap < kTileM) p->rows_cap = kTileM;
+  p->route_blocks = static_cast<int>((p->S + moe::kRouteChunk - 1) / moe::kRouteChunk);
+  moe::compute_layout(p);
+  *out = p;
+  return MOE_OK;
+}
+
+void moe_plan_destroy(moe_plan_t plan) { delete plan; }
+
+size_t moe_workspace_bytes(moe_plan_t plan) { return plan ? plan->ws.total : 0; }
+
+moe_status moe_plan_set_debug(moe_plan_t plan, int capture_act_f32) {
+  if (plan == nullptr) return MOE_ERR_INVALID_ARG;
+  plan->debug_act_f32 = capture_act_f32 ? 1 : 0;
+  moe::compute_layout(plan);
+  return MOE_OK;
+}
+
+int moe_forward_launch_count(moe_plan_t plan) {
+  (void)plan;
+  return 6;   // route histogram, route scatter, gather, FC1, FC2, combine
+}
+
+static moe_status check_ws(moe_plan_t plan, const void* workspace) {
+  if (plan == nullptr) return MOE_ERR_INVALID_ARG;
+  if (workspace == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256)) return MOE_ERR_ALIGNMENT;
+  return MOE_OK;
+}
+
+static moe_status check_weights(moe_plan_t plan, const void* w, const uint8_t* ws) {
+  if (w == nullptr || ws == nullptr) return MOE_ERR_INVALID_ARG;
+  const size_t wa = plan->w_dtype == MOE_W_E2M1_UE8M0_1x32 ? 32 : 16;
+  if (!aligned(w, wa)) return MOE_ERR_ALIGNMENT;
+  if (plan->w_dtype == MOE_W_E2M1_UE8M0_1x32 && !aligned(ws, 4)) return MOE_ERR_ALIGNMENT;
+  return MOE_OK;
+}
+
+moe_status moe_route(moe_plan_t plan, const int32_t* topk_idx, void* workspace,
+                     moe_stream_t stream) {
+  moe_status s = check_ws(plan, workspace);
+  if (s != MOE_OK) return s;
+  if (topk_idx == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned(topk_idx, 4)) return MOE_ERR_ALIGNMENT;
+  return cuda_status(moe::launch_route(plan, topk_idx, static_cast<uint8_t*>(workspace),
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_gather(moe_plan_t plan, const void* x, const uint8_t* x_scales, void* workspace,
+                      moe_stream_t stream) {
+  moe_status s = check_ws(plan, workspace);
+  if (s != MOE_OK) return s;
+  if (x == nullptr || x_scales == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16)) return MOE_ERR_ALIGNMENT;
+  return cuda_status(moe::launch_gather(plan, static_cast<const uint8_t*>(x), x_scales,
+                                        static_cast<uint8_t*>(workspace),
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_fc1(moe_plan_t plan, const void* w1, const uint8_t* w1_scales, void* workspace,
+                   moe_stream_t stream) {
+  moe_status s = check_ws(plan, workspace);
+  if (s != MOE_OK) return s;
+  if ((s = check_weights(plan, w1, w1_scales)) != MOE_OK) return s;
+  return cuda_status(moe::launch_fc1(plan, w1, w1_scales, static_cast<uint8_t*>(workspace),
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_fc2(moe_plan_t plan, const void* w2, const uint8_t* w2_scales, void* workspace,
+                   moe_stream_t stream) {
+  moe_status s = check_ws(plan, workspace);
+  if (s != MOE_OK) return s;
+  if ((s = check_weights(plan, w2, w2_scales)) != MOE_OK) return s;
+  return cuda_status(moe::launch_fc2(plan, w2, w2_scales, static_cast<uint8_t*>(workspace),
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_combine(moe_plan_t plan, const float* topk_w, void* out, void* workspace,
+                       moe_stream_t stream) {
+  moe_status s = check_ws(plan, workspace);
+  if (s != MOE_OK) return s;
+  if (topk_w == nullptr || out == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned(topk_w, 4) || !aligned(out, 16)) return MOE_ERR_ALIGNMENT;
+  return cuda_status(moe::launch_combine(plan, topk_w, out, static_cast<uint8_t*>(workspace),
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_forward(moe_plan_t plan, const void* x, const uint8_t* x_scales,
+                       const int32_t* topk_idx, const float* topk_w, const void* w1,
+                       const uint8_t* w1_scales, const void* w2, const uint8_t* w2_scales,
+                       void* out, void* workspace, moe_stream_t stream) {
+  // Validate everything before the first launch.
+  moe_status s = check_ws(plan, workspace);
+  if (s != MOE_OK) return s;
+  if (x == nullptr || x_scales == nullptr || topk_idx == nullptr || topk_w == nullptr ||
+      out == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(topk_idx, 4) || !aligned(topk_w, 4) || !aligned(out, 16))
+    return MOE_ERR_ALIGNMENT;
+  if ((s = check_weights(plan, w1, w1_scales)) != MOE_OK) return s;
+  if ((s = check_weights(plan, w2, w2_scales)) != MOE_OK) return s;
+  if ((s = moe_route(plan, topk_idx, workspace, stream)) != MOE_OK) return s;
+  if ((s = moe_gather(plan, x, x_scales, workspace, stream)) != MOE_OK) return s;
+  if ((s = moe_fc1(plan, w1, w1_scales, workspace, stream)) != MOE_OK) return s;
+  if ((s = moe_fc2(plan, w2, w2_scales, workspace, stream)) != MOE_OK) return s;
+  return moe_combine(plan, topk_w, out, workspace, stream);
+}
+
+moe_status moe_forward_hostio(moe_plan_t plan, const void* x_host, const uint8_t* x_scales_host,
+                              const int32_t* topk_idx_host, const float* topk_w_host,
+                              const void* w1, const uint8_t* w1_scales, const void* w2,
+                              const uint8_t* w2_scales, void* out_host, void* workspace,
+                              moe_stream_t stream) {
+  moe_status s = check_ws(plan, workspace);
+  if (s != MOE_OK) return s;
+  if (x_host == nullptr || x_scales_host == nullptr || topk_idx_host == nullptr ||
+      topk_w_host == nullptr || out_host == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if ((s = check_weights(plan, w1, w1_scales)) != MOE_OK) return s;
+  if ((s = check_weights(plan, w2, w2_scales)) != MOE_OK) return s;
+  auto ws = static_cast<uint8_t*>(workspace);
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  const auto& L = plan->ws;
+  const size_t T = plan->T, H = plan->H, S = static_cast<size_t>(plan->S);
+  if (cudaMemcpyAsync(ws + L.in_x, x_host, T * H, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(ws + L.in_xs, x_scales_host, T * (H / 128), cudaMemcpyHostToDevice, st) !=
+          cudaSuccess ||
+      cudaMemcpyAsync(ws + L.in_idx, topk_idx_host, S * 4, cudaMemcpyHostToDevice, st) !=
+          cudaSuccess ||
+      cudaMemcpyAsync(ws + L.in_w, topk_w_host, S * 4, cudaMemcpyHostToDevice, st) !=
+          cudaSuccess)
+    return MOE_ERR_CUDA;
+  uint8_t* out_dev = ws + L.out_stage;
+  s = moe_forward(plan, ws + L.in_x, ws + L.in_xs, reinterpret_cast<const int32_t*>(ws + L.in_idx),
+                  reinterpret_cast<const float*>(ws + L.in_w), w1, w1_scales, w2, w2_scales,
+                  out_dev, workspace, stream);
+  if (s != MOE_OK) return s;
+  if (cudaMemcpyAsync(out_host, out_dev, T * H * 2, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status moe_workspace_view(moe_plan_t plan, void* workspace, moe_workspace_view_t* v) {
+  moe_status s = check_ws(plan, workspace);
+  if (s != MOE_OK) return s;
+  if (v == nullptr) return MOE_ERR_INVALID_ARG;
+  auto ws = static_cast<uint8_t*>(workspace);
+  const auto& L = plan->ws;
+  v->counts = reinterpret_cast<int32_t*>(ws + L.counts);
+  v->offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+  v->perm = reinterpret_cast<int32_t*>(ws + L.perm);
+  v->inv = reinterpret_cast<int32_t*>(ws + L.inv);
+  v->pad_offsets = reinterpret_cast<int32_t*>(ws + L.pad_off);
+  v->act = ws + L.act;
+  v->act_f32 = plan->debug_act_f32 ? reinterpret_cast<float*>(ws + L.act_f32) : nullptr;
+  v->y = reinterpret_cast<uint16_t*>(ws + L.y);
+  v->error_word = reinterpret_cast<uint32_t*>(ws + L.err);
+  v->rows = plan->rows_cap;
+  return MOE_OK;
+}
+
+moe_status moe_copy_act_scales(moe_plan_t plan, const void* workspace, uint8_t* dst,
+                               moe_stream_t stream) {
+  moe_status s = check_ws(plan, workspace);
+  if (s != MOE_OK) return s;
+  if (dst == nullptr) return MOE_ERR_INVALID_ARG;
+  return cuda_status(moe::launch_unpack_act_scales(plan, static_cast<const uint8_t*>(workspace),
+                                                   dst, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_clear_device_error(moe_plan_t plan, void* workspace, moe_stream_t stream) {
+  moe_status s = check_ws(plan, workspace);
+  if (s != MOE_OK) return s;
+  return cuda_status(cudaMemsetAsync(static_cast<uint8_t*>(workspace) + plan->ws.err, 0, 4,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_check_device_error(moe_plan_t plan, const void* workspace, moe_stream_t stream) {
+  moe_status s = check_ws(plan, workspace);
+  if (s != MOE_OK) return s;
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, static_cast<const uint8_t*>(workspace) + plan->ws.err, 4,
+                      cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (word & (1u << MOE_ERR_DEVICE_TIMEOUT)) return MOE_ERR_DEVICE_TIMEOUT;
+  if (word & (1u << MOE_ERR_BAD_ROUTING)) return MOE_ERR_BAD_ROUTING;
+  return MOE_OK;
+}
+
+const char* moe_status_str(moe_status status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_ALIGNMENT: return "MOE_ERR_ALIGNMENT";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
+    case MOE_ERR_BAD_ROUTING: return "MOE_ERR_BAD_ROUTING";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+}  // extern "C"

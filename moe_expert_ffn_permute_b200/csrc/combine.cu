@@ -1,0 +1,64 @@
+// combine.cu -- step 4, the direct weighted top-k combine back to token order
+// (DeepGEMM PR #386 "Optimize sm100 version with token-aware BM240 tiling,
+// native UE8M0, and direct combine", title):
+//   out[t, c] = bf16( sum_{j=0}^{k-1} topk_w[t, j] * y[t*k + j, c] )
+// summed in fp32 with j ascending (deterministic).  A slot whose expert id was
+// out of range (inv[s] < 0) contributes nothing.  HBM-bound: each thread reads
+// k 16-byte vectors of y and writes one 16-byte vector of out.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ y,
+                                                      const float* __restrict__ topk_w,
+                                                      const int32_t* __restrict__ inv, int T,
+                                                      int H, int k, uint16_t* __restrict__ out) {
+  const int vecs = H / 8;
+  const long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+  if (i >= static_cast<long long>(T) * vecs) return;
+  const int t = static_cast<int>(i / vecs);
+  const int c = static_cast<int>(i - static_cast<long long>(t) * vecs);
+  float acc[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
+  for (int j = 0; j < k; ++j) {
+    const long long s = static_cast<long long>(t) * k + j;
+    if (__ldg(&inv[s]) < 0) continue;
+    const float w = __ldg(&topk_w[s]);
+    const uint4 v = __ldcs(reinterpret_cast<const uint4*>(y + s * H) + c);
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float lo = __uint_as_float(wv[q] << 16);
+      const float hi = __uint_as_float(wv[q] & 0xFFFF0000u);
+      acc[2 * q] = fmaf(w, lo, acc[2 * q]);
+      acc[2 * q + 1] = fmaf(w, hi, acc[2 * q + 1]);
+    }
+  }
+  uint32_t o[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+    o[q] = *reinterpret_cast<uint32_t*>(&b);
+  }
+  reinterpret_cast<uint4*>(out + static_cast<long long>(t) * H)[c] =
+      make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const moe_plan_s* p, const float* topk_w, void* out, uint8_t* ws,
+                           cudaStream_t st) {
+  const long long n = static_cast<long long>(p->T) * (p->H / 8);
+  const int blocks = static_cast<int>((n + 255) / 256);
+  combine_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const uint16_t*>(ws + p->ws.y), topk_w,
+                                         reinterpret_cast<const int32_t*>(ws + p->ws.inv), p->T,
+                                         p->H, p->k, reinterpret_cast<uint16_t*>(out));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,555 @@
+// gemm.cu -- FC1 and FC2 grouped GEMMs on the 5th-generation tensor cores.
+//
+// One persistent CTA per SM computes 128 x 256 output tiles of one expert:
+//   FC1: A = gathered x rows [128 x H] (E4M3), B = 128 gate rows + 128 up rows of
+//        W1[e] (E4M3 or E2M1), D = fp32 [128 x 256] in tensor memory; the
+//        epilogue applies the (OAI-)SwiGLU and requantises the 128-wide
+//        activation block to E4M3 + one UE8M0 scale per row.
+//   FC2: A = FP8 activation rows [128 x I], B = 256 rows of W2[e]; the epilogue
+//        writes bf16 rows to their slot (t*k + j) for the combine.
+// Block scales (1x128 for activations, 128x128 or 1x32 for weights, all UE8M0)
+// are applied by the MMA itself (tcgen05.mma.kind::mxf8f6f4.block_scale, one
+// scale per 32-wide K sub-block; the coarser blocks are replicated).
+//
+// Warp roles (12 warps):
+//   warp 0   producer: TMA loads of A/B tiles, scale chunks (bulk copy / cp.async)
+//   warp 1   MMA issuer; owns the tensor-memory allocation
+//   warp 2   tile scheduler: writes task infos into a ring of shared-memory slots
+//   warp 3   idle
+//   warps 4-11 epilogue: two warps per 32-lane TMEM sub-partition
+//
+// Scheduler slot release (fw-ai/DeepGEMM PR #16 "Sync upstream through PR #441:
+// fix Mega MoE scheduler ordering", Overview): a consumer copies the task info
+// out of its slot, then executes fence.acq_rel.cta, and only then arrives on the
+// slot's empty barrier, so the scheduler can never overwrite metadata that is
+// still being read.
+//
+// Activation (DeepGEMM PR #445 "fix(sm90): support parameterized SwiGLU in FP8
+// MegaMoE", Summary): gate = min(gate, limit), up = clamp(up, -limit, limit),
+// a = gate * sigmoid(alpha * gate) * (up + up_bias).
+// Requantisation (TensorRT-LLM PR #16346 "DSV4 o_proj: fuse fp8/UE8M0 quantize
+// ...", Description): per 1x128 block, amax -> UE8M0 exponent -> E4M3 codes,
+// done in the producing GEMM's epilogue.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 128, STAGES = 4, SCHED_DEPTH = 4;
+constexpr int kThreads = 384;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccCol = 0, kSfaCol = 256, kSfbCol = 264;
+constexpr int kEpiWarps = 8;
+constexpr int kSchedConsumers = 2 + kEpiWarps;   // producer, MMA, epilogue warps
+
+struct __align__(1024) Smem {
+  uint8_t a[STAGES][BM * BK];
+  uint8_t b[STAGES][BN * BK];
+  uint8_t sfa[STAGES][512];
+  uint8_t sfb[STAGES][1024];
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tmem_full;
+  uint64_t tmem_empty;
+  uint64_t sched_full[SCHED_DEPTH];
+  uint64_t sched_empty[SCHED_DEPTH];
+  uint64_t pair[4];
+  int4 task[SCHED_DEPTH];          // expert, m-tile (padded), n-tile, valid rows
+  int task_pos[SCHED_DEPTH];       // position (unpadded) of the tile's first row
+  float amax[2][2][BM];            // [tile parity][half][row]
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct Params {
+  int E, n_tiles, k_blocks;
+  int b_rows_per_expert;     // 2I (FC1) or H (FC2)
+  int I, H;
+  int fp4;                   // weights are E2M1 + 1x32 scales
+  int fc1;
+  const int32_t* tile_off;
+  const int32_t* counts;
+  const int32_t* offsets;
+  const int32_t* perm;
+  const uint8_t* sfa_chunks; // [m-tiles][k_blocks][512]
+  const uint8_t* w_sf;
+  // FC1 epilogue
+  uint8_t* act;
+  uint8_t* act_sf_chunks;
+  float* act_f32;
+  int oai;
+  float alpha, up_bias, limit;
+  // FC2 epilogue
+  uint16_t* y;
+  uint32_t* err;
+};
+
+struct Task {
+  int e, mt, nt, rows, pos;
+};
+
+// Consumer side of the scheduler ring: copy the task info out of the slot,
+// order those reads before the release (acquire/release fence at CTA scope),
+// then arrive on the slot's empty barrier.
+__device__ __forceinline__ bool get_task(Smem& sm, int& slot, uint32_t& phase, Task& t,
+                                         uint32_t* err) {
+  if (!mbar_wait(&sm.sched_full[slot], phase, err, &sm.abort_flag)) return false;
+  const int4 v = sm.task[slot];
+  t.e = v.x;
+  t.mt = v.y;
+  t.nt = v.z;
+  t.rows = v.w;
+  t.pos = sm.task_pos[slot];
+  __syncwarp();
+  fence_acq_rel_cta();
+  if (lane_id() == 0) mbar_arrive(&sm.sched_empty[slot]);
+  if (++slot == SCHED_DEPTH) {
+    slot = 0;
+    phase ^= 1u;
+  }
+  return true;
+}
+
+__device__ __forceinline__ float sigmoidf_fast(float z) { return __frcp_rn(1.0f + __expf(-z)); }
+
+// Smallest n with amax <= 448 * 2^n, from the fp32 bits (448 = 1.75 * 2^8):
+// amax = m * 2^e with m in [1, 2): n = e - 8 if m <= 1.75, else e - 7.
+__device__ __forceinline__ int ue8m0_exponent(float amax) {
+  amax = fmaxf(amax, 1e-4f);
+  const uint32_t bits = __float_as_uint(amax);
+  const int e = static_cast<int>((bits >> 23) & 0xFF) - 127;
+  const uint32_t man = bits & 0x7FFFFF;
+  return (man <= 0x600000u) ? e - 8 : e - 7;
+}
+
+template <bool kFc1, bool kFp4>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                        const __grid_constant__ CUtensorMap tmap_b, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&sm.full[s], 33);
+      mbar_init(&sm.empty[s], 1);
+    }
+    mbar_init(&sm.tmem_full, 1);
+    mbar_init(&sm.tmem_empty, kEpiWarps);
+    for (int r = 0; r < SCHED_DEPTH; ++r) {
+      mbar_init(&sm.sched_full[r], 1);
+      mbar_init(&sm.sched_empty[r], kSchedConsumers);
+    }
+    for (int q = 0; q < 4; ++q) mbar_init(&sm.pair[q], 2);
+    sm.abort_flag = 0;
+    fence_mbarrier_init();
+    tma_prefetch_desc(&tmap_a);
+    tma_prefetch_desc(&tmap_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 2) {
+    // ------------------------------------------------------------ scheduler
+    if (lane == 0) {
+      const int total_m = p.tile_off[p.E];
+      const int total = total_m * p.n_tiles;
+      int slot = 0;
+      uint32_t phase = 0;
+      int e = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok; tile += gridDim.x) {
+        Task t{-1, 0, 0, 0, 0};
+        if (tile < total) {
+          t.mt = tile / p.n_tiles;
+          t.nt = tile - t.mt * p.n_tiles;
+          while (p.tile_off[e + 1] <= t.mt) ++e;
+          const int local = (t.mt - p.tile_off[e]) * BM;
+          t.e = e;
+          t.rows = min(BM, p.counts[e] - local);
+          t.pos = p.offsets[e] + local;
+        }
+        ok = mbar_wait(&sm.sched_empty[slot], phase ^ 1u, p.err, &sm.abort_flag);
+        if (!ok) break;
+        sm.task[slot] = make_int4(t.e, t.mt, t.nt, t.rows);
+        sm.task_pos[slot] = t.pos;
+        mbar_arrive(&sm.sched_full[slot]);   // release: the slot's contents are visible
+        if (++slot == SCHED_DEPTH) {
+          slot = 0;
+          phase ^= 1u;
+        }
+        if (t.e < 0) break;
+      }
+    }
+  } else if (warp == 0) {
+    // ------------------------------------------------------------- producer
+    int slot = 0, stage = 0;
+    uint32_t sphase = 0, phase = 0;
+    const uint64_t pol_a = l2_policy_evict_last();
+    const uint64_t pol_b = l2_policy_evict_first();
+    const uint32_t tx_bytes = BM * BK + (kFp4 ? BN * BK / 2 : BN * BK) + 512;
+    Task t;
+    while (get_task(sm, slot, sphase, t, p.err)) {
+      if (t.e < 0) break;
+      // Rows of B for this tile: two 128-row halves.
+      int brow0, brow1;
+      if (kFc1) {
+        brow0 = t.e * p.b_rows_per_expert + t.nt * 128;          // gate rows
+        brow1 = brow0 + p.I;                                     // up rows
+      } else {
+        brow0 = t.e * p.b_rows_per_expert + t.nt * 256;
+        brow1 = brow0 + 128;
+      }
+      uint32_t sf0 = 0, sf1 = 0;   // FP8 weight scales for k-blocks kb = 32*c + lane
+      bool aborted = false;
+      for (int kb = 0; kb < p.k_blocks; ++kb) {
+        if (!kFp4 && (kb & 31) == 0) {
+          const int kq = kb + lane;
+          const int kbs = p.k_blocks;
+          if (kq < kbs) {
+            sf0 = p.w_sf[static_cast<size_t>(brow0 / 128) * kbs + kq];
+            sf1 = p.w_sf[static_cast<size_t>(brow1 / 128) * kbs + kq];
+          }
+        }
+        if (!mbar_wait(&sm.empty[stage], phase ^ 1u, p.err, &sm.abort_flag)) {
+          aborted = true;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&sm.full[stage], tx_bytes);
+          tma_load_2d(sm.a[stage], &tmap_a, kb * BK, t.mt * BM, &sm.full[stage], pol_a);
+          if (kFc1) {
+            tma_load_2d(sm.b[stage], &tmap_b, kb * BK, brow0, &sm.full[stage], pol_b);
+            tma_load_2d(sm.b[stage] + 128 * BK, &tmap_b, kb * BK, brow1, &sm.full[stage], pol_b);
+          } else {
+            tma_load_2d(sm.b[stage], &tmap_b, kb * BK, brow0, &sm.full[stage], pol_b);
+          }
+          bulk_load(sm.sfa[stage],
+                    p.sfa_chunks + (static_cast<size_t>(t.mt) * p.k_blocks + kb) * 512, 512,
+                    &sm.full[stage]);
+        }
+        if (kFp4) {
+          // One 32-bit word = the four 1x32 scales of this 128-wide k-block.
+          const int kw = p.k_blocks * 4;   // scale bytes per weight row
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const int rb = c ? brow1 : brow0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int r = lane + 32 * q;
+              cp_async_4(sm.sfb[stage] + c * 512 + lane * 16 + q * 4,
+                         p.w_sf + static_cast<size_t>(rb + r) * kw + kb * 4);
+            }
+          }
+          cp_async_mbar_arrive_noinc(&sm.full[stage]);
+        } else {
+          const uint32_t g = __shfl_sync(0xffffffffu, sf0, kb & 31) * 0x01010101u;
+          const uint32_t u = __shfl_sync(0xffffffffu, sf1, kb & 31) * 0x01010101u;
+          reinterpret_cast<uint4*>(sm.sfb[stage])[lane] = make_uint4(g, g, g, g);
+          reinterpret_cast<uint4*>(sm.sfb[stage] + 512)[lane] = make_uint4(u, u, u, u);
+          fence_proxy_async_smem();
+          mbar_arrive(&sm.full[stage]);
+        }
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (aborted) break;
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issue
+    int slot = 0, stage = 0;
+    uint32_t sphase = 0, phase = 0, acc_phase = 0;
+    Task t;
+    while (get_task(sm, slot, sphase, t, p.err)) {
+      if (t.e < 0) break;
+      if (!mbar_wait(&sm.tmem_empty, acc_phase ^ 1u, p.err, &sm.abort_flag)) break;
+      tc_fence_after();
+      bool aborted = false;
+      for (int kb = 0; kb < p.k_blocks; ++kb) {
+        if (!mbar_wait(&sm.full[stage], phase, p.err, &sm.abort_flag)) {
+          aborted = true;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          fence_proxy_async_smem();
+          tmem_cp_32x128b_warpx4(tmem + kSfaCol, sf_desc(smem_u32(sm.sfa[stage])));
+          tmem_cp_32x128b_warpx4(tmem + kSfbCol, sf_desc(smem_u32(sm.sfb[stage])));
+          tmem_cp_32x128b_warpx4(tmem + kSfbCol + 4, sf_desc(smem_u32(sm.sfb[stage] + 512)));
+          const uint32_t a_base = smem_u32(sm.a[stage]);
+          const uint32_t b_base = smem_u32(sm.b[stage]);
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint32_t idesc = mxf8f6f4_idesc(kFp4 ? 5u : 0u, BN, ks);
+            mma_mxf8f6f4(tmem + kAccCol, umma_desc_sw128(a_base + ks * 32),
+                         umma_desc_sw128(b_base + ks * 32), idesc,
+                         (tmem + kSfaCol) | (static_cast<uint32_t>(ks) << 30),
+                         (tmem + kSfbCol) | (static_cast<uint32_t>(ks) << 30),
+                         (kb > 0 || ks > 0) ? 1u : 0u);
+          }
+          tc_commit(&sm.empty[stage]);
+        }
+        __syncwarp();
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (aborted) break;
+      if (lane == 0) tc_commit(&sm.tmem_full);
+      __syncwarp();
+      acc_phase ^= 1u;
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------- epilogue
+    const int q = warp & 3;            // TMEM sub-partition (lanes 32q .. 32q+31)
+    const int half = (warp - 4) >> 2;  // which half of the tile's columns
+    const int row = q * 32 + lane;
+    const uint32_t t_row = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    int slot = 0;
+    uint32_t sphase = 0, acc_phase = 0, pair_phase = 0;
+    int tile_par = 0;
+    Task t;
+    while (get_task(sm, slot, sphase, t, p.err)) {
+      if (t.e < 0) break;
+      if (!mbar_wait(&sm.tmem_full, acc_phase, p.err, &sm.abort_flag)) break;
+      tc_fence_after();
+      if (kFc1) {
+        uint32_t g[64], u[64];
+        tmem_ld_32x32b_x32(t_row + kAccCol + half * 64, *reinterpret_cast<uint32_t(*)[32]>(g));
+        tmem_ld_32x32b_x32(t_row + kAccCol + half * 64 + 32,
+                           *reinterpret_cast<uint32_t(*)[32]>(g + 32));
+        tmem_ld_32x32b_x32(t_row + kAccCol + 128 + half * 64,
+                           *reinterpret_cast<uint32_t(*)[32]>(u));
+        tmem_ld_32x32b_x32(t_row + kAccCol + 128 + half * 64 + 32,
+                           *reinterpret_cast<uint32_t(*)[32]>(u + 32));
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.tmem_empty);
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          float gv = __uint_as_float(g[i]);
+          float uv = __uint_as_float(u[i]);
+          float a;
+          if (p.oai) {
+            gv = fminf(gv, p.limit);
+            uv = fminf(fmaxf(uv, -p.limit), p.limit);
+            a = gv * sigmoidf_fast(p.alpha * gv) * (uv + p.up_bias);
+          } else {
+            a = gv * sigmoidf_fast(gv) * uv;
+          }
+          g[i] = __float_as_uint(a);
+          amax = fmaxf(amax, fabsf(a));
+        }
+        // Combine the two halves' amax of this row (the other warp of the pair).
+        sm.amax[tile_par][half][row] = amax;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.pair[q]);
+        if (!mbar_wait(&sm.pair[q], pair_phase, p.err, &sm.abort_flag)) break;
+        pair_phase ^= 1u;
+        amax = fmaxf(amax, sm.amax[tile_par][half ^ 1][row]);
+        const int n = ue8m0_exponent(amax);
+        const float inv_scale = __uint_as_float(static_cast<uint32_t>(127 - n) << 23);
+        const size_t prow = static_cast<size_t>(t.mt) * BM + row;
+        uint4* dst = reinterpret_cast<uint4*>(p.act + prow * p.I + t.nt * 128 + half * 64);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          uint32_t w[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int i0 = v * 16 + j * 4;
+            const uint32_t lo = cvt_e4m3x2(__uint_as_float(g[i0]) * inv_scale,
+                                           __uint_as_float(g[i0 + 1]) * inv_scale);
+            const uint32_t hi = cvt_e4m3x2(__uint_as_float(g[i0 + 2]) * inv_scale,
+                                           __uint_as_float(g[i0 + 3]) * inv_scale);
+            w[j] = lo | (hi << 16);
+          }
+          dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        if (half == 0) {
+          const uint32_t sbyte = static_cast<uint32_t>(n + 127) & 0xFFu;
+          const int nb = p.I / 128;
+          uint32_t* sfd = reinterpret_cast<uint32_t*>(
+              p.act_sf_chunks + (static_cast<size_t>(t.mt) * nb + t.nt) * 512 +
+              (row & 31) * 16 + (row >> 5) * 4);
+          *sfd = sbyte * 0x01010101u;
+        }
+        if (p.act_f32 != nullptr) {
+          float4* fd = reinterpret_cast<float4*>(p.act_f32 + prow * p.I + t.nt * 128 + half * 64);
+#pragma unroll
+          for (int v = 0; v < 16; ++v)
+            fd[v] = make_float4(__uint_as_float(g[4 * v]), __uint_as_float(g[4 * v + 1]),
+                                __uint_as_float(g[4 * v + 2]), __uint_as_float(g[4 * v + 3]));
+        }
+      } else {
+        uint32_t v[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          tmem_ld_32x32b_x32(t_row + kAccCol + half * 128 + c * 32,
+                             *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c));
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.tmem_empty);
+        if (row < t.rows) {
+          const int s = p.perm[t.pos + row];
+          uint4* dst = reinterpret_cast<uint4*>(p.y + static_cast<size_t>(s) * p.H + t.nt * 256 +
+                                                half * 128);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const uint32_t w0 = pack_bf16x2(__uint_as_float(v[8 * c + 0]), __uint_as_float(v[8 * c + 1]));
+            const uint32_t w1 = pack_bf16x2(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3]));
+            const uint32_t w2 = pack_bf16x2(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5]));
+            const uint32_t w3 = pack_bf16x2(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]));
+            dst[c] = make_uint4(w0, w1, w2, w3);
+          }
+        }
+      }
+      acc_phase ^= 1u;
+      tile_par ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// --------------------------------------------------------------- host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2-D K-major tensor map: inner dimension `inner` elements, `outer` rows, box
+// 128 (K) x box_rows, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_rows, bool fp4) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r =
+      enc(m, fp4 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+          const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <bool kFc1, bool kFp4>
+cudaError_t launch_gemm(const moe_plan_s* pl, const void* w, const uint8_t* wsf, uint8_t* ws,
+                        cudaStream_t st) {
+  const auto& L = pl->ws;
+  const int K = kFc1 ? pl->H : pl->I;
+  const int brows = kFc1 ? 2 * pl->I : pl->H;
+  CUtensorMap ta, tb;
+  const uint8_t* a_base = kFc1 ? ws + L.xg : ws + L.act;
+  if (!make_map(&ta, a_base, K, pl->rows_cap, K, 128, false)) return cudaErrorInvalidValue;
+  const uint64_t b_rows_total = static_cast<uint64_t>(pl->E) * brows;
+  if (!make_map(&tb, w, K, b_rows_total, kFp4 ? K / 2 : K, kFc1 ? 128 : 256, kFp4))
+    return cudaErrorInvalidValue;
+  Params p{};
+  p.E = pl->E;
+  p.n_tiles = kFc1 ? pl->I / 128 : pl->H / 256;
+  p.k_blocks = K / 128;
+  p.b_rows_per_expert = brows;
+  p.I = pl->I;
+  p.H = pl->H;
+  p.fp4 = kFp4;
+  p.fc1 = kFc1;
+  p.tile_off = reinterpret_cast<const int32_t*>(ws + L.tile_off);
+  p.counts = reinterpret_cast<const int32_t*>(ws + L.counts);
+  p.offsets = reinterpret_cast<const int32_t*>(ws + L.offsets);
+  p.perm = reinterpret_cast<const int32_t*>(ws + L.perm);
+  p.sfa_chunks = kFc1 ? ws + L.xg_sf : ws + L.act_sf;
+  p.w_sf = wsf;
+  p.act = ws + L.act;
+  p.act_sf_chunks = ws + L.act_sf;
+  p.act_f32 = pl->debug_act_f32 ? reinterpret_cast<float*>(ws + L.act_f32) : nullptr;
+  p.oai = pl->act.kind == MOE_ACT_SWIGLU_OAI;
+  p.alpha = pl->act.alpha;
+  p.up_bias = pl->act.up_bias;
+  p.limit = pl->act.limit;
+  p.y = reinterpret_cast<uint16_t*>(ws + L.y);
+  p.err = reinterpret_cast<uint32_t*>(ws + L.err);
+  const size_t smem = sizeof(Smem) + 1024;
+  auto kern = grouped_gemm_kernel<kFc1, kFp4>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const long long max_tiles = (pl->rows_cap / BM) * p.n_tiles;
+  const int grid = static_cast<int>(std::min<long long>(num_sms(), max_tiles));
+  kern<<<grid, kThreads, smem, st>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t gemm_smem_bytes() { return sizeof(Smem) + 1024; }
+
+cudaError_t launch_fc1(const moe_plan_s* p, const void* w1, const uint8_t* w1s, uint8_t* ws,
+                       cudaStream_t st) {
+  if (p->w_dtype == MOE_W_E2M1_UE8M0_1x32) return launch_gemm<true, true>(p, w1, w1s, ws, st);
+  return launch_gemm<true, false>(p, w1, w1s, ws, st);
+}
+
+cudaError_t launch_fc2(const moe_plan_s* p, const void* w2, const uint8_t* w2s, uint8_t* ws,
+                       cudaStream_t st) {
+  if (p->w_dtype == MOE_W_E2M1_UE8M0_1x32) return launch_gemm<false, true>(p, w2, w2s, ws, st);
+  return launch_gemm<false, false>(p, w2, w2s, ws, st);
+}
+
+}  // namespace moe

@@ -1,0 +1,62 @@
+// internal.h -- plan object, workspace layout and kernel launchers shared by the
+// translation units of the MoE library (not part of the public ABI).
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr int kRouteChunk = 2048;   // slots per routing block
+constexpr int kRouteThreads = 256;
+constexpr int kTileM = 128;          // rows per m-tile (expert blocks are padded to it)
+
+// Byte offsets of every buffer inside the caller's workspace (256-B aligned).
+struct WorkspaceLayout {
+  size_t err, counts, offsets, pad_off, tile_off;
+  size_t block_hist;
+  size_t perm, inv;
+  size_t xg, xg_sf;         // gathered x (expert order, padded) + its scale chunks
+  size_t act, act_sf;       // FC1 output: FP8 activation + scale chunks
+  size_t act_f32;           // debug capture (0 bytes when off)
+  size_t y;                 // FC2 output, bf16, slot order
+  size_t in_x, in_xs, in_idx, in_w;   // staging for moe_forward_hostio inputs
+  size_t out_stage;                   // and its bf16 output
+  size_t total;
+};
+
+}  // namespace moe
+
+struct moe_plan_s {
+  int T, H, I, E, k;
+  int w_dtype;
+  moe_act_params act;
+  int debug_act_f32;
+  long long S;           // T*k
+  long long rows_cap;    // padded row capacity (multiple of 128)
+  int route_blocks;
+  moe::WorkspaceLayout ws;
+};
+
+namespace moe {
+
+void compute_layout(moe_plan_s* p);
+
+// Kernel launchers (return cudaGetLastError()).
+cudaError_t launch_route(const moe_plan_s* p, const int32_t* topk_idx, uint8_t* ws,
+                         cudaStream_t st);
+cudaError_t launch_gather(const moe_plan_s* p, const uint8_t* x, const uint8_t* xs, uint8_t* ws,
+                          cudaStream_t st);
+cudaError_t launch_fc1(const moe_plan_s* p, const void* w1, const uint8_t* w1s, uint8_t* ws,
+                       cudaStream_t st);
+cudaError_t launch_fc2(const moe_plan_s* p, const void* w2, const uint8_t* w2s, uint8_t* ws,
+                       cudaStream_t st);
+cudaError_t launch_combine(const moe_plan_s* p, const float* topk_w, void* out, uint8_t* ws,
+                           cudaStream_t st);
+cudaError_t launch_unpack_act_scales(const moe_plan_s* p, const uint8_t* ws, uint8_t* dst,
+                                     cudaStream_t st);
+
+}  // namespace moe

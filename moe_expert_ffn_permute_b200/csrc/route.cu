@@ -1,0 +1,250 @@
+// route.cu -- step 1 (routing) and the FC1 operand gather.
+//
+// Routing groups the T*k slots (slot s = t*k + j holds expert topk_idx[t, j]) by
+// expert: a per-expert histogram, an exclusive scan, and a stable scatter that
+// keeps each expert's slots in ascending slot order (DeepGEMM PR #386 "Optimize
+// sm100 version with token-aware BM240 tiling, native UE8M0, and direct
+// combine", Description: tokens are grouped per expert before the grouped
+// GEMMs).  The result is integer and deterministic: it does not depend on the
+// order in which blocks run.
+//
+// Layout produced for the GEMMs: every expert's rows start at a multiple of 128
+// (pad_off[e] = 128 * tile_off[e]), so an m-tile never straddles two experts and
+// the scale chunks can be addressed per tile.
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+namespace {
+
+// Kernel 1: per-block histograms of the block's kRouteChunk slots.
+__global__ void __launch_bounds__(kRouteThreads) route_hist_kernel(
+    const int32_t* __restrict__ idx, int S, int E, int32_t* __restrict__ block_hist,
+    uint32_t* err) {
+  __shared__ int32_t hist[256];
+  const int tid = threadIdx.x;
+  for (int e = tid; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int base = blockIdx.x * kRouteChunk;
+  bool bad = false;
+  for (int i = tid; i < kRouteChunk; i += blockDim.x) {
+    const int s = base + i;
+    if (s < S) {
+      const int e = idx[s];
+      if (e >= 0 && e < E) {
+        atomicAdd(&hist[e], 1);
+      } else {
+        bad = true;
+      }
+    }
+  }
+  if (bad) atomicOr(err, kErrRoutingBit);
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) block_hist[blockIdx.x * E + e] = hist[e];
+}
+
+// Kernel 2: scan + stable scatter.  Every block re-derives, from the block
+// histograms, the per-expert totals, the exclusive scan over experts and its
+// own starting position per expert (the histograms are small, so this costs
+// less than a separate scan launch); block 0 publishes counts / offsets and
+// the padded tile offsets.  Then the block walks its chunk in sub-chunks of
+// 256 slots: inside a warp the rank of a slot among equal experts comes from
+// __match_any_sync, across warps from per-warp counts, across sub-chunks from
+// a running count per expert.
+__global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
+    const int32_t* __restrict__ idx, int S, int E, int nblk,
+    const int32_t* __restrict__ block_hist, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ tile_off, int32_t* __restrict__ pad_off,
+    int32_t* __restrict__ perm, int32_t* __restrict__ inv, uint32_t* err) {
+  constexpr int kWarps = kRouteThreads / 32;
+  __shared__ int32_t running[256];
+  __shared__ int32_t total[256];
+  __shared__ int32_t scan[257];
+  __shared__ int32_t wcount[kWarps][256];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int e = tid; e < E; e += blockDim.x) {
+    int before = 0, all = 0;
+    for (int b = 0; b < nblk; ++b) {
+      const int c = block_hist[b * E + e];
+      if (b < static_cast<int>(blockIdx.x)) before += c;
+      all += c;
+    }
+    running[e] = before;
+    total[e] = all;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0, tacc = 0;
+    for (int e = 0; e < E; ++e) {
+      scan[e] = acc;
+      if (blockIdx.x == 0) {
+        offsets[e] = acc;
+        counts[e] = total[e];
+        tile_off[e] = tacc;
+        pad_off[e] = tacc * kTileM;
+      }
+      acc += total[e];
+      tacc += (total[e] + kTileM - 1) / kTileM;
+    }
+    scan[E] = acc;
+    if (blockIdx.x == 0) {
+      offsets[E] = acc;
+      tile_off[E] = tacc;
+      pad_off[E] = tacc * kTileM;
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) running[e] += scan[e];
+  // Positions past the routed slots (left by out-of-range ids) read -1.
+  const int routed = scan[E];
+  const int base = blockIdx.x * kRouteChunk;
+  for (int p = base + tid; p < base + kRouteChunk && p < S; p += blockDim.x)
+    if (p >= routed) perm[p] = -1;
+  for (int sub = 0; sub < kRouteChunk; sub += kRouteThreads) {
+    for (int i = tid; i < kWarps * 256; i += blockDim.x) (&wcount[0][0])[i] = 0;
+    __syncthreads();
+    const int s = base + sub + tid;
+    int e = -1;
+    if (s < S) {
+      e = idx[s];
+      if (e < 0 || e >= E) e = -1;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (e >= 0 && rank == 0) wcount[warp][e] = __popc(peers);
+    __syncthreads();
+    if (s < S) {
+      if (e >= 0) {
+        int pos = running[e] + rank;
+        for (int w = 0; w < warp; ++w) pos += wcount[w][e];
+        if (pos >= 0 && pos < S) {   // always true; guards the store
+          perm[pos] = s;
+          inv[s] = pos;
+        } else {
+          atomicOr(err, kErrRoutingBit);
+          inv[s] = -1;
+        }
+      } else {
+        inv[s] = -1;
+      }
+    }
+    __syncthreads();
+    for (int ee = tid; ee < E; ee += blockDim.x) {
+      int add = 0;
+      for (int w = 0; w < kWarps; ++w) add += wcount[w][ee];
+      running[ee] += add;
+    }
+    __syncthreads();
+    if (base + sub + kRouteThreads >= S) break;
+  }
+}
+
+// Gather: row r of padded m-tile `tile` receives x[perm[...] / k]; its scale
+// bytes are written in the tensor-core scale-chunk layout: for k-block kb the
+// 512-byte chunk holds, at byte (r % 32) * 16 + (r / 32) * 4 + j (j = 0..3), the
+// row's UE8M0 byte (replicated over the four 32-wide K sub-blocks).
+__global__ void __launch_bounds__(256) gather_kernel(
+    const uint8_t* __restrict__ x, const uint8_t* __restrict__ xs, int H, int k, int E,
+    const int32_t* __restrict__ tile_off, const int32_t* __restrict__ counts,
+    const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm,
+    uint8_t* __restrict__ xg, uint8_t* __restrict__ xg_sf) {
+  __shared__ int32_t tok[kTileM];
+  __shared__ int e_sh, rows_sh;
+  const int tile = blockIdx.x;
+  const int tid = threadIdx.x;
+  if (tile >= __ldg(&tile_off[E])) return;
+  if (tid == 0) {
+    int lo = 0, hi = E;   // last e with tile_off[e] <= tile
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (tile_off[mid] <= tile) lo = mid; else hi = mid;
+    }
+    while (lo + 1 <= E && tile_off[lo + 1] <= tile) ++lo;
+    e_sh = lo;
+    const int local = (tile - tile_off[lo]) * kTileM;
+    rows_sh = min(kTileM, counts[lo] - local);
+  }
+  __syncthreads();
+  const int e = e_sh, rows = rows_sh;
+  const int local = (tile - tile_off[e]) * kTileM;
+  for (int r = tid; r < kTileM; r += blockDim.x)
+    tok[r] = (r < rows) ? perm[offsets[e] + local + r] / k : -1;
+  __syncthreads();
+  const int kb_n = H / 128;
+  const int vec_per_row = H / 16;
+  const uint4* __restrict__ x4 = reinterpret_cast<const uint4*>(x);
+  uint4* __restrict__ g4 = reinterpret_cast<uint4*>(xg + static_cast<size_t>(tile) * kTileM * H);
+  for (int i = tid; i < rows * vec_per_row; i += blockDim.x) {
+    const int r = i / vec_per_row, c = i - r * vec_per_row;
+    g4[static_cast<size_t>(r) * vec_per_row + c] =
+        __ldg(&x4[static_cast<size_t>(tok[r]) * vec_per_row + c]);
+  }
+  uint4* __restrict__ sf4 =
+      reinterpret_cast<uint4*>(xg_sf + static_cast<size_t>(tile) * kb_n * 512);
+  for (int i = tid; i < kb_n * 32; i += blockDim.x) {
+    const int kb = i >> 5, r32 = i & 31;
+    uint32_t w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int t = tok[r32 + 32 * q];
+      const uint32_t b = (t >= 0) ? xs[static_cast<size_t>(t) * kb_n + kb] : 127u;
+      w[q] = b * 0x01010101u;
+    }
+    sf4[kb * 32 + r32] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// Unpack the FC1 activation's scale chunks to a plain u8 [rows, I/128] array.
+__global__ void unpack_act_scales_kernel(const uint8_t* __restrict__ chunks, int nb,
+                                         long long rows, uint8_t* __restrict__ dst) {
+  const long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+  if (i >= rows * nb) return;
+  const long long r = i / nb;
+  const int b = static_cast<int>(i - r * nb);
+  const long long tile = r / kTileM;
+  const int rr = static_cast<int>(r - tile * kTileM);
+  dst[i] = chunks[(tile * nb + b) * 512 + (rr & 31) * 16 + (rr >> 5) * 4];
+}
+
+}  // namespace
+
+cudaError_t launch_route(const moe_plan_s* p, const int32_t* topk_idx, uint8_t* ws,
+                         cudaStream_t st) {
+  const auto& L = p->ws;
+  const int S = static_cast<int>(p->S);
+  route_hist_kernel<<<p->route_blocks, kRouteThreads, 0, st>>>(
+      topk_idx, S, p->E, reinterpret_cast<int32_t*>(ws + L.block_hist),
+      reinterpret_cast<uint32_t*>(ws + L.err));
+  route_scatter_kernel<<<p->route_blocks, kRouteThreads, 0, st>>>(
+      topk_idx, S, p->E, p->route_blocks, reinterpret_cast<const int32_t*>(ws + L.block_hist),
+      reinterpret_cast<int32_t*>(ws + L.counts), reinterpret_cast<int32_t*>(ws + L.offsets),
+      reinterpret_cast<int32_t*>(ws + L.tile_off), reinterpret_cast<int32_t*>(ws + L.pad_off),
+      reinterpret_cast<int32_t*>(ws + L.perm), reinterpret_cast<int32_t*>(ws + L.inv),
+      reinterpret_cast<uint32_t*>(ws + L.err));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const moe_plan_s* p, const uint8_t* x, const uint8_t* xs, uint8_t* ws,
+                          cudaStream_t st) {
+  const auto& L = p->ws;
+  const int tiles = static_cast<int>(p->rows_cap / kTileM);
+  gather_kernel<<<tiles, 256, 0, st>>>(
+      x, xs, p->H, p->k, p->E, reinterpret_cast<const int32_t*>(ws + L.tile_off),
+      reinterpret_cast<const int32_t*>(ws + L.counts),
+      reinterpret_cast<const int32_t*>(ws + L.offsets),
+      reinterpret_cast<const int32_t*>(ws + L.perm), ws + L.xg, ws + L.xg_sf);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpack_act_scales(const moe_plan_s* p, const uint8_t* ws, uint8_t* dst,
+                                     cudaStream_t st) {
+  const long long n = p->rows_cap * (p->I / 128);
+  const int blocks = static_cast<int>((n + 255) / 256);
+  unpack_act_scales_kernel<<<blocks, 256, 0, st>>>(ws + p->ws.act_sf, p->I / 128, p->rows_cap,
+                                                   dst);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

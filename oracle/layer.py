@@ -89,18 +89,25 @@ def route(topk_idx, num_experts):
 
 
 # ----------------------------------------------------------------------- dequantise
+# The decoders evaluated once for every code; indexing these tables is the same
+# function as calling them element by element.
+_E4M3 = decode_e4m3(np.arange(256, dtype=np.uint8))
+_UE8M0 = decode_ue8m0(np.arange(256, dtype=np.uint8))
+_E2M1 = decode_e2m1(np.arange(16))
+
+
 def dequant_act(codes, scales):
     """E4M3 codes [R, C] with one UE8M0 scale per 1x128 block [R, C/128] -> f64."""
-    v = decode_e4m3(codes)
-    s = decode_ue8m0(scales)
+    v = _E4M3[np.asarray(codes, dtype=np.uint8)]
+    s = _UE8M0[np.asarray(scales, dtype=np.uint8)]
     return v * np.repeat(s, BLOCK, axis=1)
 
 
 def dequant_w_fp8(codes, scales):
     """E4M3 weight codes [R, C] with UE8M0 scales per 128x128 block
     [R/128, C/128] -> f64."""
-    v = decode_e4m3(codes)
-    s = decode_ue8m0(scales)
+    v = _E4M3[np.asarray(codes, dtype=np.uint8)]
+    s = _UE8M0[np.asarray(scales, dtype=np.uint8)]
     s = np.repeat(np.repeat(s, BLOCK, axis=0), BLOCK, axis=1)
     return v * s
 
@@ -108,8 +115,8 @@ def dequant_w_fp8(codes, scales):
 def dequant_w_fp4(packed, scales):
     """E2M1 weights packed two per byte [R, C/2] with UE8M0 scales per 1x32 block
     [R, C/32] -> f64."""
-    v = decode_e2m1(unpack_e2m1_pairs(packed))
-    s = decode_ue8m0(scales)
+    v = _E2M1[unpack_e2m1_pairs(packed)]
+    s = _UE8M0[np.asarray(scales, dtype=np.uint8)]
     return v * np.repeat(s, FP4_BLOCK, axis=1)
 
 

@@ -1,0 +1,103 @@
+"""The C-ABI library: it loads, exports every entry point include/moe.h
+declares, and validates arguments on the host before launching anything
+(these calls never reach the GPU, so they run on CPU-only machines)."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+import moe_expert_ffn_permute_b200 as moe
+from moe_expert_ffn_permute_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build()
+    return moe.lib()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_entry_points():
+    names = _declared()
+    for n in ("moe_plan", "moe_forward", "moe_route", "moe_gather", "moe_fc1", "moe_fc2", "moe_combine",
+              "moe_workspace_bytes", "moe_check_device_error", "moe_plan_destroy",
+              "moe_status_str"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in _declared():
+        assert hasattr(L, name), name
+    assert set(_declared()) <= set(moe._SIGS)
+
+
+def test_plan_validation():
+    ok = moe.moe_plan(64, 512, 256, 8, 2)
+    assert moe.moe_workspace_bytes(ok) > 0
+    moe.moe_plan_destroy(ok)
+    bad = [dict(T=0, H=512, I=256, E=8, k=2), dict(T=4, H=500, I=256, E=8, k=2),
+           dict(T=4, H=512, I=200, E=8, k=2), dict(T=4, H=512, I=256, E=2, k=3),
+           dict(T=4, H=512, I=256, E=300, k=2), dict(T=4, H=384, I=256, E=8, k=2)]
+    codes = []
+    for b in bad:
+        with pytest.raises(moe.MoEError) as ei:
+            moe.moe_plan(b["T"], b["H"], b["I"], b["E"], b["k"])
+        codes.append(ei.value.status)
+    assert codes == [1, 2, 2, 1, 2, 2]
+    with pytest.raises(moe.MoEError):
+        moe.moe_plan(4, 512, 256, 8, 2, act="swiglu_oai", alpha=1.0, up_bias=0.0, limit=-1.0)
+    with pytest.raises(moe.MoEError):
+        moe.moe_plan(4, 512, 256, 8, 2, act="swiglu_oai", alpha=math.nan)
+
+
+def test_workspace_grows_with_debug_capture():
+    p = moe.moe_plan(64, 512, 256, 8, 2)
+    a = moe.moe_workspace_bytes(p)
+    moe.moe_plan_set_debug(p, True)
+    b = moe.moe_workspace_bytes(p)
+    assert b > a
+    moe.moe_plan_destroy(p)
+
+
+def test_forward_rejects_bad_pointers_before_launch():
+    p = moe.moe_plan(64, 512, 256, 8, 2)
+    good = 1 << 20                        # aligned fake addresses: never dereferenced
+    args = [good] * 9
+    with pytest.raises(moe.MoEError) as ei:             # null workspace
+        moe.moe_forward(p, *args, None, stream=0)
+    assert ei.value.status == 1
+    with pytest.raises(moe.MoEError) as ei:             # misaligned workspace
+        moe.moe_forward(p, *args, good + 8, stream=0)
+    assert ei.value.status == 3
+    with pytest.raises(moe.MoEError) as ei:             # null x
+        moe.moe_forward(p, None, *args[1:], good, stream=0)
+    assert ei.value.status == 1
+    with pytest.raises(moe.MoEError) as ei:             # misaligned w1
+        moe.moe_forward(p, good, good, good, good, good + 4, good, good, good, good, good,
+                        stream=0)
+    assert ei.value.status == 3
+    moe.moe_plan_destroy(p)
+
+
+def test_fp4_weights_need_32_byte_alignment():
+    p = moe.moe_plan(8, 512, 256, 8, 2, w_dtype="e2m1")
+    g = 1 << 20
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_fc2(p, g + 16, g, g, stream=0)
+    assert ei.value.status == 3
+    moe.moe_plan_destroy(p)
+
+
+def test_status_strings():
+    assert moe.moe_status_str(0) == "MOE_OK"
+    assert moe.moe_status_str(5) == "MOE_ERR_DEVICE_TIMEOUT"

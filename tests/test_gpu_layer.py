@@ -1,0 +1,135 @@
+"""Whole-layer parity of the CUDA path (through the C ABI) against the oracle,
+plus the FC1 epilogue's requantisation checked byte for byte."""
+import numpy as np
+import pytest
+import torch
+
+import moe_expert_ffn_permute_b200 as moe
+from moe_expert_ffn_permute_b200.synth import WORKLOADS, Workload, to_numpy
+from oracle import layer as L
+
+from gpu_helpers import (assert_parity, ensure_built, inputs, oracle_args, oracle_kw,
+                         oracle_tokens, run_gpu)
+
+pytestmark = pytest.mark.gpu
+
+RAGGED = Workload("ragged", 300, 1024, 512, 8, 4, cfg_id=20)
+RAGGED_FP4 = Workload("ragged-fp4", 300, 1024, 512, 8, 4, w_dtype="e2m1", cfg_id=21)
+RAGGED_OAI = Workload("ragged-oai", 200, 512, 384, 6, 3, act="swiglu_oai", alpha=1.702,
+                      up_bias=1.0, limit=7.0, cfg_id=22)
+SINGLE = Workload("single", 1, 256, 128, 1, 1, cfg_id=23)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    ensure_built()
+
+
+def _ws_bytes(lay, ptr, nbytes):
+    off = ptr - lay.workspace.data_ptr()
+    return lay.workspace[off:off + nbytes]
+
+
+@pytest.mark.parametrize("wl", [WORKLOADS["tiny"], RAGGED, RAGGED_FP4, RAGGED_OAI, SINGLE],
+                         ids=lambda w: w.name)
+def test_layer_parity_small(wl):
+    d = inputs(wl)
+    out, lay = run_gpu(wl, d)
+    assert lay.check() == 0
+    dn = to_numpy(d)
+    ref = L.layer(*oracle_args(dn), **oracle_kw(wl))
+    assert_parity(out.float().cpu().numpy(), ref, wl.name)
+
+
+@pytest.mark.parametrize("wl", [WORKLOADS["tiny"], RAGGED, RAGGED_FP4, RAGGED_OAI],
+                         ids=lambda w: w.name)
+def test_fc1_requant_bytes_exact_and_activation_close(wl):
+    """The FP8 codes and UE8M0 bytes the FC1 epilogue writes equal the oracle's
+    quantiser applied to the epilogue's own fp32 activation; that activation
+    agrees with the oracle's float64 one."""
+    d = inputs(wl)
+    out, lay = run_gpu(wl, d, debug=True)
+    v = lay.view()
+    rows = v.rows
+    act = _ws_bytes(lay, v.act, rows * wl.I).view(rows, wl.I).cpu().numpy()
+    a32 = _ws_bytes(lay, v.act_f32, rows * wl.I * 4).view(torch.float32).view(rows, wl.I)
+    a32 = a32.cpu().numpy()
+    sf = torch.empty(rows, wl.I // 128, dtype=torch.uint8, device="cuda")
+    moe.moe_copy_act_scales(lay.plan, lay.workspace, sf)
+    sf = sf.cpu().numpy()
+    pad = _ws_bytes(lay, v.pad_offsets, 4 * (wl.E + 1)).view(torch.int32).cpu().numpy()
+    dn = to_numpy(d)
+    _, inter = L.layer(*oracle_args(dn), **oracle_kw(wl), keep=True)
+    for e, a_ref in inter["a"].items():
+        n = a_ref.shape[0]
+        rows_e = slice(pad[e], pad[e] + n)
+        q_ref, s_ref = L.requant_1x128(a32[rows_e].astype(np.float64))
+        np.testing.assert_array_equal(act[rows_e], q_ref, err_msg=f"codes, expert {e}")
+        np.testing.assert_array_equal(sf[rows_e], s_ref, err_msg=f"scales, expert {e}")
+        assert_parity(a32[rows_e], a_ref, f"activation expert {e}")
+
+
+def test_layer_is_bitwise_repeatable():
+    wl = RAGGED
+    d = inputs(wl)
+    a, _ = run_gpu(wl, d)
+    b, _ = run_gpu(wl, d)
+    assert torch.equal(a, b)
+
+
+def test_out_of_range_ids_contribute_nothing():
+    wl = RAGGED
+    d = inputs(wl)
+    d["topk_idx"][5, 2] = -3
+    d["topk_idx"][100, 0] = wl.E + 7
+    out, lay = run_gpu(wl, d)
+    assert lay.check() == 6
+    dn = to_numpy(d)
+    ref = L.layer(*oracle_args(dn), **oracle_kw(wl))
+    assert_parity(out.float().cpu().numpy(), ref, "bad ids")
+
+
+def test_step_calls_equal_forward():
+    wl = RAGGED_OAI
+    d = inputs(wl)
+    full, lay = run_gpu(wl, d)
+    out = torch.empty_like(full)
+    moe.moe_route(lay.plan, d["topk_idx"], lay.workspace)
+    moe.moe_gather(lay.plan, d["x"], d["x_scales"], lay.workspace)
+    moe.moe_fc1(lay.plan, d["w1"], d["w1_scales"], lay.workspace)
+    moe.moe_fc2(lay.plan, d["w2"], d["w2_scales"], lay.workspace)
+    moe.moe_combine(lay.plan, d["topk_w"], out, lay.workspace)
+    torch.cuda.synchronize()
+    assert torch.equal(out, full)
+
+
+def test_hostio_equals_device_forward():
+    wl = RAGGED
+    d = inputs(wl)
+    full, lay = run_gpu(wl, d)
+    host = {k: v.cpu().pin_memory() for k, v in d.items() if k in ("x", "x_scales", "topk_idx",
+                                                                   "topk_w")}
+    out_h = torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory()
+    moe.moe_forward_hostio(lay.plan, host["x"], host["x_scales"], host["topk_idx"],
+                           host["topk_w"], d["w1"], d["w1_scales"], d["w2"], d["w2_scales"],
+                           out_h, lay.workspace)
+    torch.cuda.synchronize()
+    assert torch.equal(out_h, full.cpu())
+
+
+@pytest.mark.parametrize("name,T,ntok", [("decode", None, 48), ("prefill", None, 12),
+                                         ("oai", None, 64), ("mxfp4", 128, 12),
+                                         ("mxfp4", 8192, 6)])
+def test_layer_parity_full_size_sampled(name, T, ntok):
+    """Full-size workloads in the launch configuration the bench uses; the
+    oracle computes a seeded sample of tokens (each token's output depends only
+    on its own inputs)."""
+    wl = WORKLOADS[name] if T is None else WORKLOADS[name].with_tokens(T)
+    d = inputs(wl)
+    out, lay = run_gpu(wl, d)
+    assert lay.check() == 0
+    rng = np.random.default_rng(wl.T)
+    tokens = np.sort(rng.choice(wl.T, size=min(ntok, wl.T), replace=False))
+    dn = {k: v.cpu().numpy() for k, v in d.items()}
+    ref = oracle_tokens(wl, dn, tokens)
+    assert_parity(out.float().cpu().numpy()[tokens], ref, wl.name)
