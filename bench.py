@@ -69,7 +69,7 @@ class Clocks:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -99,7 +99,9 @@ class Clocks:
                     reasons.add(name)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "window": "continuous steps of the same layer, 0.6 s before and after "
+                          "the timed steps"}
 
 
 def algorithmic_bytes(wl, d):
@@ -161,12 +163,24 @@ def run_b200(args, wl):
     if lay.check() != 0:
         raise RuntimeError("device error during warm-up")
 
-    # ---- timed: whole layer, device-resident inputs
+    # ---- timed: whole layer, device-resident inputs.  The clock sampler needs
+    # ~100 ms per sample, longer than K steps of this layer take, so the timed
+    # steps sit inside a window of continuous (untimed) steps of the same layer
+    # that starts and ends 0.6 s around them; all samples are taken under load.
     clocks = Clocks(local)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clocks.start()
+
+    def soak(seconds):
+        t_end = time.perf_counter() + seconds
+        while time.perf_counter() < t_end:
+            for _ in range(20):
+                fwd()
+            torch.cuda.synchronize()
+
+    soak(0.6)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     for i in range(args.steps):
@@ -175,6 +189,7 @@ def run_b200(args, wl):
         fwd()
         ev[i][1].record(stream)
     torch.cuda.synchronize()
+    soak(0.6)
     clk = clocks.stop()
     if world > 1:
         dist.barrier()

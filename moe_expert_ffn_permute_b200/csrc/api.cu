@@ -108,8 +108,9 @@ moe_status moe_plan_set_debug(moe_plan_t plan, int capture_act_f32) {
 }
 
 int moe_forward_launch_count(moe_plan_t plan) {
-  (void)plan;
-  return 6;   // route histogram, route scatter, gather, FC1, FC2, combine
+  if (plan == nullptr) return 0;
+  // [route histogram,] route scan+scatter, gather, FC1, FC2, combine
+  return (plan->route_blocks > 1 ? 1 : 0) + 5;
 }
 
 static moe_status check_ws(moe_plan_t plan, const void* workspace) {

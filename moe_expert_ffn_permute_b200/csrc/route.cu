@@ -64,15 +64,30 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
   __shared__ int32_t scan[257];
   __shared__ int32_t wcount[kWarps][256];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int e = tid; e < E; e += blockDim.x) {
-    int before = 0, all = 0;
-    for (int b = 0; b < nblk; ++b) {
-      const int c = block_hist[b * E + e];
-      if (b < static_cast<int>(blockIdx.x)) before += c;
-      all += c;
+  if (nblk == 1) {
+    // A single block holds every slot: count them here (no histogram launch).
+    for (int e = tid; e < E; e += blockDim.x) {
+      running[e] = 0;
+      total[e] = 0;
     }
-    running[e] = before;
-    total[e] = all;
+    __syncthreads();
+    bool bad = false;
+    for (int s = tid; s < S; s += blockDim.x) {
+      const int e = idx[s];
+      if (e >= 0 && e < E) atomicAdd(&total[e], 1); else bad = true;
+    }
+    if (bad) atomicOr(err, kErrRoutingBit);
+  } else {
+    for (int e = tid; e < E; e += blockDim.x) {
+      int before = 0, all = 0;
+      for (int b = 0; b < nblk; ++b) {
+        const int c = block_hist[b * E + e];
+        if (b < static_cast<int>(blockIdx.x)) before += c;
+        all += c;
+      }
+      running[e] = before;
+      total[e] = all;
+    }
   }
   __syncthreads();
   if (tid == 0) {
@@ -141,58 +156,44 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
   }
 }
 
-// Gather: row r of padded m-tile `tile` receives x[perm[...] / k]; its scale
-// bytes are written in the tensor-core scale-chunk layout: for k-block kb the
-// 512-byte chunk holds, at byte (r % 32) * 16 + (r / 32) * 4 + j (j = 0..3), the
-// row's UE8M0 byte (replicated over the four 32-wide K sub-blocks).
-__global__ void __launch_bounds__(256) gather_kernel(
+// Gather: padded row P (m-tile P / 128, row r = P % 128) of expert e receives
+// x[perm[offsets[e] + local + r] / k]; one warp per row, 16-byte accesses.
+// Its scale bytes go to the tensor-core scale-chunk layout: for k-block kb the
+// 512-byte chunk of the tile holds, at byte (r % 32) * 16 + (r / 32) * 4 + j
+// (j = 0..3), the row's UE8M0 byte, replicated over the four 32-wide K
+// sub-blocks.  Padding rows are left untouched (their results are never
+// stored).
+constexpr int kGatherWarps = 8;
+
+__global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(
     const uint8_t* __restrict__ x, const uint8_t* __restrict__ xs, int H, int k, int E,
     const int32_t* __restrict__ tile_off, const int32_t* __restrict__ counts,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm,
     uint8_t* __restrict__ xg, uint8_t* __restrict__ xg_sf) {
-  __shared__ int32_t tok[kTileM];
-  __shared__ int e_sh, rows_sh;
-  const int tile = blockIdx.x;
-  const int tid = threadIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long P = static_cast<long long>(blockIdx.x) * kGatherWarps + warp;
+  const int tile = static_cast<int>(P / kTileM);
+  const int r = static_cast<int>(P % kTileM);
   if (tile >= __ldg(&tile_off[E])) return;
-  if (tid == 0) {
-    int lo = 0, hi = E;   // last e with tile_off[e] <= tile
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (tile_off[mid] <= tile) lo = mid; else hi = mid;
-    }
-    while (lo + 1 <= E && tile_off[lo + 1] <= tile) ++lo;
-    e_sh = lo;
-    const int local = (tile - tile_off[lo]) * kTileM;
-    rows_sh = min(kTileM, counts[lo] - local);
+  int lo = 0, hi = E;   // the expert owning the tile: last e with tile_off[e] <= tile
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(&tile_off[mid]) <= tile) lo = mid; else hi = mid;
   }
-  __syncthreads();
-  const int e = e_sh, rows = rows_sh;
-  const int local = (tile - tile_off[e]) * kTileM;
-  for (int r = tid; r < kTileM; r += blockDim.x)
-    tok[r] = (r < rows) ? perm[offsets[e] + local + r] / k : -1;
-  __syncthreads();
+  while (lo + 1 <= E && __ldg(&tile_off[lo + 1]) <= tile) ++lo;
+  const int e = lo;
+  const int local = (tile - __ldg(&tile_off[e])) * kTileM + r;
+  if (local >= __ldg(&counts[e])) return;
+  const int t = __ldg(&perm[__ldg(&offsets[e]) + local]) / k;
+  const int vec = H / 16;
+  const uint4* __restrict__ src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
+  uint4* __restrict__ dst = reinterpret_cast<uint4*>(xg + static_cast<size_t>(P) * H);
+  for (int c = lane; c < vec; c += 32) dst[c] = __ldg(&src[c]);
   const int kb_n = H / 128;
-  const int vec_per_row = H / 16;
-  const uint4* __restrict__ x4 = reinterpret_cast<const uint4*>(x);
-  uint4* __restrict__ g4 = reinterpret_cast<uint4*>(xg + static_cast<size_t>(tile) * kTileM * H);
-  for (int i = tid; i < rows * vec_per_row; i += blockDim.x) {
-    const int r = i / vec_per_row, c = i - r * vec_per_row;
-    g4[static_cast<size_t>(r) * vec_per_row + c] =
-        __ldg(&x4[static_cast<size_t>(tok[r]) * vec_per_row + c]);
-  }
-  uint4* __restrict__ sf4 =
-      reinterpret_cast<uint4*>(xg_sf + static_cast<size_t>(tile) * kb_n * 512);
-  for (int i = tid; i < kb_n * 32; i += blockDim.x) {
-    const int kb = i >> 5, r32 = i & 31;
-    uint32_t w[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int t = tok[r32 + 32 * q];
-      const uint32_t b = (t >= 0) ? xs[static_cast<size_t>(t) * kb_n + kb] : 127u;
-      w[q] = b * 0x01010101u;
-    }
-    sf4[kb * 32 + r32] = make_uint4(w[0], w[1], w[2], w[3]);
+  uint8_t* chunk = xg_sf + static_cast<size_t>(tile) * kb_n * 512 + (r & 31) * 16 + (r >> 5) * 4;
+  for (int kb = lane; kb < kb_n; kb += 32) {
+    const uint32_t b = __ldg(&xs[static_cast<size_t>(t) * kb_n + kb]);
+    *reinterpret_cast<uint32_t*>(chunk + static_cast<size_t>(kb) * 512) = b * 0x01010101u;
   }
 }
 
@@ -214,9 +215,10 @@ cudaError_t launch_route(const moe_plan_s* p, const int32_t* topk_idx, uint8_t* 
                          cudaStream_t st) {
   const auto& L = p->ws;
   const int S = static_cast<int>(p->S);
-  route_hist_kernel<<<p->route_blocks, kRouteThreads, 0, st>>>(
-      topk_idx, S, p->E, reinterpret_cast<int32_t*>(ws + L.block_hist),
-      reinterpret_cast<uint32_t*>(ws + L.err));
+  if (p->route_blocks > 1)
+    route_hist_kernel<<<p->route_blocks, kRouteThreads, 0, st>>>(
+        topk_idx, S, p->E, reinterpret_cast<int32_t*>(ws + L.block_hist),
+        reinterpret_cast<uint32_t*>(ws + L.err));
   route_scatter_kernel<<<p->route_blocks, kRouteThreads, 0, st>>>(
       topk_idx, S, p->E, p->route_blocks, reinterpret_cast<const int32_t*>(ws + L.block_hist),
       reinterpret_cast<int32_t*>(ws + L.counts), reinterpret_cast<int32_t*>(ws + L.offsets),
@@ -229,8 +231,8 @@ cudaError_t launch_route(const moe_plan_s* p, const int32_t* topk_idx, uint8_t* 
 cudaError_t launch_gather(const moe_plan_s* p, const uint8_t* x, const uint8_t* xs, uint8_t* ws,
                           cudaStream_t st) {
   const auto& L = p->ws;
-  const int tiles = static_cast<int>(p->rows_cap / kTileM);
-  gather_kernel<<<tiles, 256, 0, st>>>(
+  const int blocks = static_cast<int>(p->rows_cap / kGatherWarps);
+  gather_kernel<<<blocks, kGatherWarps * 32, 0, st>>>(
       x, xs, p->H, p->k, p->E, reinterpret_cast<const int32_t*>(ws + L.tile_off),
       reinterpret_cast<const int32_t*>(ws + L.counts),
       reinterpret_cast<const int32_t*>(ws + L.offsets),
