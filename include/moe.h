@@ -169,6 +169,31 @@ moe_status moe_fc2(moe_plan_t plan, const void *w2, const uint8_t *w2_scales,
 moe_status moe_combine(moe_plan_t plan, const float *topk_w, void *out,
                        void *workspace, moe_stream_t stream);
 
+/* Allocation-free routing.  The pages have no counterpart of this entry point.
+ *
+ * Same result as moe_route() (counts i32[E], offsets i32[E+1], perm i32[S],
+ * inv i32[S], all device pointers owned by the caller; out-of-range expert ids
+ * give inv[s] = -1), but it needs no workspace and allocates nothing: its
+ * scratch (per-block histograms, tile offsets, an error word) is a ~515 KiB
+ * array in the library's static device memory, which every GPU that loads the
+ * library keeps until the process exits.  It is meant for callers that cannot
+ * allocate device memory where they route -- e.g. a runtime whose pooled
+ * allocator owns the device's whole budget, or a latency-critical loop where
+ * an allocation could synchronise the device.
+ *   - Sizes: S = T*k <= MOE_ROUTE_STATIC_MAX_SLOTS and E <= 256; larger
+ *     requests return MOE_ERR_UNSUPPORTED and enqueue nothing.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - All calls share the one array and it keeps the last call's contents;
+ *     the call clears what must start at zero.  Calls that overlap on the GPU
+ *     (different streams, no ordering between them) race on the array and
+ *     must not be issued.                                                   */
+#define MOE_ROUTE_STATIC_MAX_SLOTS (1 << 20)
+moe_status moe_route_static(const int32_t *topk_idx, int T, int k, int E,
+                            int32_t *counts, int32_t *offsets, int32_t *perm,
+                            int32_t *inv, moe_stream_t stream);
+
 /* Device pointers (inside `workspace`) of the intermediate results, for
  * inspection.  Rows of act / act_f32 are in expert order with every expert's
  * block starting at a multiple of 128 rows: expert e's rows are

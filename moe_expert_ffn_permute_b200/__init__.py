@@ -54,6 +54,7 @@ _SIGS = {
     "moe_forward": (ctypes.c_int, [_P] * 12),
     "moe_forward_hostio": (ctypes.c_int, [_P] * 12),
     "moe_route": (ctypes.c_int, [_P] * 4),
+    "moe_route_static": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int] + [_P] * 5),
     "moe_gather": (ctypes.c_int, [_P] * 5),
     "moe_fc1": (ctypes.c_int, [_P] * 5),
     "moe_fc2": (ctypes.c_int, [_P] * 5),
@@ -154,6 +155,17 @@ def moe_forward_hostio(plan, x_host, x_scales_host, topk_idx_host, topk_w_host, 
 
 def moe_route(plan, topk_idx, workspace, stream=None):
     _check(lib().moe_route(plan, _ptr(topk_idx), _ptr(workspace), _stream(stream)), "moe_route")
+
+
+def moe_route_static(topk_idx, T, k, E, counts, offsets, perm, inv, stream=None):
+    """Routing without a workspace: scratch lives in the library's static device
+    memory (at most MOE_ROUTE_STATIC_MAX_SLOTS slots; calls must not overlap)."""
+    _check(lib().moe_route_static(_ptr(topk_idx), T, k, E, *map(_ptr, (counts, offsets, perm,
+                                                                         inv)),
+                                  _stream(stream)), "moe_route_static")
+
+
+ROUTE_STATIC_MAX_SLOTS = 1 << 20
 
 
 def moe_gather(plan, x, x_scales, workspace, stream=None):

@@ -13,6 +13,8 @@
 // the scale chunks can be addressed per tile.
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -250,3 +252,88 @@ cudaError_t launch_unpack_act_scales(const moe_plan_s* p, const uint8_t* ws, uin
 }
 
 }  // namespace moe
+
+// ---------------------------------------------------------------------------
+// Allocation-free routing (moe_route_static in include/moe.h).
+//
+// Some callers cannot allocate device memory at the point where they route: a
+// serving runtime whose pooled allocator owns the whole device budget, or a
+// latency-critical loop in which a device allocation could synchronise the
+// device.  For them the routing step can take its scratch (the per-block
+// histograms, the padded tile offsets and the error word) from a buffer that
+// lives in this module's static device memory, sized once for at most
+// MOE_ROUTE_STATIC_MAX_SLOTS slots and kept by every GPU that loads the library
+// until the process exits.  The routing kernels themselves are the ones above;
+// only where their scratch lives differs.
+namespace moe {
+namespace {
+
+constexpr long long kStaticMaxSlots = MOE_ROUTE_STATIC_MAX_SLOTS;
+constexpr size_t kStaticErrOff = 0;
+constexpr size_t kStaticTileOff = 256;
+constexpr size_t kStaticPadOff = kStaticTileOff + 257 * 4 + 252;   // 256-B aligned
+constexpr size_t kStaticHistOff = kStaticPadOff + 257 * 4 + 252;
+constexpr size_t kStaticHistBytes =
+    static_cast<size_t>((kStaticMaxSlots + kRouteChunk - 1) / kRouteChunk) * 256 * 4;
+constexpr size_t kStaticScratchBytes = kStaticHistOff + kStaticHistBytes;   // ~515 KiB
+
+// Host code must not hand this name to a kernel: on the host it is only a
+// stand-in for the symbol.  Its device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) uint8_t g_route_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+uint8_t* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the static scratch on the current device, looked up once
+// per device (with that device current) and cached.
+cudaError_t static_scratch(uint8_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_route_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = static_cast<uint8_t*>(ptr);
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" moe_status moe_route_static(const int32_t* topk_idx, int T, int k, int E,
+                                       int32_t* counts, int32_t* offsets, int32_t* perm,
+                                       int32_t* inv, moe_stream_t stream) {
+  using namespace moe;
+  if (topk_idx == nullptr || counts == nullptr || offsets == nullptr || perm == nullptr ||
+      inv == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (T < 1 || k < 1 || E < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (E > 256) return MOE_ERR_UNSUPPORTED;
+  const long long S = static_cast<long long>(T) * k;
+  if (S > kStaticMaxSlots) return MOE_ERR_UNSUPPORTED;   // beyond the static scratch
+  for (const void* p : {static_cast<const void*>(topk_idx), static_cast<const void*>(counts),
+                        static_cast<const void*>(offsets), static_cast<const void*>(perm),
+                        static_cast<const void*>(inv)})
+    if (reinterpret_cast<uintptr_t>(p) % 4 != 0) return MOE_ERR_ALIGNMENT;
+  uint8_t* scratch = nullptr;
+  if (static_scratch(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  const int nblk = static_cast<int>((S + kRouteChunk - 1) / kRouteChunk);
+  // The error word keeps the previous call's bits: clear it first.
+  if (cudaMemsetAsync(scratch + kStaticErrOff, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+  auto err = reinterpret_cast<uint32_t*>(scratch + kStaticErrOff);
+  auto hist = reinterpret_cast<int32_t*>(scratch + kStaticHistOff);
+  if (nblk > 1)
+    route_hist_kernel<<<nblk, kRouteThreads, 0, st>>>(topk_idx, static_cast<int>(S), E, hist, err);
+  route_scatter_kernel<<<nblk, kRouteThreads, 0, st>>>(
+      topk_idx, static_cast<int>(S), E, nblk, hist, counts, offsets,
+      reinterpret_cast<int32_t*>(scratch + kStaticTileOff),
+      reinterpret_cast<int32_t*>(scratch + kStaticPadOff), perm, inv, err);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
