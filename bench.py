@@ -104,6 +104,35 @@ class Clocks:
                           "the timed steps"}
 
 
+KERNEL_SOURCES = ("moe_expert_ffn_permute_b200/csrc/gemm.cu",
+                  "moe_expert_ffn_permute_b200/csrc/sm100.cuh",
+                  "moe_expert_ffn_permute_b200/csrc/internal.h")
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload):
+    """DRAM bytes per launch of the GEMM kernel from the committed ncu summary
+    (profiles/gemm_traffic.json), or None when the kernel sources changed since
+    the counters were taken or no capture exists for this workload."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "gemm_traffic.json")) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = rec.get(workload)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
 def algorithmic_bytes(wl, d):
     """Bytes the layer must move at minimum: the weights and scales of the
     experts that receive tokens, x and its scales, the routing, the output."""
@@ -111,10 +140,9 @@ def algorithmic_bytes(wl, d):
     counts = torch.bincount(d["topk_idx"].reshape(-1).long(), minlength=wl.E)[:wl.E]
     active = int((counts > 0).sum())
     per_expert_w = sum(d[k][0].numel() for k in ("w1", "w1_scales", "w2", "w2_scales"))
-    fc1_w = d["w1"][0].numel() + d["w1_scales"][0].numel()
     act_bytes = (d["x"].numel() + d["x_scales"].numel() + d["topk_idx"].numel() * 4 +
                  d["topk_w"].numel() * 4 + wl.T * wl.H * 2)
-    return active * per_expert_w + act_bytes, active * fc1_w, active
+    return active * per_expert_w + act_bytes, active * per_expert_w, active
 
 
 def run_b200(args, wl):
@@ -144,24 +172,39 @@ def run_b200(args, wl):
     args_dev = (d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], d["w1"], d["w1_scales"],
                 d["w2"], d["w2_scales"])
 
-    def fwd():
-        moe.moe_forward(lay.plan, *args_dev, out, lay.workspace, stream)
+    def fwd(st=None):
+        moe.moe_forward(lay.plan, *args_dev, out, lay.workspace,
+                        st if st is not None else torch.cuda.current_stream())
 
     steps = [("route", lambda: moe.moe_route(lay.plan, d["topk_idx"], lay.workspace, stream)),
              ("gather", lambda: moe.moe_gather(lay.plan, d["x"], d["x_scales"], lay.workspace,
                                                stream)),
-             ("fc1", lambda: moe.moe_fc1(lay.plan, d["w1"], d["w1_scales"], lay.workspace,
-                                         stream)),
-             ("fc2", lambda: moe.moe_fc2(lay.plan, d["w2"], d["w2_scales"], lay.workspace,
-                                         stream)),
+             ("fc1_fc2", lambda: moe.moe_fc1_fc2(lay.plan, d["w1"], d["w1_scales"], d["w2"],
+                                                 d["w2_scales"], lay.workspace, stream)),
              ("combine", lambda: moe.moe_combine(lay.plan, d["topk_w"], out, lay.workspace,
                                                  stream))]
+    # The two GEMMs as separate launches (informational; moe_forward fuses them).
+    extra = [("fc1_alone", lambda: moe.moe_fc1(lay.plan, d["w1"], d["w1_scales"],
+                                               lay.workspace, stream)),
+             ("fc2_alone", lambda: moe.moe_fc2(lay.plan, d["w2"], d["w2_scales"],
+                                               lay.workspace, stream))]
 
     for _ in range(args.warmup):
         fwd()
     torch.cuda.synchronize()
     if lay.check() != 0:
         raise RuntimeError("device error during warm-up")
+
+    # The timed step replays a CUDA graph of moe_forward (the same kernels with
+    # the same arguments; the routing kernel resets the GEMM scheduler's
+    # counters inside the graph, so every replay starts from a clean state).
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        fwd()
+    torch.cuda.synchronize()
+
+    def step():
+        graph.replay()
 
     # ---- timed: whole layer, device-resident inputs.  The clock sampler needs
     # ~100 ms per sample, longer than K steps of this layer take, so the timed
@@ -177,37 +220,43 @@ def run_b200(args, wl):
         t_end = time.perf_counter() + seconds
         while time.perf_counter() < t_end:
             for _ in range(20):
-                fwd()
+                step()
             torch.cuda.synchronize()
 
+    def timed(fn):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            fn()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in ev]
+
     soak(0.6)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush.fill_(i & 0xFF)
-        ev[i][0].record(stream)
-        fwd()
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
+    step_ms = timed(step)
     soak(0.6)
     clk = clocks.stop()
+    eager_ms = timed(fwd)
     if world > 1:
         dist.barrier()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = sum(step_ms)
 
-    # ---- per-kernel split (same launch sequence, one event per step boundary)
-    split = {name: [] for name, _ in steps}
-    for i in range(args.steps):
-        flush.fill_(i & 0xFF)
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(steps) + 1)]
-        evs[0].record(stream)
-        for j, (_, fn) in enumerate(steps):
-            fn()
-            evs[j + 1].record(stream)
-        torch.cuda.synchronize()
-        for j, (name, _) in enumerate(steps):
-            split[name].append(evs[j].elapsed_time(evs[j + 1]))
+    # ---- per-kernel split (the launch sequence of moe_forward, one event per
+    # step boundary, on the launching stream), then the unfused GEMMs.
+    split = {name: [] for name, _ in steps + extra}
+    for seq in (steps, steps[:2] + extra):
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(seq) + 1)]
+            evs[0].record(stream)
+            for j, (_, fn) in enumerate(seq):
+                fn()
+                evs[j + 1].record(stream)
+            torch.cuda.synchronize()
+            for j, (name, _) in enumerate(seq):
+                split[name].append(evs[j].elapsed_time(evs[j + 1]))
 
     # ---- e2e through the host-buffer entry point
     host = {k: d[k].cpu().pin_memory() for k in ("x", "x_scales", "topk_idx", "topk_w")}
@@ -237,21 +286,23 @@ def run_b200(args, wl):
         dist.all_reduce(vals, op=dist.ReduceOp.MAX)
     total_ms, e2e_total = float(vals[0]), float(vals[1])
 
-    alg_bytes, fc1_bytes, active = algorithmic_bytes(wl, d)
+    alg_bytes, w_bytes, active = algorithmic_bytes(wl, d)
     hbm, bf16, bf16_sus, peak_src = _peaks()
     flops = 6.0 * wl.S * wl.H * wl.I
-    fc1_flops = 4.0 * wl.S * wl.H * wl.I
-    fc1_ms = statistics.mean(split["fc1"])
+    gemm_ms = statistics.mean(split["fc1_fc2"])
     hbm_bound = alg_bytes / (hbm * 1e9) > flops / (2 * bf16 * 1e12)
     if hbm_bound:
-        roof = {"bound": "hbm", "achieved": round(fc1_bytes / (fc1_ms * 1e-3) / 1e9, 1),
+        roof = {"bound": "hbm", "achieved": round(w_bytes / (gemm_ms * 1e-3) / 1e9, 1),
                 "peak": hbm, "unit": "GB/s"}
     else:
-        roof = {"bound": "tensor", "achieved": round(fc1_flops / (fc1_ms * 1e-3) / 1e12, 1),
+        roof = {"bound": "tensor", "achieved": round(flops / (gemm_ms * 1e-3) / 1e12, 1),
                 "peak": round(2 * bf16, 1), "unit": "TFLOP/s"}
     roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
-    roof["traffic"] = None
-    roof["kernel"] = "fc1 (grouped GEMM + SwiGLU + FP8 requant)"
+    roof["traffic"] = measured_traffic(wl.name)
+    roof["kernel"] = ("moe_gemm_kernel: FC1 + SwiGLU + FP8 requant and FC2 in one persistent "
+                      "launch")
+    roof["per_launch"] = (f"{w_bytes} B of expert weights+scales ({active} active experts)"
+                          if hbm_bound else f"{flops:.4g} FLOP (6*S*H*I)")
     roof["peak_source"] = f"{peak_src}" + ("" if roof["unit"] == "GB/s" else
                                            " bf16 burst x2 (FP8 = 2x bf16 nominal)")
 
@@ -271,6 +322,8 @@ def run_b200(args, wl):
                      "hbm_gbs": round(alg_bytes / (ms_per_step * 1e-3) / 1e9, 1),
                      "alg_bytes": alg_bytes, "flops": flops},
         "kernels_ms": {k: round(statistics.mean(v), 4) for k, v in split.items()},
+        "eager_ms_per_step": round(sum(eager_ms) / args.steps, 4),
+        "timing": "CUDA-graph replay of moe_forward, events on the launching stream",
         "roofline": roof,
         "e2e": {"value": round(tokens / (e2e_total * 1e-3 / args.steps), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(sum(v.numel() * v.element_size() for v in host.values())),

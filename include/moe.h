@@ -163,6 +163,16 @@ moe_status moe_fc1(moe_plan_t plan, const void *w1, const uint8_t *w1_scales,
 moe_status moe_fc2(moe_plan_t plan, const void *w2, const uint8_t *w2_scales,
                    void *workspace, moe_stream_t stream);
 
+/* Steps 3 + 4 in one persistent launch (what moe_forward uses): FC1 tiles and
+ * FC2 tiles are handed out by one dynamic tile counter, all FC1 tiles first;
+ * an FC2 tile of an m-tile starts once every FC1 tile of that m-tile has
+ * published its activation rows.  Same results as moe_fc1() then moe_fc2().
+ * Needs moe_gather() first (and moe_route() before it, which resets the
+ * launch's counters).                                                      */
+moe_status moe_fc1_fc2(moe_plan_t plan, const void *w1, const uint8_t *w1_scales,
+                       const void *w2, const uint8_t *w2_scales, void *workspace,
+                       moe_stream_t stream);
+
 /* Step 5, combine: out[t] = bf16(sum_j topk_w[t,j] * y[t*k+j]) in fp32, j
  * ascending; unrouted slots are skipped.  Needs moe_fc2() first.
  * Sources: DeepGEMM PR #386 title ("direct combine").                        */

@@ -58,6 +58,7 @@ _SIGS = {
     "moe_gather": (ctypes.c_int, [_P] * 5),
     "moe_fc1": (ctypes.c_int, [_P] * 5),
     "moe_fc2": (ctypes.c_int, [_P] * 5),
+    "moe_fc1_fc2": (ctypes.c_int, [_P] * 7),
     "moe_combine": (ctypes.c_int, [_P] * 5),
     "moe_workspace_view": (ctypes.c_int, [_P, _P, ctypes.POINTER(WorkspaceView)]),
     "moe_copy_act_scales": (ctypes.c_int, [_P] * 4),
@@ -181,6 +182,11 @@ def moe_fc1(plan, w1, w1_scales, workspace, stream=None):
 def moe_fc2(plan, w2, w2_scales, workspace, stream=None):
     _check(lib().moe_fc2(plan, *map(_ptr, (w2, w2_scales, workspace)), _stream(stream)),
            "moe_fc2")
+
+
+def moe_fc1_fc2(plan, w1, w1_scales, w2, w2_scales, workspace, stream=None):
+    _check(lib().moe_fc1_fc2(plan, *map(_ptr, (w1, w1_scales, w2, w2_scales, workspace)),
+                             _stream(stream)), "moe_fc1_fc2")
 
 
 def moe_combine(plan, topk_w, out, workspace, stream=None):

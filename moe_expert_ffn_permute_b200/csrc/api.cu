@@ -27,8 +27,10 @@ void compute_layout(moe_plan_s* p) {
   L.pad_off = take((E + 1) * 4);
   L.tile_off = take((E + 1) * 4);
   L.block_hist = take(static_cast<size_t>(p->route_blocks) * E * 4);
+  L.sched = take(256 + rows / kTileM * 4);
   L.perm = take(S * 4);
   L.inv = take(S * 4);
+  L.row_token = take(rows * 4);
   L.xg = take(rows * p->H);
   L.xg_sf = take(rows / kTileM * (p->H / 128) * 512);
   L.act = take(rows * p->I);
@@ -109,8 +111,8 @@ moe_status moe_plan_set_debug(moe_plan_t plan, int capture_act_f32) {
 
 int moe_forward_launch_count(moe_plan_t plan) {
   if (plan == nullptr) return 0;
-  // [route histogram,] route scan+scatter, gather, FC1, FC2, combine
-  return (plan->route_blocks > 1 ? 1 : 0) + 5;
+  // [route histogram,] route scan+scatter, gather, FC1+FC2 (one launch), combine
+  return (plan->route_blocks > 1 ? 1 : 0) + 4;
 }
 
 static moe_status check_ws(moe_plan_t plan, const void* workspace) {
@@ -167,6 +169,17 @@ moe_status moe_fc2(moe_plan_t plan, const void* w2, const uint8_t* w2_scales, vo
                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_fc1_fc2(moe_plan_t plan, const void* w1, const uint8_t* w1_scales, const void* w2,
+                       const uint8_t* w2_scales, void* workspace, moe_stream_t stream) {
+  moe_status s = check_ws(plan, workspace);
+  if (s != MOE_OK) return s;
+  if ((s = check_weights(plan, w1, w1_scales)) != MOE_OK) return s;
+  if ((s = check_weights(plan, w2, w2_scales)) != MOE_OK) return s;
+  return cuda_status(moe::launch_fc12(plan, w1, w1_scales, w2, w2_scales,
+                                      static_cast<uint8_t*>(workspace),
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_combine(moe_plan_t plan, const float* topk_w, void* out, void* workspace,
                        moe_stream_t stream) {
   moe_status s = check_ws(plan, workspace);
@@ -193,8 +206,10 @@ moe_status moe_forward(moe_plan_t plan, const void* x, const uint8_t* x_scales,
   if ((s = check_weights(plan, w2, w2_scales)) != MOE_OK) return s;
   if ((s = moe_route(plan, topk_idx, workspace, stream)) != MOE_OK) return s;
   if ((s = moe_gather(plan, x, x_scales, workspace, stream)) != MOE_OK) return s;
-  if ((s = moe_fc1(plan, w1, w1_scales, workspace, stream)) != MOE_OK) return s;
-  if ((s = moe_fc2(plan, w2, w2_scales, workspace, stream)) != MOE_OK) return s;
+  // FC1 and FC2 share one persistent launch: FC2 tiles of an m-tile start as
+  // soon as that m-tile's FC1 tiles are done (no wave tail between the GEMMs).
+  if ((s = moe_fc1_fc2(plan, w1, w1_scales, w2, w2_scales, workspace, stream)) != MOE_OK)
+    return s;
   return moe_combine(plan, topk_w, out, workspace, stream);
 }
 

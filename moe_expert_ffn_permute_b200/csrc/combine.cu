@@ -9,14 +9,19 @@
 #include <cuda_runtime.h>
 
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace moe {
 namespace {
+
+constexpr int kMaxK = 16;
 
 __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ y,
                                                       const float* __restrict__ topk_w,
                                                       const int32_t* __restrict__ inv, int T,
                                                       int H, int k, uint16_t* __restrict__ out) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int vecs = H / 8;
   const long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
   if (i >= static_cast<long long>(T) * vecs) return;
@@ -25,18 +30,28 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
   float acc[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
-  for (int j = 0; j < k; ++j) {
-    const long long s = static_cast<long long>(t) * k + j;
-    if (__ldg(&inv[s]) < 0) continue;
-    const float w = __ldg(&topk_w[s]);
-    const uint4 v = __ldcs(reinterpret_cast<const uint4*>(y + s * H) + c);
-    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+  for (int j0 = 0; j0 < k; j0 += kMaxK) {
+    // Issue every load of this group before using any (more bytes in flight).
+    float w[kMaxK];
+    uint4 v[kMaxK];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float lo = __uint_as_float(wv[q] << 16);
-      const float hi = __uint_as_float(wv[q] & 0xFFFF0000u);
-      acc[2 * q] = fmaf(w, lo, acc[2 * q]);
-      acc[2 * q + 1] = fmaf(w, hi, acc[2 * q + 1]);
+    for (int j = 0; j < kMaxK; ++j) {
+      const long long s = static_cast<long long>(t) * k + j0 + j;
+      const bool live = (j0 + j < k) && __ldg(&inv[s]) >= 0;
+      w[j] = live ? __ldg(&topk_w[s]) : 0.0f;
+      v[j] = live ? __ldcs(reinterpret_cast<const uint4*>(y + s * H) + c) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (j0 + j >= k) break;
+      const uint32_t wv[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float lo = __uint_as_float(wv[q] << 16);
+        const float hi = __uint_as_float(wv[q] & 0xFFFF0000u);
+        acc[2 * q] = fmaf(w[j], lo, acc[2 * q]);
+        acc[2 * q + 1] = fmaf(w[j], hi, acc[2 * q + 1]);
+      }
     }
   }
   uint32_t o[4];
@@ -55,10 +70,10 @@ cudaError_t launch_combine(const moe_plan_s* p, const float* topk_w, void* out, 
                            cudaStream_t st) {
   const long long n = static_cast<long long>(p->T) * (p->H / 8);
   const int blocks = static_cast<int>((n + 255) / 256);
-  combine_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const uint16_t*>(ws + p->ws.y), topk_w,
-                                         reinterpret_cast<const int32_t*>(ws + p->ws.inv), p->T,
-                                         p->H, p->k, reinterpret_cast<uint16_t*>(out));
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3(blocks), dim3(256), 0, st,
+                    reinterpret_cast<const uint16_t*>(ws + p->ws.y), topk_w,
+                    reinterpret_cast<const int32_t*>(ws + p->ws.inv), p->T, p->H, p->k,
+                    reinterpret_cast<uint16_t*>(out));
 }
 
 }  // namespace moe

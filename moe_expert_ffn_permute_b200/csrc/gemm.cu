@@ -34,6 +34,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstring>
 
 #include "internal.h"
 #include "sm100.cuh"
@@ -47,6 +48,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 0, kSfaCol = 256, kSfbCol = 264;
 constexpr int kEpiWarps = 8;
 constexpr int kSchedConsumers = 2 + kEpiWarps;   // producer, MMA, epilogue warps
+constexpr uint64_t kDepWaitLimitNs = 2000000000ull;
 
 struct __align__(1024) Smem {
   uint8_t a[STAGES][BM * BK];
@@ -60,25 +62,34 @@ struct __align__(1024) Smem {
   uint64_t sched_full[SCHED_DEPTH];
   uint64_t sched_empty[SCHED_DEPTH];
   uint64_t pair[4];
-  int4 task[SCHED_DEPTH];          // expert, m-tile (padded), n-tile, valid rows
+  int4 task[SCHED_DEPTH];          // kind | reuse << 1 | expert << 2, m-tile, n-tile, rows
   int task_pos[SCHED_DEPTH];       // position (unpadded) of the tile's first row
   float amax[2][2][BM];            // [tile parity][half][row]
   uint32_t tmem_base;
   int abort_flag;
 };
 
-struct Params {
-  int E, n_tiles, k_blocks;
+// One GEMM "phase": FC1 (x rows x W1, SwiGLU + requant epilogue) or FC2
+// (activation rows x W2, bf16 slot-order epilogue).
+struct Phase {
+  int n_tiles;               // per m-tile: I/128 (FC1) or H/256 (FC2)
+  int k_blocks;              // K / 128
   int b_rows_per_expert;     // 2I (FC1) or H (FC2)
-  int I, H;
-  int fp4;                   // weights are E2M1 + 1x32 scales
-  int fc1;
+  const uint8_t* sfa_chunks; // [m-tiles][k_blocks][512]
+  const uint8_t* w_sf;       // weight scales
+};
+
+struct Params {
+  int E, I, H;
+  int phases;                // bit 0: FC1 tiles, bit 1: FC2 tiles
+  int dynamic;               // tiles from a global counter (else round-robin)
+  Phase ph[2];
   const int32_t* tile_off;
   const int32_t* counts;
   const int32_t* offsets;
   const int32_t* perm;
-  const uint8_t* sfa_chunks; // [m-tiles][k_blocks][512]
-  const uint8_t* w_sf;
+  uint32_t* tile_counter;    // dynamic scheduling (zeroed by the routing kernel)
+  uint32_t* fc1_done;        // per m-tile: FC1 epilogue warps finished (zeroed by routing)
   // FC1 epilogue
   uint8_t* act;
   uint8_t* act_sf_chunks;
@@ -91,7 +102,8 @@ struct Params {
 };
 
 struct Task {
-  int e, mt, nt, rows, pos;
+  int kind, e, mt, nt, rows, pos;
+  int reuse;   // the expert has more than one m-tile: its weight tiles are read again
 };
 
 // Consumer side of the scheduler ring: copy the task info out of the slot,
@@ -101,7 +113,9 @@ __device__ __forceinline__ bool get_task(Smem& sm, int& slot, uint32_t& phase, T
                                          uint32_t* err) {
   if (!mbar_wait(&sm.sched_full[slot], phase, err, &sm.abort_flag)) return false;
   const int4 v = sm.task[slot];
-  t.e = v.x;
+  t.kind = v.x & 1;
+  t.reuse = (v.x >> 1) & 1;
+  t.e = v.x >> 2;
   t.mt = v.y;
   t.nt = v.z;
   t.rows = v.w;
@@ -128,11 +142,20 @@ __device__ __forceinline__ int ue8m0_exponent(float amax) {
   return (man <= 0x600000u) ? e - 8 : e - 7;
 }
 
-template <bool kFc1, bool kFp4>
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+template <bool kFp4>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                        const __grid_constant__ CUtensorMap tmap_b, const Params p) {
+    moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a1,
+                    const __grid_constant__ CUtensorMap tmap_b1,
+                    const __grid_constant__ CUtensorMap tmap_a2,
+                    const __grid_constant__ CUtensorMap tmap_b2, const Params p) {
   extern __shared__ uint8_t smem_raw[];
+  griddep_launch_dependents();
   Smem& sm = *reinterpret_cast<Smem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5;
@@ -152,8 +175,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int q = 0; q < 4; ++q) mbar_init(&sm.pair[q], 2);
     sm.abort_flag = 0;
     fence_mbarrier_init();
-    tma_prefetch_desc(&tmap_a);
-    tma_prefetch_desc(&tmap_b);
+    if (p.phases & 1) {
+      tma_prefetch_desc(&tmap_a1);
+      tma_prefetch_desc(&tmap_b1);
+    }
+    if (p.phases & 2) {
+      tma_prefetch_desc(&tmap_a2);
+      tma_prefetch_desc(&tmap_b2);
+    }
   }
   if (warp == 1) {
     tmem_alloc(&sm.tmem_base, kTmemCols);
@@ -163,30 +192,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  // Everything above is local set-up that overlaps the previous kernel's tail.
+  griddep_wait();
 
   if (warp == 2) {
     // ------------------------------------------------------------ scheduler
+    // Tile index space: [0, T1) FC1 tiles, [T1, T1 + T2) FC2 tiles, m-tile
+    // major within a phase.  With dynamic scheduling every FC1 tile is handed
+    // out before any FC2 tile, so an FC2 tile only ever waits for FC1 tiles
+    // that running CTAs already own (no deadlock, even if not all CTAs are
+    // resident).
     if (lane == 0) {
       const int total_m = p.tile_off[p.E];
-      const int total = total_m * p.n_tiles;
+      const int T1 = (p.phases & 1) ? total_m * p.ph[0].n_tiles : 0;
+      const int T2 = (p.phases & 2) ? total_m * p.ph[1].n_tiles : 0;
       int slot = 0;
       uint32_t phase = 0;
-      int e = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; ok; tile += gridDim.x) {
-        Task t{-1, 0, 0, 0, 0};
-        if (tile < total) {
-          t.mt = tile / p.n_tiles;
-          t.nt = tile - t.mt * p.n_tiles;
+      int e_cur[2] = {0, 0};
+      for (int i = 0;; ++i) {
+        const int tile = p.dynamic ? static_cast<int>(atomicAdd(p.tile_counter, 1u))
+                                   : static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+        Task t{0, -1, 0, 0, 0, 0, 0};
+        if (tile < T1 + T2) {
+          const int kind = tile < T1 ? 0 : 1;
+          const int local_tile = kind ? tile - T1 : tile;
+          const int nt_n = p.ph[kind].n_tiles;
+          t.kind = kind;
+          t.mt = local_tile / nt_n;
+          t.nt = local_tile - t.mt * nt_n;
+          int& e = e_cur[kind];
+          if (p.tile_off[e] > t.mt) e = 0;   // round-robin order is monotone per phase
           while (p.tile_off[e + 1] <= t.mt) ++e;
           const int local = (t.mt - p.tile_off[e]) * BM;
           t.e = e;
           t.rows = min(BM, p.counts[e] - local);
           t.pos = p.offsets[e] + local;
+          t.reuse = (p.tile_off[e + 1] - p.tile_off[e]) > 1;
         }
-        ok = mbar_wait(&sm.sched_empty[slot], phase ^ 1u, p.err, &sm.abort_flag);
-        if (!ok) break;
-        sm.task[slot] = make_int4(t.e, t.mt, t.nt, t.rows);
+        if (!mbar_wait(&sm.sched_empty[slot], phase ^ 1u, p.err, &sm.abort_flag)) break;
+        sm.task[slot] = make_int4(t.kind | (t.reuse << 1) | (t.e << 2), t.mt, t.nt, t.rows);
         sm.task_pos[slot] = t.pos;
         mbar_arrive(&sm.sched_full[slot]);   // release: the slot's contents are visible
         if (++slot == SCHED_DEPTH) {
@@ -200,30 +244,62 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------- producer
     int slot = 0, stage = 0;
     uint32_t sphase = 0, phase = 0;
+    // A tiles are re-read by every n-tile of their m-tile: keep them in L2.
+    // Weight tiles are re-read only when the expert has several m-tiles;
+    // otherwise they stream through L2 once and go first.
     const uint64_t pol_a = l2_policy_evict_last();
-    const uint64_t pol_b = l2_policy_evict_first();
+    const uint64_t pol_b_once = l2_policy_evict_first();
+    const uint64_t pol_b_reused = l2_policy_evict_normal();
     const uint32_t tx_bytes = BM * BK + (kFp4 ? BN * BK / 2 : BN * BK) + 512;
+    const uint32_t fc1_target = static_cast<uint32_t>(kEpiWarps * p.ph[0].n_tiles);
     Task t;
-    while (get_task(sm, slot, sphase, t, p.err)) {
+    bool aborted = false;
+    while (!aborted && get_task(sm, slot, sphase, t, p.err)) {
       if (t.e < 0) break;
+      const Phase& ph = p.ph[t.kind];
+      const uint64_t pol_b = t.reuse ? pol_b_reused : pol_b_once;
+      const CUtensorMap* ta = t.kind ? &tmap_a2 : &tmap_a1;
+      const CUtensorMap* tb = t.kind ? &tmap_b2 : &tmap_b1;
       // Rows of B for this tile: two 128-row halves.
       int brow0, brow1;
-      if (kFc1) {
-        brow0 = t.e * p.b_rows_per_expert + t.nt * 128;          // gate rows
-        brow1 = brow0 + p.I;                                     // up rows
+      if (t.kind == 0) {
+        brow0 = t.e * ph.b_rows_per_expert + t.nt * 128;          // gate rows
+        brow1 = brow0 + p.I;                                      // up rows
       } else {
-        brow0 = t.e * p.b_rows_per_expert + t.nt * 256;
+        brow0 = t.e * ph.b_rows_per_expert + t.nt * 256;
         brow1 = brow0 + 128;
       }
+      if (t.kind == 1 && (p.phases & 1)) {
+        // FC2 after FC1 in the same launch: wait until every FC1 epilogue warp
+        // of this m-tile has published its rows, then order those generic-proxy
+        // writes before this thread's async-proxy (TMA) reads.
+        if (lane == 0) {
+          const uint32_t* flag = p.fc1_done + t.mt;
+          if (ld_acquire_gpu(flag) < fc1_target) {
+            const uint64_t t0 = globaltimer();
+            while (ld_acquire_gpu(flag) < fc1_target) {
+              if (sm.abort_flag) break;
+              if (globaltimer() - t0 > kDepWaitLimitNs) {
+                atomicOr(p.err, kErrTimeoutBit);
+                sm.abort_flag = 1;
+                break;
+              }
+              __nanosleep(128);
+            }
+          }
+          fence_proxy_async_global();
+        }
+        __syncwarp();
+        if (sm.abort_flag) break;
+      }
       uint32_t sf0 = 0, sf1 = 0;   // FP8 weight scales for k-blocks kb = 32*c + lane
-      bool aborted = false;
-      for (int kb = 0; kb < p.k_blocks; ++kb) {
+      for (int kb = 0; kb < ph.k_blocks; ++kb) {
         if (!kFp4 && (kb & 31) == 0) {
           const int kq = kb + lane;
-          const int kbs = p.k_blocks;
+          const int kbs = ph.k_blocks;
           if (kq < kbs) {
-            sf0 = p.w_sf[static_cast<size_t>(brow0 / 128) * kbs + kq];
-            sf1 = p.w_sf[static_cast<size_t>(brow1 / 128) * kbs + kq];
+            sf0 = ph.w_sf[static_cast<size_t>(brow0 / 128) * kbs + kq];
+            sf1 = ph.w_sf[static_cast<size_t>(brow1 / 128) * kbs + kq];
           }
         }
         if (!mbar_wait(&sm.empty[stage], phase ^ 1u, p.err, &sm.abort_flag)) {
@@ -232,20 +308,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (lane == 0) {
           mbar_arrive_expect_tx(&sm.full[stage], tx_bytes);
-          tma_load_2d(sm.a[stage], &tmap_a, kb * BK, t.mt * BM, &sm.full[stage], pol_a);
-          if (kFc1) {
-            tma_load_2d(sm.b[stage], &tmap_b, kb * BK, brow0, &sm.full[stage], pol_b);
-            tma_load_2d(sm.b[stage] + 128 * BK, &tmap_b, kb * BK, brow1, &sm.full[stage], pol_b);
+          tma_load_2d(sm.a[stage], ta, kb * BK, t.mt * BM, &sm.full[stage], pol_a);
+          if (t.kind == 0) {
+            tma_load_2d(sm.b[stage], tb, kb * BK, brow0, &sm.full[stage], pol_b);
+            tma_load_2d(sm.b[stage] + 128 * BK, tb, kb * BK, brow1, &sm.full[stage], pol_b);
           } else {
-            tma_load_2d(sm.b[stage], &tmap_b, kb * BK, brow0, &sm.full[stage], pol_b);
+            tma_load_2d(sm.b[stage], tb, kb * BK, brow0, &sm.full[stage], pol_b);
           }
           bulk_load(sm.sfa[stage],
-                    p.sfa_chunks + (static_cast<size_t>(t.mt) * p.k_blocks + kb) * 512, 512,
+                    ph.sfa_chunks + (static_cast<size_t>(t.mt) * ph.k_blocks + kb) * 512, 512,
                     &sm.full[stage]);
         }
         if (kFp4) {
           // One 32-bit word = the four 1x32 scales of this 128-wide k-block.
-          const int kw = p.k_blocks * 4;   // scale bytes per weight row
+          const int kw = ph.k_blocks * 4;   // scale bytes per weight row
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             const int rb = c ? brow1 : brow0;
@@ -253,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int q = 0; q < 4; ++q) {
               const int r = lane + 32 * q;
               cp_async_4(sm.sfb[stage] + c * 512 + lane * 16 + q * 4,
-                         p.w_sf + static_cast<size_t>(rb + r) * kw + kb * 4);
+                         ph.w_sf + static_cast<size_t>(rb + r) * kw + kb * 4);
             }
           }
           cp_async_mbar_arrive_noinc(&sm.full[stage]);
@@ -270,19 +346,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           phase ^= 1u;
         }
       }
-      if (aborted) break;
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     int slot = 0, stage = 0;
     uint32_t sphase = 0, phase = 0, acc_phase = 0;
     Task t;
-    while (get_task(sm, slot, sphase, t, p.err)) {
+    bool aborted = false;
+    while (!aborted && get_task(sm, slot, sphase, t, p.err)) {
       if (t.e < 0) break;
       if (!mbar_wait(&sm.tmem_empty, acc_phase ^ 1u, p.err, &sm.abort_flag)) break;
       tc_fence_after();
-      bool aborted = false;
-      for (int kb = 0; kb < p.k_blocks; ++kb) {
+      const int k_blocks = p.ph[t.kind].k_blocks;
+      for (int kb = 0; kb < k_blocks; ++kb) {
         if (!mbar_wait(&sm.full[stage], phase, p.err, &sm.abort_flag)) {
           aborted = true;
           break;
@@ -331,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (t.e < 0) break;
       if (!mbar_wait(&sm.tmem_full, acc_phase, p.err, &sm.abort_flag)) break;
       tc_fence_after();
-      if (kFc1) {
+      if (t.kind == 0) {
         uint32_t g[64], u[64];
         tmem_ld_32x32b_x32(t_row + kAccCol + half * 64, *reinterpret_cast<uint32_t(*)[32]>(g));
         tmem_ld_32x32b_x32(t_row + kAccCol + half * 64 + 32,
@@ -399,6 +475,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int v = 0; v < 16; ++v)
             fd[v] = make_float4(__uint_as_float(g[4 * v]), __uint_as_float(g[4 * v + 1]),
                                 __uint_as_float(g[4 * v + 2]), __uint_as_float(g[4 * v + 3]));
+        }
+        if (p.phases & 2) {
+          // Publish this warp's rows to FC2 tiles of the same launch: make the
+          // stores visible at GPU scope, then count this warp as done.
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) atomicAdd(p.fc1_done + t.mt, 1u);
         }
       } else {
         uint32_t v[128];
@@ -485,33 +568,44 @@ int num_sms() {
   return n;
 }
 
-template <bool kFc1, bool kFp4>
-cudaError_t launch_gemm(const moe_plan_s* pl, const void* w, const uint8_t* wsf, uint8_t* ws,
+template <bool kFp4>
+cudaError_t launch_gemm(const moe_plan_s* pl, int phases, bool dynamic, const void* w1,
+                        const uint8_t* w1s, const void* w2, const uint8_t* w2s, uint8_t* ws,
                         cudaStream_t st) {
   const auto& L = pl->ws;
-  const int K = kFc1 ? pl->H : pl->I;
-  const int brows = kFc1 ? 2 * pl->I : pl->H;
-  CUtensorMap ta, tb;
-  const uint8_t* a_base = kFc1 ? ws + L.xg : ws + L.act;
-  if (!make_map(&ta, a_base, K, pl->rows_cap, K, 128, false)) return cudaErrorInvalidValue;
-  const uint64_t b_rows_total = static_cast<uint64_t>(pl->E) * brows;
-  if (!make_map(&tb, w, K, b_rows_total, kFp4 ? K / 2 : K, kFc1 ? 128 : 256, kFp4))
-    return cudaErrorInvalidValue;
+  CUtensorMap maps[4];
+  std::memset(maps, 0, sizeof(maps));
   Params p{};
   p.E = pl->E;
-  p.n_tiles = kFc1 ? pl->I / 128 : pl->H / 256;
-  p.k_blocks = K / 128;
-  p.b_rows_per_expert = brows;
   p.I = pl->I;
   p.H = pl->H;
-  p.fp4 = kFp4;
-  p.fc1 = kFc1;
+  p.phases = phases;
+  p.dynamic = dynamic ? 1 : 0;
+  long long max_tiles = 0;
+  if (phases & 1) {
+    const int K = pl->H;
+    if (!make_map(&maps[0], ws + L.xg, K, pl->rows_cap, K, 128, false) ||
+        !make_map(&maps[1], w1, K, static_cast<uint64_t>(pl->E) * 2 * pl->I, kFp4 ? K / 2 : K,
+                  128, kFp4))
+      return cudaErrorInvalidValue;
+    p.ph[0] = Phase{pl->I / 128, K / 128, 2 * pl->I, ws + L.xg_sf, w1s};
+    max_tiles += (pl->rows_cap / BM) * p.ph[0].n_tiles;
+  }
+  if (phases & 2) {
+    const int K = pl->I;
+    if (!make_map(&maps[2], ws + L.act, K, pl->rows_cap, K, 128, false) ||
+        !make_map(&maps[3], w2, K, static_cast<uint64_t>(pl->E) * pl->H, kFp4 ? K / 2 : K, 256,
+                  kFp4))
+      return cudaErrorInvalidValue;
+    p.ph[1] = Phase{pl->H / 256, K / 128, pl->H, ws + L.act_sf, w2s};
+    max_tiles += (pl->rows_cap / BM) * p.ph[1].n_tiles;
+  }
   p.tile_off = reinterpret_cast<const int32_t*>(ws + L.tile_off);
   p.counts = reinterpret_cast<const int32_t*>(ws + L.counts);
   p.offsets = reinterpret_cast<const int32_t*>(ws + L.offsets);
   p.perm = reinterpret_cast<const int32_t*>(ws + L.perm);
-  p.sfa_chunks = kFc1 ? ws + L.xg_sf : ws + L.act_sf;
-  p.w_sf = wsf;
+  p.tile_counter = reinterpret_cast<uint32_t*>(ws + L.sched);
+  p.fc1_done = reinterpret_cast<uint32_t*>(ws + L.sched) + 64;
   p.act = ws + L.act;
   p.act_sf_chunks = ws + L.act_sf;
   p.act_f32 = pl->debug_act_f32 ? reinterpret_cast<float*>(ws + L.act_f32) : nullptr;
@@ -522,7 +616,7 @@ cudaError_t launch_gemm(const moe_plan_s* pl, const void* w, const uint8_t* wsf,
   p.y = reinterpret_cast<uint16_t*>(ws + L.y);
   p.err = reinterpret_cast<uint32_t*>(ws + L.err);
   const size_t smem = sizeof(Smem) + 1024;
-  auto kern = grouped_gemm_kernel<kFc1, kFp4>;
+  auto kern = moe_gemm_kernel<kFp4>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e =
@@ -530,10 +624,9 @@ cudaError_t launch_gemm(const moe_plan_s* pl, const void* w, const uint8_t* wsf,
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const long long max_tiles = (pl->rows_cap / BM) * p.n_tiles;
   const int grid = static_cast<int>(std::min<long long>(num_sms(), max_tiles));
-  kern<<<grid, kThreads, smem, st>>>(ta, tb, p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, maps[0], maps[1], maps[2],
+                    maps[3], p);
 }
 
 }  // namespace
@@ -542,14 +635,23 @@ size_t gemm_smem_bytes() { return sizeof(Smem) + 1024; }
 
 cudaError_t launch_fc1(const moe_plan_s* p, const void* w1, const uint8_t* w1s, uint8_t* ws,
                        cudaStream_t st) {
-  if (p->w_dtype == MOE_W_E2M1_UE8M0_1x32) return launch_gemm<true, true>(p, w1, w1s, ws, st);
-  return launch_gemm<true, false>(p, w1, w1s, ws, st);
+  if (p->w_dtype == MOE_W_E2M1_UE8M0_1x32)
+    return launch_gemm<true>(p, 1, false, w1, w1s, nullptr, nullptr, ws, st);
+  return launch_gemm<false>(p, 1, false, w1, w1s, nullptr, nullptr, ws, st);
 }
 
 cudaError_t launch_fc2(const moe_plan_s* p, const void* w2, const uint8_t* w2s, uint8_t* ws,
                        cudaStream_t st) {
-  if (p->w_dtype == MOE_W_E2M1_UE8M0_1x32) return launch_gemm<false, true>(p, w2, w2s, ws, st);
-  return launch_gemm<false, false>(p, w2, w2s, ws, st);
+  if (p->w_dtype == MOE_W_E2M1_UE8M0_1x32)
+    return launch_gemm<true>(p, 2, false, nullptr, nullptr, w2, w2s, ws, st);
+  return launch_gemm<false>(p, 2, false, nullptr, nullptr, w2, w2s, ws, st);
+}
+
+cudaError_t launch_fc12(const moe_plan_s* p, const void* w1, const uint8_t* w1s, const void* w2,
+                        const uint8_t* w2s, uint8_t* ws, cudaStream_t st) {
+  if (p->w_dtype == MOE_W_E2M1_UE8M0_1x32)
+    return launch_gemm<true>(p, 3, true, w1, w1s, w2, w2s, ws, st);
+  return launch_gemm<false>(p, 3, true, w1, w1s, w2, w2s, ws, st);
 }
 
 }  // namespace moe

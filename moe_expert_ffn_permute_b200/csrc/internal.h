@@ -3,6 +3,7 @@
 #pragma once
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -18,7 +19,9 @@ constexpr int kTileM = 128;          // rows per m-tile (expert blocks are padde
 struct WorkspaceLayout {
   size_t err, counts, offsets, pad_off, tile_off;
   size_t block_hist;
+  size_t sched;             // fused-GEMM tile counter + per-m-tile FC1 completion counts
   size_t perm, inv;
+  size_t row_token;         // padded row -> token index (-1 for padding rows)
   size_t xg, xg_sf;         // gathered x (expert order, padded) + its scale chunks
   size_t act, act_sf;       // FC1 output: FP8 activation + scale chunks
   size_t act_f32;           // debug capture (0 bytes when off)
@@ -45,6 +48,25 @@ namespace moe {
 
 void compute_layout(moe_plan_s* p);
 
+// Launch with programmatic stream serialization: the kernel may start while its
+// predecessor in the stream finishes; it must execute griddep_wait() before
+// touching memory the predecessor writes or reads.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Kernel launchers (return cudaGetLastError()).
 cudaError_t launch_route(const moe_plan_s* p, const int32_t* topk_idx, uint8_t* ws,
                          cudaStream_t st);
@@ -54,6 +76,9 @@ cudaError_t launch_fc1(const moe_plan_s* p, const void* w1, const uint8_t* w1s, 
                        cudaStream_t st);
 cudaError_t launch_fc2(const moe_plan_s* p, const void* w2, const uint8_t* w2s, uint8_t* ws,
                        cudaStream_t st);
+// FC1 and FC2 in one persistent launch (dynamic tile scheduler).
+cudaError_t launch_fc12(const moe_plan_s* p, const void* w1, const uint8_t* w1s, const void* w2,
+                        const uint8_t* w2s, uint8_t* ws, cudaStream_t st);
 cudaError_t launch_combine(const moe_plan_s* p, const float* topk_w, void* out, uint8_t* ws,
                            cudaStream_t st);
 cudaError_t launch_unpack_act_scales(const moe_plan_s* p, const uint8_t* ws, uint8_t* dst,

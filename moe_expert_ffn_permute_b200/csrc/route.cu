@@ -27,6 +27,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_hist_kernel(
     uint32_t* err) {
   __shared__ int32_t hist[256];
   const int tid = threadIdx.x;
+  griddep_launch_dependents();
+  griddep_wait();
   for (int e = tid; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
   const int base = blockIdx.x * kRouteChunk;
@@ -59,11 +61,19 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
     const int32_t* __restrict__ idx, int S, int E, int nblk,
     const int32_t* __restrict__ block_hist, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ tile_off, int32_t* __restrict__ pad_off,
-    int32_t* __restrict__ perm, int32_t* __restrict__ inv, uint32_t* err) {
+    int32_t* __restrict__ perm, int32_t* __restrict__ inv, uint32_t* err,
+    uint32_t* __restrict__ sched, int sched_words, int32_t* __restrict__ row_token, int k) {
   constexpr int kWarps = kRouteThreads / 32;
+  griddep_launch_dependents();
+  griddep_wait();
+  // Block 0 also zeroes the fused GEMM's tile counter and per-m-tile
+  // completion counts (sched may be null when no GEMM follows).
+  if (blockIdx.x == 0 && sched != nullptr)
+    for (int i = threadIdx.x; i < sched_words; i += blockDim.x) sched[i] = 0u;
   __shared__ int32_t running[256];
   __shared__ int32_t total[256];
   __shared__ int32_t scan[257];
+  __shared__ int32_t tscan[257];   // padded m-tile offsets
   __shared__ int32_t wcount[kWarps][256];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (nblk == 1) {
@@ -96,6 +106,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
     int acc = 0, tacc = 0;
     for (int e = 0; e < E; ++e) {
       scan[e] = acc;
+      tscan[e] = tacc;
       if (blockIdx.x == 0) {
         offsets[e] = acc;
         counts[e] = total[e];
@@ -106,6 +117,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
       tacc += (total[e] + kTileM - 1) / kTileM;
     }
     scan[E] = acc;
+    tscan[E] = tacc;
     if (blockIdx.x == 0) {
       offsets[E] = acc;
       tile_off[E] = tacc;
@@ -114,6 +126,13 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
   }
   __syncthreads();
   for (int e = tid; e < E; e += blockDim.x) running[e] += scan[e];
+  // Padding rows of the row -> token map read -1 (experts split over blocks).
+  if (row_token != nullptr) {
+    for (int e = blockIdx.x; e < E; e += gridDim.x) {
+      const int lo = tscan[e] * kTileM + total[e], hi = tscan[e + 1] * kTileM;
+      for (int r = lo + tid; r < hi; r += blockDim.x) row_token[r] = -1;
+    }
+  }
   // Positions past the routed slots (left by out-of-range ids) read -1.
   const int routed = scan[E];
   const int base = blockIdx.x * kRouteChunk;
@@ -139,6 +158,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
         if (pos >= 0 && pos < S) {   // always true; guards the store
           perm[pos] = s;
           inv[s] = pos;
+          if (row_token != nullptr) row_token[tscan[e] * kTileM + (pos - scan[e])] = s / k;
         } else {
           atomicOr(err, kErrRoutingBit);
           inv[s] = -1;
@@ -168,25 +188,18 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
 constexpr int kGatherWarps = 8;
 
 __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(
-    const uint8_t* __restrict__ x, const uint8_t* __restrict__ xs, int H, int k, int E,
-    const int32_t* __restrict__ tile_off, const int32_t* __restrict__ counts,
-    const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm,
+    const uint8_t* __restrict__ x, const uint8_t* __restrict__ xs, int H, int E,
+    const int32_t* __restrict__ pad_off, const int32_t* __restrict__ row_token,
     uint8_t* __restrict__ xg, uint8_t* __restrict__ xg_sf) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long P = static_cast<long long>(blockIdx.x) * kGatherWarps + warp;
+  if (P >= __ldg(&pad_off[E])) return;
+  const int t = __ldg(&row_token[P]);
+  if (t < 0) return;   // padding row
   const int tile = static_cast<int>(P / kTileM);
   const int r = static_cast<int>(P % kTileM);
-  if (tile >= __ldg(&tile_off[E])) return;
-  int lo = 0, hi = E;   // the expert owning the tile: last e with tile_off[e] <= tile
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(&tile_off[mid]) <= tile) lo = mid; else hi = mid;
-  }
-  while (lo + 1 <= E && __ldg(&tile_off[lo + 1]) <= tile) ++lo;
-  const int e = lo;
-  const int local = (tile - __ldg(&tile_off[e])) * kTileM + r;
-  if (local >= __ldg(&counts[e])) return;
-  const int t = __ldg(&perm[__ldg(&offsets[e]) + local]) / k;
   const int vec = H / 16;
   const uint4* __restrict__ src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
   uint4* __restrict__ dst = reinterpret_cast<uint4*>(xg + static_cast<size_t>(P) * H);
@@ -217,29 +230,31 @@ cudaError_t launch_route(const moe_plan_s* p, const int32_t* topk_idx, uint8_t* 
                          cudaStream_t st) {
   const auto& L = p->ws;
   const int S = static_cast<int>(p->S);
-  if (p->route_blocks > 1)
-    route_hist_kernel<<<p->route_blocks, kRouteThreads, 0, st>>>(
-        topk_idx, S, p->E, reinterpret_cast<int32_t*>(ws + L.block_hist),
-        reinterpret_cast<uint32_t*>(ws + L.err));
-  route_scatter_kernel<<<p->route_blocks, kRouteThreads, 0, st>>>(
-      topk_idx, S, p->E, p->route_blocks, reinterpret_cast<const int32_t*>(ws + L.block_hist),
+  if (p->route_blocks > 1) {
+    cudaError_t e = launch_pdl(route_hist_kernel, dim3(p->route_blocks), dim3(kRouteThreads), 0,
+                               st, topk_idx, S, p->E,
+                               reinterpret_cast<int32_t*>(ws + L.block_hist),
+                               reinterpret_cast<uint32_t*>(ws + L.err));
+    if (e != cudaSuccess) return e;
+  }
+  return launch_pdl(
+      route_scatter_kernel, dim3(p->route_blocks), dim3(kRouteThreads), 0, st, topk_idx, S,
+      p->E, p->route_blocks, reinterpret_cast<const int32_t*>(ws + L.block_hist),
       reinterpret_cast<int32_t*>(ws + L.counts), reinterpret_cast<int32_t*>(ws + L.offsets),
       reinterpret_cast<int32_t*>(ws + L.tile_off), reinterpret_cast<int32_t*>(ws + L.pad_off),
       reinterpret_cast<int32_t*>(ws + L.perm), reinterpret_cast<int32_t*>(ws + L.inv),
-      reinterpret_cast<uint32_t*>(ws + L.err));
-  return cudaGetLastError();
+      reinterpret_cast<uint32_t*>(ws + L.err), reinterpret_cast<uint32_t*>(ws + L.sched),
+      static_cast<int>(64 + p->rows_cap / kTileM), reinterpret_cast<int32_t*>(ws + L.row_token),
+      p->k);
 }
 
 cudaError_t launch_gather(const moe_plan_s* p, const uint8_t* x, const uint8_t* xs, uint8_t* ws,
                           cudaStream_t st) {
   const auto& L = p->ws;
   const int blocks = static_cast<int>(p->rows_cap / kGatherWarps);
-  gather_kernel<<<blocks, kGatherWarps * 32, 0, st>>>(
-      x, xs, p->H, p->k, p->E, reinterpret_cast<const int32_t*>(ws + L.tile_off),
-      reinterpret_cast<const int32_t*>(ws + L.counts),
-      reinterpret_cast<const int32_t*>(ws + L.offsets),
-      reinterpret_cast<const int32_t*>(ws + L.perm), ws + L.xg, ws + L.xg_sf);
-  return cudaGetLastError();
+  return launch_pdl(gather_kernel, dim3(blocks), dim3(kGatherWarps * 32), 0, st, x, xs, p->H,
+                    p->E, reinterpret_cast<const int32_t*>(ws + L.pad_off),
+                    reinterpret_cast<const int32_t*>(ws + L.row_token), ws + L.xg, ws + L.xg_sf);
 }
 
 cudaError_t launch_unpack_act_scales(const moe_plan_s* p, const uint8_t* ws, uint8_t* dst,
@@ -334,6 +349,7 @@ extern "C" moe_status moe_route_static(const int32_t* topk_idx, int T, int k, in
   route_scatter_kernel<<<nblk, kRouteThreads, 0, st>>>(
       topk_idx, static_cast<int>(S), E, nblk, hist, counts, offsets,
       reinterpret_cast<int32_t*>(scratch + kStaticTileOff),
-      reinterpret_cast<int32_t*>(scratch + kStaticPadOff), perm, inv, err);
+      reinterpret_cast<int32_t*>(scratch + kStaticPadOff), perm, inv, err, nullptr, 0, nullptr,
+      k);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

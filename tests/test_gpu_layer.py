@@ -133,3 +133,32 @@ def test_layer_parity_full_size_sampled(name, T, ntok):
     dn = {k: v.cpu().numpy() for k, v in d.items()}
     ref = oracle_tokens(wl, dn, tokens)
     assert_parity(out.float().cpu().numpy()[tokens], ref, wl.name)
+
+
+def test_cuda_graph_replay_is_bitwise_identical():
+    """moe_forward captured once in a CUDA graph and replayed: every replay
+    recomputes routing and resets the GEMM scheduler's counters in-graph, so
+    each replay equals the eager result bit for bit (also after the inputs'
+    routing changes in place between replays)."""
+    wl = RAGGED
+    d = inputs(wl)
+    eager, lay = run_gpu(wl, d)
+    out = torch.empty_like(eager)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        moe.moe_forward(lay.plan, d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], d["w1"],
+                        d["w1_scales"], d["w2"], d["w2_scales"], out, lay.workspace,
+                        torch.cuda.current_stream())
+    for _ in range(3):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, eager)
+    # new routing in the same buffers: the replay follows it
+    d2 = inputs(wl, seed=777)
+    d["topk_idx"].copy_(d2["topk_idx"])
+    d["topk_w"].copy_(d2["topk_w"])
+    g.replay()
+    torch.cuda.synchronize()
+    ref2, _ = run_gpu(wl, d)
+    assert torch.equal(out, ref2)
