@@ -29,7 +29,7 @@ def _declared():
 
 def test_header_declares_entry_points():
     names = _declared()
-    for n in ("moe_plan", "moe_forward", "moe_route", "moe_gather", "moe_fc1", "moe_fc2", "moe_combine",
+    for n in ("moe_plan", "moe_forward", "moe_route", "moe_gather", "moe_fc1_fc2", "moe_fc1", "moe_fc2", "moe_combine",
               "moe_workspace_bytes", "moe_check_device_error", "moe_plan_destroy",
               "moe_status_str"):
         assert n in names

@@ -17,7 +17,7 @@ RAGGED = Workload("ragged", 300, 1024, 512, 8, 4, cfg_id=20)
 RAGGED_FP4 = Workload("ragged-fp4", 300, 1024, 512, 8, 4, w_dtype="e2m1", cfg_id=21)
 RAGGED_OAI = Workload("ragged-oai", 200, 512, 384, 6, 3, act="swiglu_oai", alpha=1.702,
                       up_bias=1.0, limit=7.0, cfg_id=22)
-SINGLE = Workload("single", 1, 256, 128, 1, 1, cfg_id=23)
+SINGLE = Workload("single", 1, 512, 128, 1, 1, cfg_id=23)
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -101,6 +101,30 @@ def test_step_calls_equal_forward():
     moe.moe_combine(lay.plan, d["topk_w"], out, lay.workspace)
     torch.cuda.synchronize()
     assert torch.equal(out, full)
+
+
+def test_fused_gemm_step_equals_separate_gemms():
+    """FC1 and FC2 in one persistent launch (dynamic scheduler, per-m-tile
+    dependency counters) give the same bytes as two separate launches."""
+    for wl in (RAGGED, RAGGED_FP4):
+        d = inputs(wl)
+        _, lay = run_gpu(wl, d)
+        v = lay.view()
+        n = wl.T * wl.k * wl.H * 2
+        off = v.y - lay.workspace.data_ptr()
+        moe.moe_route(lay.plan, d["topk_idx"], lay.workspace)
+        moe.moe_gather(lay.plan, d["x"], d["x_scales"], lay.workspace)
+        moe.moe_fc1(lay.plan, d["w1"], d["w1_scales"], lay.workspace)
+        moe.moe_fc2(lay.plan, d["w2"], d["w2_scales"], lay.workspace)
+        torch.cuda.synchronize()
+        y_sep = lay.workspace[off:off + n].clone()
+        lay.workspace[off:off + n].zero_()
+        moe.moe_route(lay.plan, d["topk_idx"], lay.workspace)
+        moe.moe_gather(lay.plan, d["x"], d["x_scales"], lay.workspace)
+        moe.moe_fc1_fc2(lay.plan, d["w1"], d["w1_scales"], d["w2"], d["w2_scales"],
+                        lay.workspace)
+        torch.cuda.synchronize()
+        assert torch.equal(lay.workspace[off:off + n], y_sep), wl.name
 
 
 def test_hostio_equals_device_forward():

@@ -14,7 +14,7 @@ pytestmark = pytest.mark.gpu
 
 def _route_gpu(T, k, E, idx):
     ensure_built()
-    plan = moe.moe_plan(T, 256, 128, E, k)
+    plan = moe.moe_plan(T, 512, 128, E, k)
     ws = torch.empty(moe.moe_workspace_bytes(plan), dtype=torch.uint8, device="cuda")
     moe.moe_clear_device_error(plan, ws)
     d_idx = torch.from_numpy(idx.astype(np.int32)).cuda()

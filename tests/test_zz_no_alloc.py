@@ -20,7 +20,7 @@ pytestmark = pytest.mark.gpu
 
 
 def _workspace_route(idx, T, k, E):
-    plan = moe.moe_plan(T, 256, 128, E, k)
+    plan = moe.moe_plan(T, 512, 128, E, k)
     ws = torch.empty(moe.moe_workspace_bytes(plan), dtype=torch.uint8, device="cuda")
     moe.moe_route(plan, idx, ws)
     v = moe.moe_workspace_view(plan, ws)
