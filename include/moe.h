@@ -32,10 +32,11 @@
  *   - Errors are returned as moe_status; nothing is thrown across the ABI.
  *     Argument validation happens before anything is enqueued: a call that
  *     returns an error has launched nothing.
- *   - Device-side problems (an expert id outside [0,E), a bounded wait that ran
+ *   - Masked slots: topk_idx = -1 marks a slot that is not routed (it
+ *     contributes nothing to its token's output); this is not an error.
+ *   - Device-side problems (an expert id >= E or < -1, a bounded wait that ran
  *     out) are recorded in an error word inside the workspace; read it with
- *     moe_check_device_error().  A slot with an out-of-range expert id is not
- *     routed: it contributes nothing to its token's output.
+ *     moe_check_device_error().  A slot with such an id is not routed either.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream) unless stated otherwise.  Calls with different plans or
  *     different workspaces may run concurrently; two calls sharing one
@@ -178,6 +179,17 @@ moe_status moe_fc1_fc2(moe_plan_t plan, const void *w1, const uint8_t *w1_scales
  * Sources: DeepGEMM PR #386 title ("direct combine").                        */
 moe_status moe_combine(moe_plan_t plan, const float *topk_w, void *out,
                        void *workspace, moe_stream_t stream);
+
+/* The step before the layer: quantise bf16 activations x_bf16 [T,H] (device)
+ * to the layer's input format -- E4M3 codes x_codes u8 [T,H] and one UE8M0
+ * scale byte per 1x128 block x_scales u8 [T,H/128] -- with the rule the FC1
+ * epilogue uses for the activation: n = smallest integer with
+ * max(amax, 1e-4) <= 448 * 2^n, codes = round-to-nearest-even saturating E4M3
+ * of x / 2^n, scale byte n + 127 (TensorRT-LLM PR #16346 "DSV4 o_proj: fuse
+ * fp8/UE8M0 quantize ...", Description).  Inputs must be finite.  H % 128 == 0,
+ * x_bf16 16-byte and x_codes 8-byte aligned.  Needs no plan or workspace.   */
+moe_status moe_quantize_act(const void *x_bf16, int T, int H, uint8_t *x_codes,
+                            uint8_t *x_scales, moe_stream_t stream);
 
 /* Allocation-free routing.  The pages have no counterpart of this entry point.
  *

@@ -54,6 +54,7 @@ _SIGS = {
     "moe_forward": (ctypes.c_int, [_P] * 12),
     "moe_forward_hostio": (ctypes.c_int, [_P] * 12),
     "moe_route": (ctypes.c_int, [_P] * 4),
+    "moe_quantize_act": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int, _P, _P, _P]),
     "moe_route_static": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int] + [_P] * 5),
     "moe_gather": (ctypes.c_int, [_P] * 5),
     "moe_fc1": (ctypes.c_int, [_P] * 5),
@@ -156,6 +157,12 @@ def moe_forward_hostio(plan, x_host, x_scales_host, topk_idx_host, topk_w_host, 
 
 def moe_route(plan, topk_idx, workspace, stream=None):
     _check(lib().moe_route(plan, _ptr(topk_idx), _ptr(workspace), _stream(stream)), "moe_route")
+
+
+def moe_quantize_act(x_bf16, T, H, x_codes, x_scales, stream=None):
+    """bf16 [T,H] -> E4M3 codes [T,H] + UE8M0 scales [T,H/128] (device buffers)."""
+    _check(lib().moe_quantize_act(_ptr(x_bf16), T, H, _ptr(x_codes), _ptr(x_scales),
+                                  _stream(stream)), "moe_quantize_act")
 
 
 def moe_route_static(topk_idx, T, k, E, counts, offsets, perm, inv, stream=None):

@@ -130,16 +130,10 @@ __device__ __forceinline__ bool get_task(Smem& sm, int& slot, uint32_t& phase, T
   return true;
 }
 
-__device__ __forceinline__ float sigmoidf_fast(float z) { return __frcp_rn(1.0f + __expf(-z)); }
-
-// Smallest n with amax <= 448 * 2^n, from the fp32 bits (448 = 1.75 * 2^8):
-// amax = m * 2^e with m in [1, 2): n = e - 8 if m <= 1.75, else e - 7.
-__device__ __forceinline__ int ue8m0_exponent(float amax) {
-  amax = fmaxf(amax, 1e-4f);
-  const uint32_t bits = __float_as_uint(amax);
-  const int e = static_cast<int>((bits >> 23) & 0xFF) - 127;
-  const uint32_t man = bits & 0x7FFFFF;
-  return (man <= 0x600000u) ? e - 8 : e - 7;
+// sigmoid(z) with the fast exponential and an approximate reciprocal (the
+// epilogue's transcendental pipe is shared by the E4M3 / bf16 conversions).
+__device__ __forceinline__ float sigmoidf_fast(float z) {
+  return __fdividef(1.0f, 1.0f + __expf(-z));
 }
 
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {

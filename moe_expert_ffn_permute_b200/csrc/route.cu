@@ -21,6 +21,11 @@
 namespace moe {
 namespace {
 
+// An expert id of -1 marks a masked slot: it is skipped without an error (the
+// masked / unmasked sweeps of DeepGEMM PR #386's Description); any other id
+// outside [0, E) is skipped and reported as MOE_ERR_BAD_ROUTING.
+constexpr int kMaskedSlot = -1;
+
 // Kernel 1: per-block histograms of the block's kRouteChunk slots.
 __global__ void __launch_bounds__(kRouteThreads) route_hist_kernel(
     const int32_t* __restrict__ idx, int S, int E, int32_t* __restrict__ block_hist,
@@ -39,7 +44,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_hist_kernel(
       const int e = idx[s];
       if (e >= 0 && e < E) {
         atomicAdd(&hist[e], 1);
-      } else {
+      } else if (e != kMaskedSlot) {
         bad = true;
       }
     }
@@ -86,7 +91,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
     bool bad = false;
     for (int s = tid; s < S; s += blockDim.x) {
       const int e = idx[s];
-      if (e >= 0 && e < E) atomicAdd(&total[e], 1); else bad = true;
+      if (e >= 0 && e < E) atomicAdd(&total[e], 1); else if (e != kMaskedSlot) bad = true;
     }
     if (bad) atomicOr(err, kErrRoutingBit);
   } else {

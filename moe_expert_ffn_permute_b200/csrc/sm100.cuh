@@ -264,6 +264,17 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 
 // ------------------------------------------------------------- conversions
+// UE8M0 exponent of a 1x128 block: the smallest n with max(amax, 1e-4) <=
+// 448 * 2^n, read off the fp32 bits (448 = 1.75 * 2^8): with amax = m * 2^e,
+// m in [1, 2), n = e - 8 if m <= 1.75, else e - 7.
+__device__ __forceinline__ int ue8m0_exponent(float amax) {
+  amax = fmaxf(amax, 1e-4f);
+  const uint32_t bits = __float_as_uint(amax);
+  const int e = static_cast<int>((bits >> 23) & 0xFF) - 127;
+  const uint32_t man = bits & 0x7FFFFF;
+  return (man <= 0x600000u) ? e - 8 : e - 7;
+}
+
 // Two fp32 -> two E4M3 bytes, round to nearest even, saturating; `lo` goes to
 // the low byte (the lower address).
 __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {

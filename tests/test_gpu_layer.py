@@ -89,6 +89,17 @@ def test_out_of_range_ids_contribute_nothing():
     assert_parity(out.float().cpu().numpy(), ref, "bad ids")
 
 
+def test_masked_slots_contribute_nothing_and_are_not_errors():
+    wl = RAGGED
+    d = inputs(wl)
+    mask = torch.rand(wl.T, wl.k, device="cuda") < 0.25
+    d["topk_idx"][mask] = -1
+    out, lay = run_gpu(wl, d)
+    assert lay.check() == 0
+    ref = L.layer(*oracle_args(to_numpy(d)), **oracle_kw(wl))
+    assert_parity(out.float().cpu().numpy(), ref, "masked")
+
+
 def test_step_calls_equal_forward():
     wl = RAGGED_OAI
     d = inputs(wl)

@@ -84,3 +84,15 @@ def test_route_is_repeatable():
     b, _ = _route_gpu(8192, 8, 32, idx)
     for key in a:
         np.testing.assert_array_equal(a[key], b[key])
+
+
+def test_route_masked_slots_are_not_errors():
+    rng = np.random.default_rng(19)
+    T, k, E = 513, 4, 16
+    idx = np.stack([rng.choice(E, k, replace=False) for _ in range(T)])
+    idx[rng.random((T, k)) < 0.2] = -1          # masked slots
+    got, status = _route_gpu(T, k, E, idx)
+    counts, offsets, perm, inv = L.route(idx, E)
+    np.testing.assert_array_equal(got["perm"], perm)
+    np.testing.assert_array_equal(got["inv"], inv)
+    assert status == 0
