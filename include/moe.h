@@ -226,7 +226,8 @@ typedef struct {
   int32_t *perm;        /* [S]                                        */
   int32_t *inv;         /* [S]                                        */
   int32_t *pad_offsets; /* [E+1]  row offsets, multiples of 128       */
-  uint8_t *act;         /* [rows, I]  FP8 E4M3 activation (FC1 output) */
+  uint8_t *act;         /* FP8 E4M3 activation (FC1 output), tiled:
+                           read it row-major with moe_copy_act()      */
   float *act_f32;       /* [rows, I]  the activation before requant,
                            written only when debug capture is on      */
   uint16_t *y;          /* [S, H] bf16, slot order (FC2 output)       */
@@ -243,6 +244,31 @@ moe_status moe_workspace_view(moe_plan_t plan, void *workspace,
  * (device pointer `dst`), enqueued on `stream`.                              */
 moe_status moe_copy_act_scales(moe_plan_t plan, const void *workspace,
                                uint8_t *dst, moe_stream_t stream);
+
+/* Weight layout.  MOE_WEIGHTS_ROW_MAJOR (default): W1/W2 as described at
+ * moe_forward, read by 2-D TMA tiles.  MOE_WEIGHTS_TILED: W1/W2 are the output
+ * of moe_prepack_weights() -- the same bytes rearranged into 128 x 128-byte
+ * tiles that the tensor cores consume directly, streamed by linear bulk copies
+ * (faster; FP8 weights only, MOE_ERR_UNSUPPORTED for MXFP4).  Weight scales
+ * keep their layout in both cases.                                          */
+typedef enum { MOE_WEIGHTS_ROW_MAJOR = 0, MOE_WEIGHTS_TILED = 1 } moe_weight_layout;
+moe_status moe_plan_set_weight_layout(moe_plan_t plan, int layout);
+
+/* Rearrange row-major FP8 weights w1 [E,2I,H] and w2 [E,H,I] (device) into
+ * the tiled layout (w1_tiled, w2_tiled: device buffers of the same sizes,
+ * 16-byte aligned; must not overlap the inputs).  Tile (b, kb) -- rows
+ * 128b..128b+127 of the [E*2I, H] (or [E*H, I]) matrix, bytes 128kb..128kb+127
+ * of each row -- is 16384 bytes at offset (b * K/128 + kb) * 16384, and byte c
+ * of tile row r lies at r*128 + ((c/16) XOR (r%8))*16 + c%16.  Done once per
+ * weight set (e.g. at model load), enqueued on `stream`.                    */
+moe_status moe_prepack_weights(moe_plan_t plan, const void *w1, const void *w2,
+                               void *w1_tiled, void *w2_tiled, moe_stream_t stream);
+
+/* Copy the FC1 activation codes out of the workspace as a row-major u8
+ * [rows, I] array (device pointer `dst`, 16-byte aligned), enqueued on
+ * `stream`; inside the workspace they are kept in the tiled layout.        */
+moe_status moe_copy_act(moe_plan_t plan, const void *workspace, uint8_t *dst,
+                        moe_stream_t stream);
 
 /* Debug capture: when on, moe_fc1 also writes the fp32 activation before
  * requantisation to act_f32 (costs bandwidth; off by default).              */

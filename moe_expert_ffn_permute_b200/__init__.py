@@ -64,6 +64,9 @@ _SIGS = {
     "moe_workspace_view": (ctypes.c_int, [_P, _P, ctypes.POINTER(WorkspaceView)]),
     "moe_copy_act_scales": (ctypes.c_int, [_P] * 4),
     "moe_plan_set_debug": (ctypes.c_int, [_P, ctypes.c_int]),
+    "moe_plan_set_weight_layout": (ctypes.c_int, [_P, ctypes.c_int]),
+    "moe_prepack_weights": (ctypes.c_int, [_P] * 6),
+    "moe_copy_act": (ctypes.c_int, [_P] * 4),
     "moe_clear_device_error": (ctypes.c_int, [_P] * 3),
     "moe_check_device_error": (ctypes.c_int, [_P] * 3),
     "moe_status_str": (ctypes.c_char_p, [ctypes.c_int]),
@@ -212,6 +215,19 @@ def moe_copy_act_scales(plan, workspace, dst, stream=None):
            "moe_copy_act_scales")
 
 
+def moe_plan_set_weight_layout(plan, tiled):
+    _check(lib().moe_plan_set_weight_layout(plan, 1 if tiled else 0), "moe_plan_set_weight_layout")
+
+
+def moe_prepack_weights(plan, w1, w2, w1_tiled, w2_tiled, stream=None):
+    _check(lib().moe_prepack_weights(plan, *map(_ptr, (w1, w2, w1_tiled, w2_tiled)),
+                                     _stream(stream)), "moe_prepack_weights")
+
+
+def moe_copy_act(plan, workspace, dst, stream=None):
+    _check(lib().moe_copy_act(plan, _ptr(workspace), _ptr(dst), _stream(stream)), "moe_copy_act")
+
+
 def moe_clear_device_error(plan, workspace, stream=None):
     _check(lib().moe_clear_device_error(plan, _ptr(workspace), _stream(stream)),
            "moe_clear_device_error")
@@ -234,10 +250,12 @@ class MoELayer:
     """Convenience owner of a plan and its torch-allocated workspace."""
 
     def __init__(self, T, H, I, E, k, w_dtype="e4m3", act="swiglu", alpha=1.0, up_bias=0.0,
-                 limit=math.inf, device="cuda", debug=False):
+                 limit=math.inf, device="cuda", debug=False, tiled_weights=False):
         import torch
         self.T, self.H, self.I, self.E, self.k = T, H, I, E, k
         self.plan = moe_plan(T, H, I, E, k, w_dtype, act, alpha, up_bias, limit)
+        if tiled_weights:
+            moe_plan_set_weight_layout(self.plan, True)
         if debug:
             moe_plan_set_debug(self.plan, True)
         nbytes = moe_workspace_bytes(self.plan)
@@ -252,6 +270,13 @@ class MoELayer:
         moe_forward(self.plan, x, x_scales, topk_idx, topk_w, w1, w1_scales, w2, w2_scales, out,
                     self.workspace, stream)
         return out
+
+    def prepack(self, w1, w2):
+        """Tiled copies of row-major FP8 weights for a plan with tiled_weights."""
+        import torch
+        w1t, w2t = torch.empty_like(w1), torch.empty_like(w2)
+        moe_prepack_weights(self.plan, w1, w2, w1t, w2t)
+        return w1t, w2t
 
     def view(self):
         return moe_workspace_view(self.plan, self.workspace)

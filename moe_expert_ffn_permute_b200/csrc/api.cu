@@ -55,6 +55,21 @@ static bool aligned(const void* p, size_t a) {
 
 static moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+static moe_status check_ws(moe_plan_t plan, const void* workspace) {
+  if (plan == nullptr) return MOE_ERR_INVALID_ARG;
+  if (workspace == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256)) return MOE_ERR_ALIGNMENT;
+  return MOE_OK;
+}
+
+static moe_status check_weights(moe_plan_t plan, const void* w, const uint8_t* ws) {
+  if (w == nullptr || ws == nullptr) return MOE_ERR_INVALID_ARG;
+  const size_t wa = plan->w_dtype == MOE_W_E2M1_UE8M0_1x32 ? 32 : 16;
+  if (!aligned(w, wa)) return MOE_ERR_ALIGNMENT;
+  if (plan->w_dtype == MOE_W_E2M1_UE8M0_1x32 && !aligned(ws, 4)) return MOE_ERR_ALIGNMENT;
+  return MOE_OK;
+}
+
 extern "C" {
 
 moe_status moe_plan(int T, int H, int I, int E, int k, moe_dtypes dtypes, moe_act_params act,
@@ -88,6 +103,7 @@ moe_status moe_plan(int T, int H, int I, int E, int k, moe_dtypes dtypes, moe_ac
   p->w_dtype = dtypes.w_dtype;
   p->act = act;
   p->debug_act_f32 = 0;
+  p->w_tiled = 0;
   p->S = static_cast<long long>(T) * k;
   // Sum over experts of ceil(n_e / 128) <= floor((S + 127 E) / 128).
   p->rows_cap = ((p->S + 127ll * E) / kTileM) * kTileM;
@@ -102,6 +118,42 @@ void moe_plan_destroy(moe_plan_t plan) { delete plan; }
 
 size_t moe_workspace_bytes(moe_plan_t plan) { return plan ? plan->ws.total : 0; }
 
+moe_status moe_plan_set_weight_layout(moe_plan_t plan, int layout) {
+  if (plan == nullptr) return MOE_ERR_INVALID_ARG;
+  if (layout != MOE_WEIGHTS_ROW_MAJOR && layout != MOE_WEIGHTS_TILED) return MOE_ERR_INVALID_ARG;
+  if (layout == MOE_WEIGHTS_TILED && plan->w_dtype != MOE_W_E4M3_UE8M0_128x128)
+    return MOE_ERR_UNSUPPORTED;
+  plan->w_tiled = layout == MOE_WEIGHTS_TILED ? 1 : 0;
+  return MOE_OK;
+}
+
+moe_status moe_prepack_weights(moe_plan_t plan, const void* w1, const void* w2, void* w1_tiled,
+                               void* w2_tiled, moe_stream_t stream) {
+  if (plan == nullptr || w1 == nullptr || w2 == nullptr || w1_tiled == nullptr ||
+      w2_tiled == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (plan->w_dtype != MOE_W_E4M3_UE8M0_128x128) return MOE_ERR_UNSUPPORTED;
+  if (!aligned(w1, 16) || !aligned(w2, 16) || !aligned(w1_tiled, 16) || !aligned(w2_tiled, 16))
+    return MOE_ERR_ALIGNMENT;
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  const long long E = plan->E;
+  if (moe::launch_prepack(static_cast<const uint8_t*>(w1), E * 2 * plan->I, plan->H,
+                          static_cast<uint8_t*>(w1_tiled), st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return cuda_status(moe::launch_prepack(static_cast<const uint8_t*>(w2), E * plan->H, plan->I,
+                                         static_cast<uint8_t*>(w2_tiled), st));
+}
+
+moe_status moe_copy_act(moe_plan_t plan, const void* workspace, uint8_t* dst,
+                        moe_stream_t stream) {
+  moe_status s = check_ws(plan, workspace);
+  if (s != MOE_OK) return s;
+  if (dst == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned(dst, 16)) return MOE_ERR_ALIGNMENT;
+  return cuda_status(moe::launch_unpack_act(plan, static_cast<const uint8_t*>(workspace), dst,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_plan_set_debug(moe_plan_t plan, int capture_act_f32) {
   if (plan == nullptr) return MOE_ERR_INVALID_ARG;
   plan->debug_act_f32 = capture_act_f32 ? 1 : 0;
@@ -113,21 +165,6 @@ int moe_forward_launch_count(moe_plan_t plan) {
   if (plan == nullptr) return 0;
   // [route histogram,] route scan+scatter, gather, FC1+FC2 (one launch), combine
   return (plan->route_blocks > 1 ? 1 : 0) + 4;
-}
-
-static moe_status check_ws(moe_plan_t plan, const void* workspace) {
-  if (plan == nullptr) return MOE_ERR_INVALID_ARG;
-  if (workspace == nullptr) return MOE_ERR_INVALID_ARG;
-  if (!aligned(workspace, 256)) return MOE_ERR_ALIGNMENT;
-  return MOE_OK;
-}
-
-static moe_status check_weights(moe_plan_t plan, const void* w, const uint8_t* ws) {
-  if (w == nullptr || ws == nullptr) return MOE_ERR_INVALID_ARG;
-  const size_t wa = plan->w_dtype == MOE_W_E2M1_UE8M0_1x32 ? 32 : 16;
-  if (!aligned(w, wa)) return MOE_ERR_ALIGNMENT;
-  if (plan->w_dtype == MOE_W_E2M1_UE8M0_1x32 && !aligned(ws, 4)) return MOE_ERR_ALIGNMENT;
-  return MOE_OK;
 }
 
 moe_status moe_route(moe_plan_t plan, const int32_t* topk_idx, void* workspace,

@@ -45,7 +45,10 @@ namespace {
 constexpr int BM = 128, BN = 256, BK = 128, STAGES = 4, SCHED_DEPTH = 4;
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccCol = 0, kSfaCol = 256, kSfbCol = 264;
+// TMEM columns: accumulator 0-255; two sets of scale factors (A: 4 columns,
+// B: 8 columns), alternating per k-block so that loading the next k-block's
+// scales never waits for MMAs still reading the current ones.
+constexpr uint32_t kAccCol = 0, kSfaCol = 256, kSfbCol = 264, kSfSetStride = 16;
 constexpr int kEpiWarps = 8;
 constexpr int kSchedConsumers = 2 + kEpiWarps;   // producer, MMA, epilogue warps
 constexpr uint64_t kDepWaitLimitNs = 2000000000ull;
@@ -77,6 +80,9 @@ struct Phase {
   int b_rows_per_expert;     // 2I (FC1) or H (FC2)
   const uint8_t* sfa_chunks; // [m-tiles][k_blocks][512]
   const uint8_t* w_sf;       // weight scales
+  const uint8_t* a_tiles;    // A operand, pre-swizzled tiles [m-tiles][k_blocks][16 KB]
+  const uint8_t* w_tiles;    // weights as pre-swizzled tiles [E * n-blocks][k_blocks][16 KB],
+                             // or null: weights row-major, loaded by 2-D TMA
 };
 
 struct Params {
@@ -132,6 +138,28 @@ __device__ __forceinline__ bool get_task(Smem& sm, int& slot, uint32_t& phase, T
 
 // sigmoid(z) with the fast exponential and an approximate reciprocal (the
 // epilogue's transcendental pipe is shared by the E4M3 / bf16 conversions).
+// Single-thread variant of get_task for the MMA issuer, which runs its loop
+// on one lane only.
+__device__ __forceinline__ bool get_task_single(Smem& sm, int& slot, uint32_t& phase, Task& t,
+                                                uint32_t* err) {
+  if (!mbar_wait(&sm.sched_full[slot], phase, err, &sm.abort_flag)) return false;
+  const int4 v = sm.task[slot];
+  t.kind = v.x & 1;
+  t.reuse = (v.x >> 1) & 1;
+  t.e = v.x >> 2;
+  t.mt = v.y;
+  t.nt = v.z;
+  t.rows = v.w;
+  t.pos = sm.task_pos[slot];
+  fence_acq_rel_cta();
+  mbar_arrive(&sm.sched_empty[slot]);
+  if (++slot == SCHED_DEPTH) {
+    slot = 0;
+    phase ^= 1u;
+  }
+  return true;
+}
+
 __device__ __forceinline__ float sigmoidf_fast(float z) {
   return __fdividef(1.0f, 1.0f + __expf(-z));
 }
@@ -169,14 +197,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int q = 0; q < 4; ++q) mbar_init(&sm.pair[q], 2);
     sm.abort_flag = 0;
     fence_mbarrier_init();
-    if (p.phases & 1) {
-      tma_prefetch_desc(&tmap_a1);
-      tma_prefetch_desc(&tmap_b1);
-    }
-    if (p.phases & 2) {
-      tma_prefetch_desc(&tmap_a2);
-      tma_prefetch_desc(&tmap_b2);
-    }
+    if ((p.phases & 1) && p.ph[0].w_tiles == nullptr) tma_prefetch_desc(&tmap_b1);
+    if ((p.phases & 2) && p.ph[1].w_tiles == nullptr) tma_prefetch_desc(&tmap_b2);
   }
   if (warp == 1) {
     tmem_alloc(&sm.tmem_base, kTmemCols);
@@ -252,7 +274,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (t.e < 0) break;
       const Phase& ph = p.ph[t.kind];
       const uint64_t pol_b = t.reuse ? pol_b_reused : pol_b_once;
-      const CUtensorMap* ta = t.kind ? &tmap_a2 : &tmap_a1;
       const CUtensorMap* tb = t.kind ? &tmap_b2 : &tmap_b1;
       // Rows of B for this tile: two 128-row halves.
       int brow0, brow1;
@@ -302,8 +323,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (lane == 0) {
           mbar_arrive_expect_tx(&sm.full[stage], tx_bytes);
-          tma_load_2d(sm.a[stage], ta, kb * BK, t.mt * BM, &sm.full[stage], pol_a);
-          if (t.kind == 0) {
+          // Operand tiles are contiguous and pre-swizzled: one linear bulk copy
+          // each (row-major weights fall back to 2-D TMA tiles).
+          bulk_load_hint(sm.a[stage],
+                         ph.a_tiles + (static_cast<size_t>(t.mt) * ph.k_blocks + kb) * kTileBytes,
+                         kTileBytes, &sm.full[stage], pol_a);
+          if (ph.w_tiles != nullptr) {
+            bulk_load_hint(sm.b[stage],
+                           ph.w_tiles + (static_cast<size_t>(brow0 / 128) * ph.k_blocks + kb) *
+                                            kTileBytes,
+                           kTileBytes, &sm.full[stage], pol_b);
+            bulk_load_hint(sm.b[stage] + 128 * BK,
+                           ph.w_tiles + (static_cast<size_t>(brow1 / 128) * ph.k_blocks + kb) *
+                                            kTileBytes,
+                           kTileBytes, &sm.full[stage], pol_b);
+          } else if (t.kind == 0) {
             tma_load_2d(sm.b[stage], tb, kb * BK, brow0, &sm.full[stage], pol_b);
             tma_load_2d(sm.b[stage] + 128 * BK, tb, kb * BK, brow1, &sm.full[stage], pol_b);
           } else {
@@ -343,26 +377,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
-    int slot = 0, stage = 0;
-    uint32_t sphase = 0, phase = 0, acc_phase = 0;
-    Task t;
-    bool aborted = false;
-    while (!aborted && get_task(sm, slot, sphase, t, p.err)) {
-      if (t.e < 0) break;
-      if (!mbar_wait(&sm.tmem_empty, acc_phase ^ 1u, p.err, &sm.abort_flag)) break;
-      tc_fence_after();
-      const int k_blocks = p.ph[t.kind].k_blocks;
-      for (int kb = 0; kb < k_blocks; ++kb) {
-        if (!mbar_wait(&sm.full[stage], phase, p.err, &sm.abort_flag)) {
-          aborted = true;
-          break;
-        }
+    // One lane issues everything: a warp-wide wait + fence + __syncwarp per
+    // k-block leaves the tensor pipe idle between k-blocks.
+    if (lane == 0) {
+      int slot = 0, stage = 0;
+      uint32_t sphase = 0, phase = 0, acc_phase = 0, sfset = 0;
+      Task t;
+      bool aborted = false;
+      while (!aborted && get_task_single(sm, slot, sphase, t, p.err)) {
+        if (t.e < 0) break;
+        if (!mbar_wait(&sm.tmem_empty, acc_phase ^ 1u, p.err, &sm.abort_flag)) break;
         tc_fence_after();
-        if (lane == 0) {
-          fence_proxy_async_smem();
-          tmem_cp_32x128b_warpx4(tmem + kSfaCol, sf_desc(smem_u32(sm.sfa[stage])));
-          tmem_cp_32x128b_warpx4(tmem + kSfbCol, sf_desc(smem_u32(sm.sfb[stage])));
-          tmem_cp_32x128b_warpx4(tmem + kSfbCol + 4, sf_desc(smem_u32(sm.sfb[stage] + 512)));
+        const int k_blocks = p.ph[t.kind].k_blocks;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!mbar_wait(&sm.full[stage], phase, p.err, &sm.abort_flag)) {
+            aborted = true;
+            break;
+          }
+          // MXFP4 weight scales land by cp.async (generic proxy): order them
+          // before the tensor core's (async proxy) reads of shared memory.
+          if (kFp4) fence_proxy_async_smem();
+          const uint32_t sfa = tmem + kSfaCol + sfset * kSfSetStride;
+          const uint32_t sfb = tmem + kSfbCol + sfset * kSfSetStride;
+          tmem_cp_32x128b_warpx4(sfa, sf_desc(smem_u32(sm.sfa[stage])));
+          tmem_cp_32x128b_warpx4(sfb, sf_desc(smem_u32(sm.sfb[stage])));
+          tmem_cp_32x128b_warpx4(sfb + 4, sf_desc(smem_u32(sm.sfb[stage] + 512)));
           const uint32_t a_base = smem_u32(sm.a[stage]);
           const uint32_t b_base = smem_u32(sm.b[stage]);
 #pragma unroll
@@ -370,23 +409,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t idesc = mxf8f6f4_idesc(kFp4 ? 5u : 0u, BN, ks);
             mma_mxf8f6f4(tmem + kAccCol, umma_desc_sw128(a_base + ks * 32),
                          umma_desc_sw128(b_base + ks * 32), idesc,
-                         (tmem + kSfaCol) | (static_cast<uint32_t>(ks) << 30),
-                         (tmem + kSfbCol) | (static_cast<uint32_t>(ks) << 30),
-                         (kb > 0 || ks > 0) ? 1u : 0u);
+                         sfa | (static_cast<uint32_t>(ks) << 30),
+                         sfb | (static_cast<uint32_t>(ks) << 30), (kb > 0 || ks > 0) ? 1u : 0u);
           }
           tc_commit(&sm.empty[stage]);
+          sfset ^= 1u;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
-        __syncwarp();
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1u;
-        }
+        if (aborted) break;
+        tc_commit(&sm.tmem_full);
+        acc_phase ^= 1u;
       }
-      if (aborted) break;
-      if (lane == 0) tc_commit(&sm.tmem_full);
-      __syncwarp();
-      acc_phase ^= 1u;
     }
+    __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------- epilogue
     const int q = warp & 3;            // TMEM sub-partition (lanes 32q .. 32q+31)
@@ -440,7 +478,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n = ue8m0_exponent(amax);
         const float inv_scale = __uint_as_float(static_cast<uint32_t>(127 - n) << 23);
         const size_t prow = static_cast<size_t>(t.mt) * BM + row;
-        uint4* dst = reinterpret_cast<uint4*>(p.act + prow * p.I + t.nt * 128 + half * 64);
+        // The activation is stored as pre-swizzled 128 x 128 tiles (FC2's A).
+        uint8_t* tile = p.act + (static_cast<size_t>(t.mt) * (p.I / 128) + t.nt) * kTileBytes;
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           uint32_t w[4];
@@ -453,7 +492,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                            __uint_as_float(g[i0 + 3]) * inv_scale);
             w[j] = lo | (hi << 16);
           }
-          dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(tile + swz128(row, half * 4 + v)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
         }
         if (half == 0) {
           const uint32_t sbyte = static_cast<uint32_t>(n + 127) & 0xFFu;
@@ -576,22 +616,23 @@ cudaError_t launch_gemm(const moe_plan_s* pl, int phases, bool dynamic, const vo
   p.phases = phases;
   p.dynamic = dynamic ? 1 : 0;
   long long max_tiles = 0;
+  const bool tiled = pl->w_tiled != 0;
   if (phases & 1) {
     const int K = pl->H;
-    if (!make_map(&maps[0], ws + L.xg, K, pl->rows_cap, K, 128, false) ||
-        !make_map(&maps[1], w1, K, static_cast<uint64_t>(pl->E) * 2 * pl->I, kFp4 ? K / 2 : K,
-                  128, kFp4))
+    if (!tiled && !make_map(&maps[1], w1, K, static_cast<uint64_t>(pl->E) * 2 * pl->I,
+                            kFp4 ? K / 2 : K, 128, kFp4))
       return cudaErrorInvalidValue;
-    p.ph[0] = Phase{pl->I / 128, K / 128, 2 * pl->I, ws + L.xg_sf, w1s};
+    p.ph[0] = Phase{pl->I / 128, K / 128, 2 * pl->I, ws + L.xg_sf, w1s, ws + L.xg,
+                    tiled ? static_cast<const uint8_t*>(w1) : nullptr};
     max_tiles += (pl->rows_cap / BM) * p.ph[0].n_tiles;
   }
   if (phases & 2) {
     const int K = pl->I;
-    if (!make_map(&maps[2], ws + L.act, K, pl->rows_cap, K, 128, false) ||
-        !make_map(&maps[3], w2, K, static_cast<uint64_t>(pl->E) * pl->H, kFp4 ? K / 2 : K, 256,
-                  kFp4))
+    if (!tiled && !make_map(&maps[3], w2, K, static_cast<uint64_t>(pl->E) * pl->H,
+                            kFp4 ? K / 2 : K, 256, kFp4))
       return cudaErrorInvalidValue;
-    p.ph[1] = Phase{pl->H / 256, K / 128, pl->H, ws + L.act_sf, w2s};
+    p.ph[1] = Phase{pl->H / 256, K / 128, pl->H, ws + L.act_sf, w2s, ws + L.act,
+                    tiled ? static_cast<const uint8_t*>(w2) : nullptr};
     max_tiles += (pl->rows_cap / BM) * p.ph[1].n_tiles;
   }
   p.tile_off = reinterpret_cast<const int32_t*>(ws + L.tile_off);

@@ -38,6 +38,7 @@ struct moe_plan_s {
   int w_dtype;
   moe_act_params act;
   int debug_act_f32;
+  int w_tiled;           // weights given as pre-swizzled tiles (moe_prepack_weights)
   long long S;           // T*k
   long long rows_cap;    // padded row capacity (multiple of 128)
   int route_blocks;
@@ -80,6 +81,10 @@ cudaError_t launch_fc2(const moe_plan_s* p, const void* w2, const uint8_t* w2s, 
 cudaError_t launch_fc12(const moe_plan_s* p, const void* w1, const uint8_t* w1s, const void* w2,
                         const uint8_t* w2s, uint8_t* ws, cudaStream_t st);
 cudaError_t launch_combine(const moe_plan_s* p, const float* topk_w, void* out, uint8_t* ws,
+                           cudaStream_t st);
+cudaError_t launch_unpack_act(const moe_plan_s* p, const uint8_t* ws, uint8_t* dst,
+                              cudaStream_t st);
+cudaError_t launch_prepack(const uint8_t* src, long long rows, int K, uint8_t* dst,
                            cudaStream_t st);
 cudaError_t launch_unpack_act_scales(const moe_plan_s* p, const uint8_t* ws, uint8_t* dst,
                                      cudaStream_t st);

@@ -184,7 +184,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
 }
 
 // Gather: padded row P (m-tile P / 128, row r = P % 128) of expert e receives
-// x[perm[offsets[e] + local + r] / k]; one warp per row, 16-byte accesses.
+// x[perm[offsets[e] + local + r] / k]; one warp per row, 16-byte accesses,
+// written in the pre-swizzled tile layout the FC1 producer bulk-copies.
 // Its scale bytes go to the tensor-core scale-chunk layout: for k-block kb the
 // 512-byte chunk of the tile holds, at byte (r % 32) * 16 + (r / 32) * 4 + j
 // (j = 0..3), the row's UE8M0 byte, replicated over the four 32-wide K
@@ -206,10 +207,13 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(
   const int tile = static_cast<int>(P / kTileM);
   const int r = static_cast<int>(P % kTileM);
   const int vec = H / 16;
-  const uint4* __restrict__ src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
-  uint4* __restrict__ dst = reinterpret_cast<uint4*>(xg + static_cast<size_t>(P) * H);
-  for (int c = lane; c < vec; c += 32) dst[c] = __ldg(&src[c]);
   const int kb_n = H / 128;
+  const uint4* __restrict__ src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
+  // Destination: pre-swizzled 128 x 128-byte tiles [tile][k-block][16 KB].
+  uint8_t* __restrict__ dst = xg + static_cast<size_t>(tile) * kb_n * kTileBytes;
+  for (int c = lane; c < vec; c += 32)
+    *reinterpret_cast<uint4*>(dst + static_cast<size_t>(c >> 3) * kTileBytes + swz128(r, c & 7)) =
+        __ldg(&src[c]);
   uint8_t* chunk = xg_sf + static_cast<size_t>(tile) * kb_n * 512 + (r & 31) * 16 + (r >> 5) * 4;
   for (int kb = lane; kb < kb_n; kb += 32) {
     const uint32_t b = __ldg(&xs[static_cast<size_t>(t) * kb_n + kb]);

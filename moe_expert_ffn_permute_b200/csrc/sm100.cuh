@@ -142,6 +142,24 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, 
       : "memory");
 }
 
+__device__ __forceinline__ void bulk_load_hint(void* smem_dst, const void* gmem_src,
+                                               uint32_t bytes, uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(smem_dst)),
+      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// Operand tiles stored "pre-swizzled": a 128 x 128-byte tile is 16 KB,
+// contiguous, with byte c of row r at r * 128 + (((c / 16) ^ (r % 8)) * 16) +
+// c % 16 -- exactly the 128-byte-swizzled layout the tensor core reads, so one
+// linear bulk copy fills a shared-memory stage.
+constexpr uint32_t kTileBytes = 16384;
+__host__ __device__ __forceinline__ uint32_t swz128(uint32_t r, uint32_t c16) {
+  return r * 128u + (((c16 ^ (r & 7u)) & 7u) << 4);
+}
+
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));

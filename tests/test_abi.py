@@ -101,3 +101,14 @@ def test_fp4_weights_need_32_byte_alignment():
 def test_status_strings():
     assert moe.moe_status_str(0) == "MOE_OK"
     assert moe.moe_status_str(5) == "MOE_ERR_DEVICE_TIMEOUT"
+
+
+def test_tiled_weights_only_for_fp8():
+    p = moe.moe_plan(8, 512, 256, 8, 2, w_dtype="e2m1")
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_plan_set_weight_layout(p, True)
+    assert ei.value.status == 2
+    moe.moe_plan_destroy(p)
+    q = moe.moe_plan(8, 512, 256, 8, 2)
+    moe.moe_plan_set_weight_layout(q, True)
+    moe.moe_plan_destroy(q)

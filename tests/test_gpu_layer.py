@@ -51,7 +51,9 @@ def test_fc1_requant_bytes_exact_and_activation_close(wl):
     out, lay = run_gpu(wl, d, debug=True)
     v = lay.view()
     rows = v.rows
-    act = _ws_bytes(lay, v.act, rows * wl.I).view(rows, wl.I).cpu().numpy()
+    act_t = torch.empty(rows, wl.I, dtype=torch.uint8, device="cuda")
+    moe.moe_copy_act(lay.plan, lay.workspace, act_t)
+    act = act_t.cpu().numpy()
     a32 = _ws_bytes(lay, v.act_f32, rows * wl.I * 4).view(torch.float32).view(rows, wl.I)
     a32 = a32.cpu().numpy()
     sf = torch.empty(rows, wl.I // 128, dtype=torch.uint8, device="cuda")
@@ -197,3 +199,59 @@ def test_cuda_graph_replay_is_bitwise_identical():
     torch.cuda.synchronize()
     ref2, _ = run_gpu(wl, d)
     assert torch.equal(out, ref2)
+
+
+def _run_tiled(wl, d):
+    lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype=wl.w_dtype, act=wl.act,
+                       alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit, tiled_weights=True)
+    w1t, w2t = lay.prepack(d["w1"], d["w2"])
+    out = lay.forward(d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], w1t, d["w1_scales"],
+                      w2t, d["w2_scales"])
+    torch.cuda.synchronize()
+    return out, lay
+
+
+def _tiles_reference(w, K):
+    """Tiled layout written out from its definition (torch indexing)."""
+    rows = w.numel() // K
+    m = w.reshape(rows, K).view(rows // 128, 128, K // 128, 8, 16)   # [rb, r, kb, c16, byte]
+    r = torch.arange(128, device=w.device).view(128, 1)
+    c16 = torch.arange(8, device=w.device).view(1, 8)
+    dest_c16 = (c16 ^ (r % 8))                                        # [r, c16]
+    out = torch.empty(rows // 128, K // 128, 128, 8, 16, dtype=torch.uint8, device=w.device)
+    src = m.permute(0, 2, 1, 3, 4)                                    # [rb, kb, r, c16, byte]
+    idx = dest_c16.view(1, 1, 128, 8, 1).expand_as(src)
+    out.scatter_(3, idx, src)
+    return out.reshape(-1)
+
+
+def test_prepack_matches_layout_definition():
+    wl = RAGGED
+    d = inputs(wl)
+    lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, tiled_weights=True)
+    w1t, w2t = lay.prepack(d["w1"], d["w2"])
+    torch.cuda.synchronize()
+    assert torch.equal(w1t.reshape(-1), _tiles_reference(d["w1"], wl.H))
+    assert torch.equal(w2t.reshape(-1), _tiles_reference(d["w2"], wl.I))
+
+
+@pytest.mark.parametrize("wl", [WORKLOADS["tiny"], RAGGED, RAGGED_OAI], ids=lambda w: w.name)
+def test_tiled_weights_bitwise_equal_row_major(wl):
+    d = inputs(wl)
+    ref, _ = run_gpu(wl, d)
+    out, lay = _run_tiled(wl, d)
+    assert lay.check() == 0
+    assert torch.equal(out, ref)
+
+
+@pytest.mark.parametrize("name,ntok", [("decode", 32), ("prefill", 8)])
+def test_tiled_weights_full_size_parity(name, ntok):
+    wl = WORKLOADS[name]
+    d = inputs(wl)
+    out, lay = _run_tiled(wl, d)
+    assert lay.check() == 0
+    rng = np.random.default_rng(wl.T + 1)
+    tokens = np.sort(rng.choice(wl.T, size=ntok, replace=False))
+    dn = {k: v.cpu().numpy() for k, v in d.items()}
+    ref = oracle_tokens(wl, dn, tokens)
+    assert_parity(out.float().cpu().numpy()[tokens], ref, wl.name + "-tiled")
