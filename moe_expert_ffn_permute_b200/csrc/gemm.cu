@@ -12,10 +12,11 @@
 // scale per 32-wide K sub-block; the coarser blocks are replicated).
 //
 // Warp roles (12 warps):
-//   warp 0   producer: TMA loads of A/B tiles, scale chunks (bulk copy / cp.async)
+//   warp 0   operand producer: bulk copies of the A/B tiles
 //   warp 1   MMA issuer; owns the tensor-memory allocation
 //   warp 2   tile scheduler: writes task infos into a ring of shared-memory slots
-//   warp 3   idle
+//   warp 3   scale-factor producer: A scale chunks (bulk copy), B scales
+//            (shared-memory stores or cp.async)
 //   warps 4-11 epilogue: two warps per 32-lane TMEM sub-partition
 //
 // Scheduler slot release (fw-ai/DeepGEMM PR #16 "Sync upstream through PR #441:
@@ -50,7 +51,7 @@ constexpr uint32_t kTmemCols = 512;
 // scales never waits for MMAs still reading the current ones.
 constexpr uint32_t kAccCol = 0, kSfaCol = 256, kSfbCol = 264, kSfSetStride = 16;
 constexpr int kEpiWarps = 8;
-constexpr int kSchedConsumers = 2 + kEpiWarps;   // producer, MMA, epilogue warps
+constexpr int kSchedConsumers = 3 + kEpiWarps;   // 2 producers, MMA, epilogue warps
 constexpr uint64_t kDepWaitLimitNs = 2000000000ull;
 
 struct __align__(1024) Smem {
@@ -185,6 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
+      // operand producer's expect-tx arrive + one arrive per scale-factor lane
       mbar_init(&sm.full[s], 33);
       mbar_init(&sm.empty[s], 1);
     }
@@ -256,8 +258,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (t.e < 0) break;
       }
     }
-  } else if (warp == 0) {
-    // ------------------------------------------------------------- producer
+  } else if (warp == 0 || warp == 3) {
+    // ------------------------------------------------------------ producers
+    // Warp 0 streams the operand tiles (its bulk copies wait on the copy
+    // engine); warp 3 provides the stage's scale factors in parallel.
+    const bool operands = warp == 0;
     int slot = 0, stage = 0;
     uint32_t sphase = 0, phase = 0;
     // A tiles are re-read by every n-tile of their m-tile: keep them in L2.
@@ -266,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t pol_a = l2_policy_evict_last();
     const uint64_t pol_b_once = l2_policy_evict_first();
     const uint64_t pol_b_reused = l2_policy_evict_normal();
-    const uint32_t tx_bytes = BM * BK + (kFp4 ? BN * BK / 2 : BN * BK) + 512;
+    const uint32_t ab_bytes = BM * BK + (kFp4 ? BN * BK / 2 : BN * BK);
     const uint32_t fc1_target = static_cast<uint32_t>(kEpiWarps * p.ph[0].n_tiles);
     Task t;
     bool aborted = false;
@@ -286,8 +291,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (t.kind == 1 && (p.phases & 1)) {
         // FC2 after FC1 in the same launch: wait until every FC1 epilogue warp
-        // of this m-tile has published its rows, then order those generic-proxy
-        // writes before this thread's async-proxy (TMA) reads.
+        // of this m-tile has published its rows (activation tiles and their
+        // scale chunks), then order those generic-proxy writes before this
+        // thread's async-proxy (bulk copy) reads.
         if (lane == 0) {
           const uint32_t* flag = p.fc1_done + t.mt;
           if (ld_acquire_gpu(flag) < fc1_target) {
@@ -309,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       uint32_t sf0 = 0, sf1 = 0;   // FP8 weight scales for k-blocks kb = 32*c + lane
       for (int kb = 0; kb < ph.k_blocks; ++kb) {
-        if (!kFp4 && (kb & 31) == 0) {
+        if (!operands && !kFp4 && (kb & 31) == 0) {
           const int kq = kb + lane;
           const int kbs = ph.k_blocks;
           if (kq < kbs) {
@@ -321,53 +327,61 @@ __global__ void __launch_bounds__(kThreads, 1)
           aborted = true;
           break;
         }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&sm.full[stage], tx_bytes);
-          // Operand tiles are contiguous and pre-swizzled: one linear bulk copy
-          // each (row-major weights fall back to 2-D TMA tiles).
-          bulk_load_hint(sm.a[stage],
-                         ph.a_tiles + (static_cast<size_t>(t.mt) * ph.k_blocks + kb) * kTileBytes,
-                         kTileBytes, &sm.full[stage], pol_a);
-          if (ph.w_tiles != nullptr) {
-            bulk_load_hint(sm.b[stage],
-                           ph.w_tiles + (static_cast<size_t>(brow0 / 128) * ph.k_blocks + kb) *
-                                            kTileBytes,
-                           kTileBytes, &sm.full[stage], pol_b);
-            bulk_load_hint(sm.b[stage] + 128 * BK,
-                           ph.w_tiles + (static_cast<size_t>(brow1 / 128) * ph.k_blocks + kb) *
-                                            kTileBytes,
-                           kTileBytes, &sm.full[stage], pol_b);
-          } else if (t.kind == 0) {
-            tma_load_2d(sm.b[stage], tb, kb * BK, brow0, &sm.full[stage], pol_b);
-            tma_load_2d(sm.b[stage] + 128 * BK, tb, kb * BK, brow1, &sm.full[stage], pol_b);
-          } else {
-            tma_load_2d(sm.b[stage], tb, kb * BK, brow0, &sm.full[stage], pol_b);
-          }
-          bulk_load(sm.sfa[stage],
-                    ph.sfa_chunks + (static_cast<size_t>(t.mt) * ph.k_blocks + kb) * 512, 512,
-                    &sm.full[stage]);
-        }
-        if (kFp4) {
-          // One 32-bit word = the four 1x32 scales of this 128-wide k-block.
-          const int kw = ph.k_blocks * 4;   // scale bytes per weight row
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const int rb = c ? brow1 : brow0;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int r = lane + 32 * q;
-              cp_async_4(sm.sfb[stage] + c * 512 + lane * 16 + q * 4,
-                         ph.w_sf + static_cast<size_t>(rb + r) * kw + kb * 4);
+        if (operands) {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&sm.full[stage], ab_bytes);
+            // Operand tiles are contiguous and pre-swizzled: one linear bulk
+            // copy each (row-major weights fall back to 2-D TMA tiles).
+            bulk_load_hint(
+                sm.a[stage],
+                ph.a_tiles + (static_cast<size_t>(t.mt) * ph.k_blocks + kb) * kTileBytes,
+                kTileBytes, &sm.full[stage], pol_a);
+            if (ph.w_tiles != nullptr) {
+              bulk_load_hint(
+                  sm.b[stage],
+                  ph.w_tiles + (static_cast<size_t>(brow0 / 128) * ph.k_blocks + kb) * kTileBytes,
+                  kTileBytes, &sm.full[stage], pol_b);
+              bulk_load_hint(
+                  sm.b[stage] + 128 * BK,
+                  ph.w_tiles + (static_cast<size_t>(brow1 / 128) * ph.k_blocks + kb) * kTileBytes,
+                  kTileBytes, &sm.full[stage], pol_b);
+            } else if (t.kind == 0) {
+              tma_load_2d(sm.b[stage], tb, kb * BK, brow0, &sm.full[stage], pol_b);
+              tma_load_2d(sm.b[stage] + 128 * BK, tb, kb * BK, brow1, &sm.full[stage], pol_b);
+            } else {
+              tma_load_2d(sm.b[stage], tb, kb * BK, brow0, &sm.full[stage], pol_b);
             }
           }
-          cp_async_mbar_arrive_noinc(&sm.full[stage]);
+          __syncwarp();
         } else {
-          const uint32_t g = __shfl_sync(0xffffffffu, sf0, kb & 31) * 0x01010101u;
-          const uint32_t u = __shfl_sync(0xffffffffu, sf1, kb & 31) * 0x01010101u;
-          reinterpret_cast<uint4*>(sm.sfb[stage])[lane] = make_uint4(g, g, g, g);
-          reinterpret_cast<uint4*>(sm.sfb[stage] + 512)[lane] = make_uint4(u, u, u, u);
-          fence_proxy_async_smem();
-          mbar_arrive(&sm.full[stage]);
+          if (lane == 0) {
+            mbar_expect_tx(&sm.full[stage], 512);
+            bulk_load(sm.sfa[stage],
+                      ph.sfa_chunks + (static_cast<size_t>(t.mt) * ph.k_blocks + kb) * 512, 512,
+                      &sm.full[stage]);
+          }
+          if (kFp4) {
+            // One 32-bit word = the four 1x32 scales of this 128-wide k-block.
+            const int kw = ph.k_blocks * 4;   // scale bytes per weight row
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const int rb = c ? brow1 : brow0;
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int r = lane + 32 * q;
+                cp_async_4(sm.sfb[stage] + c * 512 + lane * 16 + q * 4,
+                           ph.w_sf + static_cast<size_t>(rb + r) * kw + kb * 4);
+              }
+            }
+            cp_async_mbar_arrive_noinc(&sm.full[stage]);
+          } else {
+            const uint32_t g = __shfl_sync(0xffffffffu, sf0, kb & 31) * 0x01010101u;
+            const uint32_t u = __shfl_sync(0xffffffffu, sf1, kb & 31) * 0x01010101u;
+            reinterpret_cast<uint4*>(sm.sfb[stage])[lane] = make_uint4(g, g, g, g);
+            reinterpret_cast<uint4*>(sm.sfb[stage] + 512)[lane] = make_uint4(u, u, u, u);
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.full[stage]);
+          }
         }
         if (++stage == STAGES) {
           stage = 0;
