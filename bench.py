@@ -105,7 +105,9 @@ class Clocks:
 
 
 KERNEL_SOURCES = ("moe_expert_ffn_permute_b200/csrc/gemm.cu",
+                  "moe_expert_ffn_permute_b200/csrc/gemm2.cu",
                   "moe_expert_ffn_permute_b200/csrc/sm100.cuh",
+                  "moe_expert_ffn_permute_b200/csrc/sm100_pair.cuh",
                   "moe_expert_ffn_permute_b200/csrc/internal.h")
 
 
@@ -169,7 +171,8 @@ def run_b200(args, wl):
     tiled = wl.w_dtype == "e4m3" and not args.row_major_weights
     lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype=wl.w_dtype, act=wl.act,
                        alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit, device=dev,
-                       tiled_weights=tiled)
+                       tiled_weights=tiled, cta_pairs=args.cta_pairs if tiled else None)
+    pairs = moe.moe_plan_cta_pairs_active(lay.plan)
     d_row_major = dict(d)          # the oracle reads the original layout
     if tiled:
         d["w1"], d["w2"] = lay.prepack(d["w1"], d["w2"])
@@ -307,8 +310,9 @@ def run_b200(args, wl):
                 "peak": round(2 * bf16, 1), "unit": "TFLOP/s"}
     roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
     roof["traffic"] = measured_traffic(wl.name)
-    roof["kernel"] = ("moe_gemm_kernel: FC1 + SwiGLU + FP8 requant and FC2 in one persistent "
-                      "launch")
+    roof["kernel"] = (("moe_gemm_pair_kernel (CTA pairs, 2-SM MMA; with its weight-scale "
+                       "expansion launch)" if pairs else "moe_gemm_kernel") +
+                      ": FC1 + SwiGLU + FP8 requant and FC2 in one persistent launch")
     roof["per_launch"] = (f"{w_bytes} B of expert weights+scales ({active} active experts)"
                           if hbm_bound else f"{flops:.4g} FLOP (6*S*H*I)")
     roof["peak_source"] = f"{peak_src}" + ("" if roof["unit"] == "GB/s" else
@@ -426,6 +430,8 @@ def main():
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--cpu-tokens", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cta-pairs", type=int, default=0, choices=[0, 1, 2],
+                    help="GEMM on CTA pairs: 0 automatic, 1 never, 2 always (tiled FP8 only)")
     ap.add_argument("--row-major-weights", action="store_true",
                     help="read FP8 weights row-major via 2-D TMA instead of prepacked tiles")
     args = ap.parse_args()

@@ -254,6 +254,21 @@ moe_status moe_copy_act_scales(moe_plan_t plan, const void *workspace,
 typedef enum { MOE_WEIGHTS_ROW_MAJOR = 0, MOE_WEIGHTS_TILED = 1 } moe_weight_layout;
 moe_status moe_plan_set_weight_layout(moe_plan_t plan, int layout);
 
+/* GEMM variant for moe_fc1_fc2 / moe_forward.  With tiled FP8 weights the two
+ * GEMMs can run on CTA pairs with the 2-SM tensor-core MMA (each pair computes
+ * 256 x 256 tiles; each SM loads half of the weight tile).  mode 0: automatic
+ * (currently the single-CTA kernel, which measured as fast at every size
+ * tried), 1: never, 2: always (MOE_ERR_UNSUPPORTED without tiled FP8
+ * weights; set the weight layout first).  Results are the same bytes either
+ * way.  On pairs,
+ * moe_fc1_fc2 enqueues two kernels: the weight scales (w1_scales, w2_scales)
+ * are first expanded into a workspace region, then the GEMMs run.          */
+moe_status moe_plan_set_cta_pairs(moe_plan_t plan, int mode);
+
+/* 1 if moe_fc1_fc2 / moe_forward run the GEMMs on CTA pairs with the plan's
+ * current settings, 0 if not (or plan is NULL).                             */
+int moe_plan_cta_pairs_active(moe_plan_t plan);
+
 /* Rearrange row-major FP8 weights w1 [E,2I,H] and w2 [E,H,I] (device) into
  * the tiled layout (w1_tiled, w2_tiled: device buffers of the same sizes,
  * 16-byte aligned; must not overlap the inputs).  Tile (b, kb) -- rows

@@ -10,8 +10,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libmoe_b200.so")
-SOURCES = ["api.cu", "route.cu", "gemm.cu", "combine.cu", "quant.cu", "layout.cu"]
-HEADERS = ["internal.h", "sm100.cuh"]
+SOURCES = ["api.cu", "route.cu", "gemm.cu", "combine.cu", "quant.cu", "layout.cu", "gemm2.cu"]
+HEADERS = ["internal.h", "sm100.cuh", "sm100_pair.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC", "-shared", "-cudart", "static", "--expt-relaxed-constexpr"]

@@ -26,6 +26,7 @@ void compute_layout(moe_plan_s* p) {
   L.offsets = take((E + 1) * 4);
   L.pad_off = take((E + 1) * 4);
   L.tile_off = take((E + 1) * 4);
+  L.pair_off = take((E + 1) * 4);
   L.block_hist = take(static_cast<size_t>(p->route_blocks) * E * 4);
   L.sched = take(256 + rows / kTileM * 4);
   L.perm = take(S * 4);
@@ -37,6 +38,11 @@ void compute_layout(moe_plan_s* p) {
   L.act_sf = take(rows / kTileM * (p->I / 128) * 512);
   L.act_f32 = take(p->debug_act_f32 ? rows * p->I * 4 : 0);
   L.y = take(S * p->H * 2);
+  // One 1 KB record per (expert, n-tile, k-block) of each GEMM: the two 128-row
+  // weight blocks of a 256-wide tile, each block's scale byte repeated 512 times.
+  const bool fp8 = p->w_dtype == MOE_W_E4M3_UE8M0_128x128;
+  L.pair_sf1 = take(fp8 ? E * (p->I / 128) * (p->H / 128) * 1024 : 0);
+  L.pair_sf2 = take(fp8 ? E * (p->H / 256) * (p->I / 128) * 1024 : 0);
   L.in_x = take(static_cast<size_t>(p->T) * p->H);
   L.in_xs = take(static_cast<size_t>(p->T) * (p->H / 128));
   L.in_idx = take(S * 4);
@@ -54,6 +60,15 @@ static bool aligned(const void* p, size_t a) {
 }
 
 static moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// 2-SM GEMM: needs tiled FP8 weights and is used only when asked for (mode
+// 2).  Automatic mode keeps the single-CTA kernel: at 8192 tokens of the
+// 7168 x 2048 x 32-expert layer both run power-capped and the pair kernel
+// measured no faster.
+static bool use_pairs(const moe_plan_s* p) {
+  if (!p->w_tiled || p->w_dtype != MOE_W_E4M3_UE8M0_128x128) return false;
+  return p->pair_mode == 2;
+}
 
 static moe_status check_ws(moe_plan_t plan, const void* workspace) {
   if (plan == nullptr) return MOE_ERR_INVALID_ARG;
@@ -104,6 +119,7 @@ moe_status moe_plan(int T, int H, int I, int E, int k, moe_dtypes dtypes, moe_ac
   p->act = act;
   p->debug_act_f32 = 0;
   p->w_tiled = 0;
+  p->pair_mode = 0;
   p->S = static_cast<long long>(T) * k;
   // Sum over experts of ceil(n_e / 128) <= floor((S + 127 E) / 128).
   p->rows_cap = ((p->S + 127ll * E) / kTileM) * kTileM;
@@ -124,6 +140,14 @@ moe_status moe_plan_set_weight_layout(moe_plan_t plan, int layout) {
   if (layout == MOE_WEIGHTS_TILED && plan->w_dtype != MOE_W_E4M3_UE8M0_128x128)
     return MOE_ERR_UNSUPPORTED;
   plan->w_tiled = layout == MOE_WEIGHTS_TILED ? 1 : 0;
+  return MOE_OK;
+}
+
+moe_status moe_plan_set_cta_pairs(moe_plan_t plan, int mode) {
+  if (plan == nullptr || mode < 0 || mode > 2) return MOE_ERR_INVALID_ARG;
+  if (mode == 2 && (!plan->w_tiled || plan->w_dtype != MOE_W_E4M3_UE8M0_128x128))
+    return MOE_ERR_UNSUPPORTED;
+  plan->pair_mode = mode;
   return MOE_OK;
 }
 
@@ -161,10 +185,15 @@ moe_status moe_plan_set_debug(moe_plan_t plan, int capture_act_f32) {
   return MOE_OK;
 }
 
+int moe_plan_cta_pairs_active(moe_plan_t plan) {
+  return plan != nullptr && use_pairs(plan) ? 1 : 0;
+}
+
 int moe_forward_launch_count(moe_plan_t plan) {
   if (plan == nullptr) return 0;
-  // [route histogram,] route scan+scatter, gather, FC1+FC2 (one launch), combine
-  return (plan->route_blocks > 1 ? 1 : 0) + 4;
+  // [route histogram,] route scan+scatter, gather, [pair scale expansion,]
+  // FC1+FC2 (one launch), combine
+  return (plan->route_blocks > 1 ? 1 : 0) + (use_pairs(plan) ? 1 : 0) + 4;
 }
 
 moe_status moe_route(moe_plan_t plan, const int32_t* topk_idx, void* workspace,
@@ -212,9 +241,11 @@ moe_status moe_fc1_fc2(moe_plan_t plan, const void* w1, const uint8_t* w1_scales
   if (s != MOE_OK) return s;
   if ((s = check_weights(plan, w1, w1_scales)) != MOE_OK) return s;
   if ((s = check_weights(plan, w2, w2_scales)) != MOE_OK) return s;
-  return cuda_status(moe::launch_fc12(plan, w1, w1_scales, w2, w2_scales,
-                                      static_cast<uint8_t*>(workspace),
-                                      reinterpret_cast<cudaStream_t>(stream)));
+  auto ws = static_cast<uint8_t*>(workspace);
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  if (use_pairs(plan))
+    return cuda_status(moe::launch_fc12_pairs(plan, w1, w1_scales, w2, w2_scales, ws, st));
+  return cuda_status(moe::launch_fc12(plan, w1, w1_scales, w2, w2_scales, ws, st));
 }
 
 moe_status moe_combine(moe_plan_t plan, const float* topk_w, void* out, void* workspace,

@@ -63,6 +63,7 @@ struct __align__(1024) Smem {
   uint64_t empty[STAGES];
   uint64_t tmem_full;
   uint64_t tmem_empty;
+  uint64_t drain;   // tensor-core completion before TMEM is freed
   uint64_t sched_full[SCHED_DEPTH];
   uint64_t sched_empty[SCHED_DEPTH];
   uint64_t pair[4];
@@ -191,6 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.empty[s], 1);
     }
     mbar_init(&sm.tmem_full, 1);
+    mbar_init(&sm.drain, 1);
     mbar_init(&sm.tmem_empty, kEpiWarps);
     for (int r = 0; r < SCHED_DEPTH; ++r) {
       mbar_init(&sm.sched_full[r], 1);
@@ -437,6 +439,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit(&sm.tmem_full);
         acc_phase ^= 1u;
       }
+      // Every MMA and TMEM copy issued above completes before the TMEM is
+      // freed, on the abort path too.
+      tc_commit(&sm.drain);
+      if (!mbar_wait_limited(&sm.drain, 0, kWaitLimitNs)) atomicOr(p.err, kErrTimeoutBit);
     }
     __syncwarp();
   } else if (warp >= 4) {

@@ -17,7 +17,7 @@ constexpr int kTileM = 128;          // rows per m-tile (expert blocks are padde
 
 // Byte offsets of every buffer inside the caller's workspace (256-B aligned).
 struct WorkspaceLayout {
-  size_t err, counts, offsets, pad_off, tile_off;
+  size_t err, counts, offsets, pad_off, tile_off, pair_off;
   size_t block_hist;
   size_t sched;             // fused-GEMM tile counter + per-m-tile FC1 completion counts
   size_t perm, inv;
@@ -26,6 +26,7 @@ struct WorkspaceLayout {
   size_t act, act_sf;       // FC1 output: FP8 activation + scale chunks
   size_t act_f32;           // debug capture (0 bytes when off)
   size_t y;                 // FC2 output, bf16, slot order
+  size_t pair_sf1, pair_sf2;   // weight scales expanded for the CTA-pair GEMM (FP8 plans)
   size_t in_x, in_xs, in_idx, in_w;   // staging for moe_forward_hostio inputs
   size_t out_stage;                   // and its bf16 output
   size_t total;
@@ -39,6 +40,7 @@ struct moe_plan_s {
   moe_act_params act;
   int debug_act_f32;
   int w_tiled;           // weights given as pre-swizzled tiles (moe_prepack_weights)
+  int pair_mode;         // 2-SM GEMM: 0 automatic, 1 never, 2 always
   long long S;           // T*k
   long long rows_cap;    // padded row capacity (multiple of 128)
   int route_blocks;
@@ -80,6 +82,9 @@ cudaError_t launch_fc2(const moe_plan_s* p, const void* w2, const uint8_t* w2s, 
 // FC1 and FC2 in one persistent launch (dynamic tile scheduler).
 cudaError_t launch_fc12(const moe_plan_s* p, const void* w1, const uint8_t* w1s, const void* w2,
                         const uint8_t* w2s, uint8_t* ws, cudaStream_t st);
+// The same on CTA pairs with the 2-SM MMA (FP8, tiled weights only).
+cudaError_t launch_fc12_pairs(const moe_plan_s* p, const void* w1, const uint8_t* w1s,
+                              const void* w2, const uint8_t* w2s, uint8_t* ws, cudaStream_t st);
 cudaError_t launch_combine(const moe_plan_s* p, const float* topk_w, void* out, uint8_t* ws,
                            cudaStream_t st);
 cudaError_t launch_unpack_act(const moe_plan_s* p, const uint8_t* ws, uint8_t* dst,

@@ -66,6 +66,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
     const int32_t* __restrict__ idx, int S, int E, int nblk,
     const int32_t* __restrict__ block_hist, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ tile_off, int32_t* __restrict__ pad_off,
+    int32_t* __restrict__ pair_off,
     int32_t* __restrict__ perm, int32_t* __restrict__ inv, uint32_t* err,
     uint32_t* __restrict__ sched, int sched_words, int32_t* __restrict__ row_token, int k) {
   constexpr int kWarps = kRouteThreads / 32;
@@ -108,18 +109,21 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
   }
   __syncthreads();
   if (tid == 0) {
-    int acc = 0, tacc = 0;
+    int acc = 0, tacc = 0, pacc = 0;
     for (int e = 0; e < E; ++e) {
       scan[e] = acc;
       tscan[e] = tacc;
+      const int tiles = (total[e] + kTileM - 1) / kTileM;
       if (blockIdx.x == 0) {
         offsets[e] = acc;
         counts[e] = total[e];
         tile_off[e] = tacc;
         pad_off[e] = tacc * kTileM;
+        if (pair_off != nullptr) pair_off[e] = pacc;   // pairs of m-tiles of one expert
       }
       acc += total[e];
-      tacc += (total[e] + kTileM - 1) / kTileM;
+      tacc += tiles;
+      pacc += (tiles + 1) / 2;
     }
     scan[E] = acc;
     tscan[E] = tacc;
@@ -127,6 +131,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
       offsets[E] = acc;
       tile_off[E] = tacc;
       pad_off[E] = tacc * kTileM;
+      if (pair_off != nullptr) pair_off[E] = pacc;
     }
   }
   __syncthreads();
@@ -251,7 +256,8 @@ cudaError_t launch_route(const moe_plan_s* p, const int32_t* topk_idx, uint8_t* 
       p->E, p->route_blocks, reinterpret_cast<const int32_t*>(ws + L.block_hist),
       reinterpret_cast<int32_t*>(ws + L.counts), reinterpret_cast<int32_t*>(ws + L.offsets),
       reinterpret_cast<int32_t*>(ws + L.tile_off), reinterpret_cast<int32_t*>(ws + L.pad_off),
-      reinterpret_cast<int32_t*>(ws + L.perm), reinterpret_cast<int32_t*>(ws + L.inv),
+      reinterpret_cast<int32_t*>(ws + L.pair_off), reinterpret_cast<int32_t*>(ws + L.perm),
+      reinterpret_cast<int32_t*>(ws + L.inv),
       reinterpret_cast<uint32_t*>(ws + L.err), reinterpret_cast<uint32_t*>(ws + L.sched),
       static_cast<int>(64 + p->rows_cap / kTileM), reinterpret_cast<int32_t*>(ws + L.row_token),
       p->k);
@@ -358,7 +364,7 @@ extern "C" moe_status moe_route_static(const int32_t* topk_idx, int T, int k, in
   route_scatter_kernel<<<nblk, kRouteThreads, 0, st>>>(
       topk_idx, static_cast<int>(S), E, nblk, hist, counts, offsets,
       reinterpret_cast<int32_t*>(scratch + kStaticTileOff),
-      reinterpret_cast<int32_t*>(scratch + kStaticPadOff), perm, inv, err, nullptr, 0, nullptr,
-      k);
+      reinterpret_cast<int32_t*>(scratch + kStaticPadOff), nullptr, perm, inv, err, nullptr, 0,
+      nullptr, k);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

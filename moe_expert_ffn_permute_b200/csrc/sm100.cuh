@@ -99,6 +99,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   }
 }
 
+// Wait with a time limit only (no abort flag): used on the way out of a
+// kernel, to let the tensor core finish before its TMEM is freed.
+__device__ __forceinline__ bool mbar_wait_limited(uint64_t* bar, uint32_t parity,
+                                                  uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer() - t0 > limit_ns) return false;
+  return true;
+}
+
 // cp.async (non-bulk) group completion tracked by an mbarrier: the arrive
 // happens when all of this thread's prior cp.async copies have landed.
 __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {

@@ -112,3 +112,29 @@ def test_tiled_weights_only_for_fp8():
     q = moe.moe_plan(8, 512, 256, 8, 2)
     moe.moe_plan_set_weight_layout(q, True)
     moe.moe_plan_destroy(q)
+
+
+def test_cta_pair_mode_selection_and_launch_count():
+    """The 2-SM GEMM runs only when asked for with tiled FP8 weights; it adds
+    the weight-scale expansion launch to the forward sequence."""
+    p = moe.moe_plan(8192, 7168, 2048, 32, 8)
+    base = moe.moe_forward_launch_count(p)
+    with pytest.raises(moe.MoEError) as ei:          # row-major weights: no pairs
+        moe.moe_plan_set_cta_pairs(p, 2)
+    assert ei.value.status == 2
+    assert not moe.moe_plan_cta_pairs_active(p)
+    moe.moe_plan_set_weight_layout(p, True)
+    for mode, active in ((0, False), (1, False), (2, True), (0, False)):
+        moe.moe_plan_set_cta_pairs(p, mode)
+        assert moe.moe_plan_cta_pairs_active(p) == active
+        assert moe.moe_forward_launch_count(p) == base + (1 if active else 0)
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_plan_set_cta_pairs(p, 3)
+    assert ei.value.status == 1
+    moe.moe_plan_destroy(p)
+    q = moe.moe_plan(64, 512, 256, 8, 2, w_dtype="e2m1")
+    with pytest.raises(moe.MoEError):
+        moe.moe_plan_set_cta_pairs(q, 2)
+    assert not moe.moe_plan_cta_pairs_active(q)
+    moe.moe_plan_destroy(q)
+    assert not moe.moe_plan_cta_pairs_active(None)

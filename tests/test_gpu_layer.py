@@ -255,3 +255,61 @@ def test_tiled_weights_full_size_parity(name, ntok):
     dn = {k: v.cpu().numpy() for k, v in d.items()}
     ref = oracle_tokens(wl, dn, tokens)
     assert_parity(out.float().cpu().numpy()[tokens], ref, wl.name + "-tiled")
+
+
+def _run_mode(wl, d, pairs, debug=False):
+    lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype=wl.w_dtype, act=wl.act,
+                       alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit, tiled_weights=True,
+                       cta_pairs=pairs, debug=debug)
+    w1t, w2t = lay.prepack(d["w1"], d["w2"])
+    out = lay.forward(d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], w1t, d["w1_scales"],
+                      w2t, d["w2_scales"])
+    torch.cuda.synchronize()
+    return out, lay
+
+
+@pytest.mark.parametrize("wl", [WORKLOADS["tiny"], RAGGED, RAGGED_OAI, SINGLE],
+                         ids=lambda w: w.name)
+def test_cta_pair_gemm_bitwise_equal_single_cta(wl):
+    """The 2-SM GEMM (CTA pairs, 256-row tiles) gives the same bytes as the
+    single-CTA GEMM, including experts with an odd number of 128-row tiles
+    (the pair's second CTA then has no rows)."""
+    d = inputs(wl)
+    ref, _ = _run_mode(wl, d, pairs=1)
+    out, lay = _run_mode(wl, d, pairs=2)
+    assert lay.check() == 0
+    assert torch.equal(out, ref)
+
+
+def test_cta_pair_gemm_requant_bytes_exact():
+    wl = RAGGED
+    d = inputs(wl)
+    out, lay = _run_mode(wl, d, pairs=2, debug=True)
+    v = lay.view()
+    rows = v.rows
+    act_t = torch.empty(rows, wl.I, dtype=torch.uint8, device="cuda")
+    moe.moe_copy_act(lay.plan, lay.workspace, act_t)
+    a32 = _ws_bytes(lay, v.act_f32, rows * wl.I * 4).view(torch.float32).view(rows, wl.I)
+    sf = torch.empty(rows, wl.I // 128, dtype=torch.uint8, device="cuda")
+    moe.moe_copy_act_scales(lay.plan, lay.workspace, sf)
+    counts = _ws_bytes(lay, v.counts, 4 * wl.E).view(torch.int32).cpu().numpy()
+    pad = _ws_bytes(lay, v.pad_offsets, 4 * (wl.E + 1)).view(torch.int32).cpu().numpy()
+    act, a32, sf = act_t.cpu().numpy(), a32.cpu().numpy(), sf.cpu().numpy()
+    for e in range(wl.E):
+        r = slice(pad[e], pad[e] + counts[e])
+        q_ref, s_ref = L.requant_1x128(a32[r].astype(np.float64))
+        np.testing.assert_array_equal(act[r], q_ref)
+        np.testing.assert_array_equal(sf[r], s_ref)
+
+
+def test_cta_pair_gemm_full_size_prefill_parity():
+    wl = WORKLOADS["prefill"]
+    d = inputs(wl)
+    out, lay = _run_mode(wl, d, pairs=2)
+    assert moe.moe_plan_cta_pairs_active(lay.plan)
+    assert lay.check() == 0
+    rng = np.random.default_rng(5)
+    tokens = np.sort(rng.choice(wl.T, size=8, replace=False))
+    dn = {k: v.cpu().numpy() for k, v in d.items()}
+    ref = oracle_tokens(wl, dn, tokens)
+    assert_parity(out.float().cpu().numpy()[tokens], ref, "prefill-pairs")
