@@ -152,6 +152,15 @@ moe_status moe_route(moe_plan_t plan, const int32_t *topk_idx, void *workspace,
 moe_status moe_gather(moe_plan_t plan, const void *x, const uint8_t *x_scales,
                       void *workspace, moe_stream_t stream);
 
+/* Steps 1 and 2 together: the same results as moe_route() followed by
+ * moe_gather() (every workspace byte except the multi-block routing scratch).
+ * Up to 4096 slots this is one launch in which each block repeats the
+ * counting sort in shared memory and then copies its share of rows; above
+ * that it enqueues the separate launches.  moe_forward() uses it.  Same
+ * argument rules as the two calls.                                          */
+moe_status moe_route_gather(moe_plan_t plan, const int32_t *topk_idx, const void *x,
+                            const uint8_t *x_scales, void *workspace, moe_stream_t stream);
+
 /* Step 3, FC1: the FC1 grouped GEMM on the 5th-generation tensor cores with
  * the block scales applied in hardware, the fused (OAI-)SwiGLU, and the FP8
  * E4M3 + UE8M0 1x128 requantisation of the activation, all in one kernel.

@@ -54,6 +54,7 @@ _SIGS = {
     "moe_forward": (ctypes.c_int, [_P] * 12),
     "moe_forward_hostio": (ctypes.c_int, [_P] * 12),
     "moe_route": (ctypes.c_int, [_P] * 4),
+    "moe_route_gather": (ctypes.c_int, [_P] * 6),
     "moe_quantize_act": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int, _P, _P, _P]),
     "moe_route_static": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int] + [_P] * 5),
     "moe_gather": (ctypes.c_int, [_P] * 5),
@@ -184,6 +185,12 @@ ROUTE_STATIC_MAX_SLOTS = 1 << 20
 def moe_gather(plan, x, x_scales, workspace, stream=None):
     _check(lib().moe_gather(plan, *map(_ptr, (x, x_scales, workspace)), _stream(stream)),
            "moe_gather")
+
+
+def moe_route_gather(plan, topk_idx, x, x_scales, workspace, stream=None):
+    """moe_route + moe_gather (one launch up to 4096 slots)."""
+    _check(lib().moe_route_gather(plan, *map(_ptr, (topk_idx, x, x_scales, workspace)),
+                                  _stream(stream)), "moe_route_gather")
 
 
 def moe_fc1(plan, w1, w1_scales, workspace, stream=None):

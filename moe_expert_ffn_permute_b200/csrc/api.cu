@@ -191,9 +191,11 @@ int moe_plan_cta_pairs_active(moe_plan_t plan) {
 
 int moe_forward_launch_count(moe_plan_t plan) {
   if (plan == nullptr) return 0;
-  // [route histogram,] route scan+scatter, gather, [pair scale expansion,]
-  // FC1+FC2 (one launch), combine
-  return (plan->route_blocks > 1 ? 1 : 0) + (use_pairs(plan) ? 1 : 0) + 4;
+  // Routing + gather (one launch up to kFusedMaxSlots slots; else [route
+  // histogram,] route scan+scatter, gather), [pair scale expansion,] FC1+FC2
+  // (one launch), combine.
+  const int front = plan->S <= moe::kFusedMaxSlots ? 1 : (plan->route_blocks > 1 ? 3 : 2);
+  return front + (use_pairs(plan) ? 1 : 0) + 2;
 }
 
 moe_status moe_route(moe_plan_t plan, const int32_t* topk_idx, void* workspace,
@@ -215,6 +217,21 @@ moe_status moe_gather(moe_plan_t plan, const void* x, const uint8_t* x_scales, v
   return cuda_status(moe::launch_gather(plan, static_cast<const uint8_t*>(x), x_scales,
                                         static_cast<uint8_t*>(workspace),
                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_route_gather(moe_plan_t plan, const int32_t* topk_idx, const void* x,
+                            const uint8_t* x_scales, void* workspace, moe_stream_t stream) {
+  moe_status s = check_ws(plan, workspace);
+  if (s != MOE_OK) return s;
+  if (topk_idx == nullptr || x == nullptr || x_scales == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned(topk_idx, 4) || !aligned(x, 16)) return MOE_ERR_ALIGNMENT;
+  if (plan->S > moe::kFusedMaxSlots) {
+    if ((s = moe_route(plan, topk_idx, workspace, stream)) != MOE_OK) return s;
+    return moe_gather(plan, x, x_scales, workspace, stream);
+  }
+  return cuda_status(moe::launch_route_gather(plan, topk_idx, static_cast<const uint8_t*>(x),
+                                              x_scales, static_cast<uint8_t*>(workspace),
+                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_fc1(moe_plan_t plan, const void* w1, const uint8_t* w1_scales, void* workspace,
@@ -272,8 +289,7 @@ moe_status moe_forward(moe_plan_t plan, const void* x, const uint8_t* x_scales,
     return MOE_ERR_ALIGNMENT;
   if ((s = check_weights(plan, w1, w1_scales)) != MOE_OK) return s;
   if ((s = check_weights(plan, w2, w2_scales)) != MOE_OK) return s;
-  if ((s = moe_route(plan, topk_idx, workspace, stream)) != MOE_OK) return s;
-  if ((s = moe_gather(plan, x, x_scales, workspace, stream)) != MOE_OK) return s;
+  if ((s = moe_route_gather(plan, topk_idx, x, x_scales, workspace, stream)) != MOE_OK) return s;
   // FC1 and FC2 share one persistent launch: FC2 tiles of an m-tile start as
   // soon as that m-tile's FC1 tiles are done (no wave tail between the GEMMs).
   if ((s = moe_fc1_fc2(plan, w1, w1_scales, w2, w2_scales, workspace, stream)) != MOE_OK)

@@ -14,7 +14,7 @@
 namespace moe {
 namespace {
 
-constexpr int kMaxK = 16;
+constexpr int kMaxK = 8;   // slots per group of loads (larger k loops over groups)
 
 __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ y,
                                                       const float* __restrict__ topk_w,
@@ -31,19 +31,24 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
 #pragma unroll
   for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
   for (int j0 = 0; j0 < k; j0 += kMaxK) {
-    // Issue every load of this group before using any (more bytes in flight).
+    // Issue every load of this group before using any: the routing check, the
+    // weight and the y vector of a slot are independent loads (a slot that
+    // was not routed has a y row too, of stale bytes, which are never used).
+    int iv[kMaxK];
     float w[kMaxK];
     uint4 v[kMaxK];
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) {
       const long long s = static_cast<long long>(t) * k + j0 + j;
-      const bool live = (j0 + j < k) && __ldg(&inv[s]) >= 0;
-      w[j] = live ? __ldg(&topk_w[s]) : 0.0f;
-      v[j] = live ? __ldcs(reinterpret_cast<const uint4*>(y + s * H) + c) : make_uint4(0, 0, 0, 0);
+      const bool in = j0 + j < k;
+      iv[j] = in ? __ldg(&inv[s]) : -1;
+      w[j] = in ? __ldg(&topk_w[s]) : 0.0f;
+      v[j] = in ? __ldcs(reinterpret_cast<const uint4*>(y + s * H) + c) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) {
       if (j0 + j >= k) break;
+      if (iv[j] < 0) continue;
       const uint32_t wv[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {

@@ -73,6 +73,10 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // Kernel launchers (return cudaGetLastError()).
 cudaError_t launch_route(const moe_plan_s* p, const int32_t* topk_idx, uint8_t* ws,
                          cudaStream_t st);
+// Routing and gather fused in one launch (slot counts up to kFusedMaxSlots).
+constexpr int kFusedMaxSlots = 4096;
+cudaError_t launch_route_gather(const moe_plan_s* p, const int32_t* topk_idx, const uint8_t* x,
+                                const uint8_t* xs, uint8_t* ws, cudaStream_t st);
 cudaError_t launch_gather(const moe_plan_s* p, const uint8_t* x, const uint8_t* xs, uint8_t* ws,
                           cudaStream_t st);
 cudaError_t launch_fc1(const moe_plan_s* p, const void* w1, const uint8_t* w1s, uint8_t* ws,

@@ -13,6 +13,7 @@
 // the scale chunks can be addressed per tile.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "internal.h"
@@ -226,6 +227,192 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(
   }
 }
 
+// Routing and gather in one launch, for small slot counts (S <= kFusedMaxSlots):
+// every block loads the slot ids into shared memory and repeats the counting
+// sort there (histogram, exclusive scan, stable scatter by __match_any_sync
+// ranks, as route_scatter_kernel), so no block waits for another; block 0
+// also publishes what the separate routing launch writes (counts, offsets,
+// tile / pad / pair offsets, perm, inv, the row -> token map, the zeroed
+// GEMM counters, the error bit).  Then each warp copies routed rows: sorted
+// position pos of expert e goes to padded row 128 * tile_off[e] + pos -
+// offsets[e], from token perm[pos] / k, in the same tiled layout and scale
+// chunks as gather_kernel.  The bytes written equal those of the two separate
+// launches.
+__global__ void __launch_bounds__(kRouteThreads) route_gather_kernel(
+    const int32_t* __restrict__ idx, int S, int E, int k, const uint8_t* __restrict__ x,
+    const uint8_t* __restrict__ xs, int H, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ tile_off, int32_t* __restrict__ pad_off,
+    int32_t* __restrict__ pair_off, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+    uint32_t* err, uint32_t* __restrict__ sched, int sched_words,
+    int32_t* __restrict__ row_token, uint8_t* __restrict__ xg, uint8_t* __restrict__ xg_sf) {
+  constexpr int kWarps = kRouteThreads / 32;
+  extern __shared__ int32_t dyn[];
+  int32_t* ids = dyn;          // [S] expert id per slot (-1: not routed)
+  int32_t* sorted = dyn + S;   // [S] slot at each sorted position
+  __shared__ int32_t running[256];
+  __shared__ int32_t total[256];
+  __shared__ int32_t scan[257];
+  __shared__ int32_t tscan[257];
+  __shared__ int32_t wcount[kWarps][256];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool lead = blockIdx.x == 0;
+  griddep_launch_dependents();
+  griddep_wait();
+  if (lead && sched != nullptr)
+    for (int i = tid; i < sched_words; i += blockDim.x) sched[i] = 0u;
+  for (int e = tid; e < E; e += blockDim.x) total[e] = 0;
+  __syncthreads();
+  bool bad = false;
+  // All of this thread's ids are loaded before any is used (one round trip).
+  constexpr int kPer = kFusedMaxSlots / kRouteThreads;
+  int v[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int i = tid + u * kRouteThreads;
+    v[u] = i < S ? __ldg(&idx[i]) : kMaskedSlot;
+  }
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int i = tid + u * kRouteThreads;
+    if (i >= S) break;
+    int e = v[u];
+    if (e >= 0 && e < E) {
+      atomicAdd(&total[e], 1);
+    } else {
+      if (e != kMaskedSlot) bad = true;
+      e = -1;
+    }
+    ids[i] = e;
+  }
+  if (lead && bad) atomicOr(err, kErrRoutingBit);
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0, tacc = 0, pacc = 0;
+    for (int e = 0; e < E; ++e) {
+      scan[e] = acc;
+      tscan[e] = tacc;
+      running[e] = acc;
+      const int tiles = (total[e] + kTileM - 1) / kTileM;
+      if (lead) {
+        offsets[e] = acc;
+        counts[e] = total[e];
+        tile_off[e] = tacc;
+        pad_off[e] = tacc * kTileM;
+        pair_off[e] = pacc;
+      }
+      acc += total[e];
+      tacc += tiles;
+      pacc += (tiles + 1) / 2;
+    }
+    scan[E] = acc;
+    tscan[E] = tacc;
+    if (lead) {
+      offsets[E] = acc;
+      tile_off[E] = tacc;
+      pad_off[E] = tacc * kTileM;
+      pair_off[E] = pacc;
+    }
+  }
+  __syncthreads();
+  const int routed = scan[E];
+  if (lead) {
+    for (int e = 0; e < E; ++e) {
+      const int lo = tscan[e] * kTileM + total[e], hi = tscan[e + 1] * kTileM;
+      for (int r = lo + tid; r < hi; r += blockDim.x) row_token[r] = -1;
+    }
+    for (int q = routed + tid; q < S; q += blockDim.x) perm[q] = -1;
+  }
+  for (int sub = 0; sub < S; sub += kRouteThreads) {
+    for (int i = tid; i < kWarps * 256; i += blockDim.x) (&wcount[0][0])[i] = 0;
+    __syncthreads();
+    const int sl = sub + tid;
+    const int e = sl < S ? ids[sl] : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (e >= 0 && rank == 0) wcount[warp][e] = __popc(peers);
+    __syncthreads();
+    if (sl < S) {
+      if (e >= 0) {
+        int q = running[e] + rank;
+        for (int w = 0; w < warp; ++w) q += wcount[w][e];
+        sorted[q] = sl;   // q < routed <= S: the counts above bound it
+        if (lead) {
+          perm[q] = sl;
+          inv[sl] = q;
+          row_token[tscan[e] * kTileM + (q - scan[e])] = sl / k;
+        }
+      } else if (lead) {
+        inv[sl] = -1;
+      }
+    }
+    __syncthreads();
+    for (int ee = tid; ee < E; ee += blockDim.x) {
+      int add = 0;
+      for (int w = 0; w < kWarps; ++w) add += wcount[w][ee];
+      running[ee] += add;
+    }
+    __syncthreads();
+  }
+  // Gather: one warp per routed row; all loads of a row are issued before its
+  // stores.
+  const int kb_n = H / 128;
+  const int vec = H / 16;
+  for (int q = blockIdx.x * kWarps + warp; q < routed; q += gridDim.x * kWarps) {
+    int lo = 0, hi = E - 1;   // expert of sorted position q: largest e with scan[e] <= q
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (scan[mid] <= q) lo = mid; else hi = mid - 1;
+    }
+    const int e = lo;
+    const long long P = static_cast<long long>(tscan[e]) * kTileM + (q - scan[e]);
+    const int t = sorted[q] / k;
+    const int tile = static_cast<int>(P / kTileM);
+    const int r = static_cast<int>(P % kTileM);
+    const uint4* __restrict__ src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
+    uint8_t* __restrict__ dst = xg + static_cast<size_t>(tile) * kb_n * kTileBytes;
+    // Rows of up to 8192 bytes (H <= 8192) move in one batch of loads; the
+    // scale bytes (up to 64 per row) are loaded with them.
+    constexpr int kBatch = 16;
+    uint8_t* chunk = xg_sf + static_cast<size_t>(tile) * kb_n * 512 + (r & 31) * 16 + (r >> 5) * 4;
+    for (int c0 = lane; c0 < vec; c0 += 32 * kBatch) {
+      uint4 xv[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int c = c0 + 32 * u;
+        if (c < vec) xv[u] = __ldg(&src[c]);
+      }
+      uint32_t sb[2] = {0u, 0u};
+      if (c0 == lane) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int kb = lane + 32 * u;
+          if (kb < kb_n) sb[u] = __ldg(&xs[static_cast<size_t>(t) * kb_n + kb]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int c = c0 + 32 * u;
+        if (c < vec)
+          *reinterpret_cast<uint4*>(dst + static_cast<size_t>(c >> 3) * kTileBytes +
+                                    swz128(r, c & 7)) = xv[u];
+      }
+      if (c0 == lane) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int kb = lane + 32 * u;
+          if (kb < kb_n)
+            *reinterpret_cast<uint32_t*>(chunk + static_cast<size_t>(kb) * 512) =
+                sb[u] * 0x01010101u;
+        }
+      }
+    }
+    for (int kb = lane + 64; kb < kb_n; kb += 32) {   // H > 8192
+      const uint32_t b = __ldg(&xs[static_cast<size_t>(t) * kb_n + kb]);
+      *reinterpret_cast<uint32_t*>(chunk + static_cast<size_t>(kb) * 512) = b * 0x01010101u;
+    }
+  }
+}
+
 // Unpack the FC1 activation's scale chunks to a plain u8 [rows, I/128] array.
 __global__ void unpack_act_scales_kernel(const uint8_t* __restrict__ chunks, int nb,
                                          long long rows, uint8_t* __restrict__ dst) {
@@ -270,6 +457,30 @@ cudaError_t launch_gather(const moe_plan_s* p, const uint8_t* x, const uint8_t* 
   return launch_pdl(gather_kernel, dim3(blocks), dim3(kGatherWarps * 32), 0, st, x, xs, p->H,
                     p->E, reinterpret_cast<const int32_t*>(ws + L.pad_off),
                     reinterpret_cast<const int32_t*>(ws + L.row_token), ws + L.xg, ws + L.xg_sf);
+}
+
+cudaError_t launch_route_gather(const moe_plan_s* p, const int32_t* topk_idx, const uint8_t* x,
+                                const uint8_t* xs, uint8_t* ws, cudaStream_t st) {
+  const auto& L = p->ws;
+  const int S = static_cast<int>(p->S);
+  // One warp per routed row (at most S), two blocks per SM at most.
+  int sms = 148;
+  {
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  const int want = (S + kRouteThreads / 32 - 1) / (kRouteThreads / 32);
+  const int blocks = std::max(1, std::min(want, 2 * sms));
+  return launch_pdl(
+      route_gather_kernel, dim3(blocks), dim3(kRouteThreads), 2 * S * sizeof(int32_t), st,
+      topk_idx, S, p->E, p->k, x, xs, p->H, reinterpret_cast<int32_t*>(ws + L.counts),
+      reinterpret_cast<int32_t*>(ws + L.offsets), reinterpret_cast<int32_t*>(ws + L.tile_off),
+      reinterpret_cast<int32_t*>(ws + L.pad_off), reinterpret_cast<int32_t*>(ws + L.pair_off),
+      reinterpret_cast<int32_t*>(ws + L.perm), reinterpret_cast<int32_t*>(ws + L.inv),
+      reinterpret_cast<uint32_t*>(ws + L.err), reinterpret_cast<uint32_t*>(ws + L.sched),
+      static_cast<int>(64 + p->rows_cap / kTileM), reinterpret_cast<int32_t*>(ws + L.row_token),
+      ws + L.xg, ws + L.xg_sf);
 }
 
 cudaError_t launch_unpack_act_scales(const moe_plan_s* p, const uint8_t* ws, uint8_t* dst,

@@ -8,8 +8,8 @@ import moe_expert_ffn_permute_b200 as moe
 from moe_expert_ffn_permute_b200.synth import WORKLOADS, Workload, to_numpy
 from oracle import layer as L
 
-from gpu_helpers import (assert_parity, ensure_built, inputs, oracle_args, oracle_kw,
-                         oracle_tokens, run_gpu)
+from gpu_helpers import (assert_parity, ensure_built, inputs, layer_for, oracle_args,
+                         oracle_kw, oracle_tokens, run_gpu)
 
 pytestmark = pytest.mark.gpu
 
@@ -313,3 +313,67 @@ def test_cta_pair_gemm_full_size_prefill_parity():
     dn = {k: v.cpu().numpy() for k, v in d.items()}
     ref = oracle_tokens(wl, dn, tokens)
     assert_parity(out.float().cpu().numpy()[tokens], ref, "prefill-pairs")
+
+
+def _whole_workspace_after(lay, d, fused):
+    """Fill the workspace with a fixed byte pattern, run the layer either as
+    moe_forward (routing and gather fused at small slot counts) or as the
+    separate step calls, and return the entire workspace."""
+    lay.workspace.fill_(0x5A)
+    moe.moe_clear_device_error(lay.plan, lay.workspace)
+    out = torch.zeros(d["x"].shape[0], lay.H, dtype=torch.bfloat16, device="cuda")
+    if fused == "forward":
+        moe.moe_forward(lay.plan, d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], d["w1"],
+                        d["w1_scales"], d["w2"], d["w2_scales"], out, lay.workspace)
+    elif fused == "steps":
+        moe.moe_route_gather(lay.plan, d["topk_idx"], d["x"], d["x_scales"], lay.workspace)
+        moe.moe_fc1_fc2(lay.plan, d["w1"], d["w1_scales"], d["w2"], d["w2_scales"],
+                        lay.workspace)
+        moe.moe_combine(lay.plan, d["topk_w"], out, lay.workspace)
+    else:
+        moe.moe_route(lay.plan, d["topk_idx"], lay.workspace)
+        moe.moe_gather(lay.plan, d["x"], d["x_scales"], lay.workspace)
+        moe.moe_fc1_fc2(lay.plan, d["w1"], d["w1_scales"], d["w2"], d["w2_scales"],
+                        lay.workspace)
+        moe.moe_combine(lay.plan, d["topk_w"], out, lay.workspace)
+    torch.cuda.synchronize()
+    return lay.workspace.clone(), out
+
+
+@pytest.mark.parametrize("case", ["ragged", "masked", "bad-ids", "decode", "boundary-4096"])
+def test_fused_route_gather_writes_the_same_bytes(case):
+    """At slot counts up to 4096 moe_forward routes and gathers in one launch;
+    every workspace byte (routing arrays, padding map, gathered tiles and
+    scale chunks, GEMM counters, error word) and the output equal those of the
+    separate launches."""
+    if case == "decode":
+        wl = WORKLOADS["decode"]
+    elif case == "boundary-4096":
+        wl = Workload("boundary", 512, 1024, 256, 16, 8, cfg_id=24)   # S = 4096
+    else:
+        wl = RAGGED
+    d = inputs(wl)
+    if case == "masked":
+        d["topk_idx"][torch.rand(wl.T, wl.k, device="cuda") < 0.25] = -1
+    if case == "bad-ids":
+        d["topk_idx"][5, 2] = -3
+        d["topk_idx"][100, 0] = wl.E + 7
+    lay = layer_for(wl, False)
+    assert moe.moe_forward_launch_count(lay.plan) == 3
+    ws_sep, out_sep = _whole_workspace_after(lay, d, fused=None)
+    for how in ("forward", "steps"):     # moe_forward, and moe_route_gather + later steps
+        ws_fused, out_fused = _whole_workspace_after(lay, d, fused=how)
+        assert torch.equal(out_fused, out_sep), how
+        diff = (ws_fused != ws_sep).nonzero().flatten()
+        if wl.T * wl.k > 2048:
+            # The separate path then routes with two blocks whose histogram
+            # scratch (between the padded offsets and perm) the fused launch
+            # does not need: only bytes there may differ.
+            base, v = lay.workspace.data_ptr(), lay.view()
+            assert diff.numel() <= 2 * wl.E * 4, how
+            if diff.numel():
+                assert int(diff.min()) >= v.pad_offsets - base, how
+                assert int(diff.max()) < v.perm - base, how
+        else:
+            assert diff.numel() == 0, how
+        assert lay.check() == (6 if case == "bad-ids" else 0)
