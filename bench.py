@@ -252,28 +252,34 @@ def run_b200(args, wl):
 
     soak(0.6)
     step_ms = timed(step)
+    # ---- per-kernel split (the launch sequence of moe_forward, one event per
+    # step boundary, on the launching stream), then the unfused launches.
+    split = {name: [] for name, _ in steps + extra}
+
+    def split_timing():
+        for seq in (steps, extra):
+            for i in range(args.steps):
+                flush.fill_(i & 0xFF)
+                evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(seq) + 1)]
+                evs[0].record(stream)
+                for j, (_, fn) in enumerate(seq):
+                    fn()
+                    evs[j + 1].record(stream)
+                torch.cuda.synchronize()
+                for j, (name, _) in enumerate(seq):
+                    split[name].append(evs[j].elapsed_time(evs[j + 1]))
+
+    # Everything on the line is measured in the same sustained state: the
+    # eager calls and the per-kernel split also sit between continuous steps.
     soak(0.3)
-    eager_ms = timed(fwd)        # the same calls launched directly, same power state
+    eager_ms = timed(fwd)
+    soak(0.3)
+    split_timing()
     soak(0.3)
     clk = clocks.stop()
     if world > 1:
         dist.barrier()
     total_ms = sum(step_ms)
-
-    # ---- per-kernel split (the launch sequence of moe_forward, one event per
-    # step boundary, on the launching stream), then the unfused launches.
-    split = {name: [] for name, _ in steps + extra}
-    for seq in (steps, extra):
-        for i in range(args.steps):
-            flush.fill_(i & 0xFF)
-            evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(seq) + 1)]
-            evs[0].record(stream)
-            for j, (_, fn) in enumerate(seq):
-                fn()
-                evs[j + 1].record(stream)
-            torch.cuda.synchronize()
-            for j, (name, _) in enumerate(seq):
-                split[name].append(evs[j].elapsed_time(evs[j + 1]))
 
     # ---- e2e through the host-buffer entry point
     host = {k: d[k].cpu().pin_memory() for k in ("x", "x_scales", "topk_idx", "topk_w")}

@@ -53,7 +53,6 @@ constexpr uint32_t kAccCol = 0, kSfaCol = 256, kSfbCol = 264, kSfSetStride = 16;
 constexpr int kEpiWarps = 8;
 constexpr int kSchedConsumers = 3 + kEpiWarps;   // 2 producers, MMA, epilogue warps
 constexpr uint64_t kDepWaitLimitNs = 2000000000ull;
-constexpr int kPrefetch = 8;   // weight k-blocks prefetched into L2 ahead of the loads
 
 struct __align__(1024) Smem {
   uint8_t a[STAGES][BM * BK];
@@ -316,34 +315,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (sm.abort_flag) break;
       }
-      // MXFP4 weight tiles stream from HBM at half the bytes per stage of FP8
-      // (the TMA widens them in shared memory), so STAGES x HBM latency bounds
-      // the pipeline: keep kPrefetch more k-blocks on their way into L2.
-      // (Measured: +9-13% for MXFP4 at 128-1024 tokens; FP8 weights fill the
-      // stages with twice the bytes and lost bandwidth with it, so they don't.)
-      auto prefetch_b = [&](int kb) {
-        if (ph.w_tiles != nullptr) {
-          prefetch_l2_bulk(ph.w_tiles + (static_cast<size_t>(brow0 / 128) * ph.k_blocks + kb) *
-                                            kTileBytes, kTileBytes);
-          prefetch_l2_bulk(ph.w_tiles + (static_cast<size_t>(brow1 / 128) * ph.k_blocks + kb) *
-                                            kTileBytes, kTileBytes);
-        } else {
-          prefetch_l2_tile_2d(tb, kb * BK, brow0);
-          if (t.kind == 0) prefetch_l2_tile_2d(tb, kb * BK, brow1);
-        }
-      };
-      if (kFp4 && operands && lane == 0) {
-        for (int kb = 0; kb < kPrefetch && kb < ph.k_blocks; ++kb) prefetch_b(kb);
-        if ((reinterpret_cast<uintptr_t>(ph.w_sf) & 15) == 0) {
-          // The tile's 1x32 weight scales: 128 rows of K/32 bytes each,
-          // contiguous (128 * K/32 is a multiple of 16).
-          const size_t kw = static_cast<size_t>(ph.k_blocks) * 4;
-          prefetch_l2_bulk(ph.w_sf + static_cast<size_t>(brow0) * kw,
-                           static_cast<uint32_t>(128 * kw));
-          prefetch_l2_bulk(ph.w_sf + static_cast<size_t>(brow1) * kw,
-                           static_cast<uint32_t>(128 * kw));
-        }
-      }
       uint32_t sf0 = 0, sf1 = 0;   // FP8 weight scales for k-blocks kb = 32*c + lane
       for (int kb = 0; kb < ph.k_blocks; ++kb) {
         if (!operands && !kFp4 && (kb & 31) == 0) {
@@ -382,7 +353,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
               tma_load_2d(sm.b[stage], tb, kb * BK, brow0, &sm.full[stage], pol_b);
             }
-            if (kFp4 && kb + kPrefetch < ph.k_blocks) prefetch_b(kb + kPrefetch);
           }
           __syncwarp();
         } else {

@@ -168,22 +168,6 @@ __device__ __forceinline__ void bulk_load_hint(void* smem_dst, const void* gmem_
       : "memory");
 }
 
-// L2 prefetch of a global range (16-byte aligned address and size): no
-// shared memory is written and nothing completes on a barrier.
-__device__ __forceinline__ void prefetch_l2_bulk(const void* gmem_src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem_src), "r"(bytes)
-               : "memory");
-}
-
-// L2 prefetch of the 2-D box a tensor map would load at (c0, c1).
-__device__ __forceinline__ void prefetch_l2_tile_2d(const CUtensorMap* map, int32_t c0,
-                                                    int32_t c1) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(c0), "r"(c1)
-               : "memory");
-}
-
 // Operand tiles stored "pre-swizzled": a 128 x 128-byte tile is 16 KB,
 // contiguous, with byte c of row r at r * 128 + (((c / 16) ^ (r % 8)) * 16) +
 // c % 16 -- exactly the 128-byte-swizzled layout the tensor core reads, so one
