@@ -14,6 +14,8 @@ format definitions:
   E2M1:       1 sign, 2 exponent (bias 1), 1 mantissa bit; magnitudes
               {0, 0.5, 1, 1.5, 2, 3, 4, 6}; no NaN / inf.
   UE8M0:      8-bit unsigned exponent, value 2^(b-127); b = 255 is NaN.
+  BF16:       the upper 16 bits of an IEEE-754 binary32 (1 sign, 8 exponent
+              bits with bias 127, 7 mantissa bits); same range as binary32.
 
 Parity: pinned by exhaustive enumeration against torch's float8_e4m3fn /
 float8_e8m0fnu / float4_e2m1fn_x2 dtypes (library routines used only in the
@@ -88,3 +90,35 @@ def decode_ue8m0(codes):
     b = np.asarray(codes, dtype=np.uint8).astype(np.int64)
     val = np.exp2(b - 127.0)
     return np.where(b == 255, np.nan, val)
+
+
+BF16_MAX = (2.0 - 2.0 ** -7) * 2.0 ** 127
+
+
+def decode_bf16(bits):
+    """BF16 bit patterns (uint16) -> float64: the pattern is the upper half of a
+    binary32, so widening it by 16 zero bits gives the exact value."""
+    b = np.asarray(bits).astype(np.uint32) << np.uint32(16)
+    with np.errstate(invalid="ignore"):
+        return b.view(np.float32).astype(np.float64)
+
+
+def encode_bf16_rne(values):
+    """float64 -> BF16 bit patterns (uint16), rounding the exact value to the
+    nearest BF16 number with ties to the even mantissa; magnitudes that round
+    past the largest finite value give infinity; NaN gives 0x7FC0.
+
+    Rounding step: for |v| in [2^E, 2^(E+1)) the BF16 spacing is 2^(E-7), and
+    2^-133 below the smallest normal 2^-126 (8 significant bits, 7 stored)."""
+    v = np.asarray(values, dtype=np.float64)
+    a = np.abs(v)
+    with np.errstate(divide="ignore", invalid="ignore", over="ignore"):
+        _, ex = np.frexp(a)                       # a = m * 2^ex, m in [0.5, 1)
+        E = np.maximum(ex.astype(np.int64) - 1, -126)
+        q = np.ldexp(1.0, (E - 7).astype(np.int64))
+        r = np.rint(a / q) * q                    # rint: round half to even
+    r = np.where(a == 0, 0.0, r)
+    r = np.where(r > BF16_MAX, np.inf, r)
+    r = np.where(np.isinf(a), np.inf, r)
+    out = (np.copysign(r, v).astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    return np.where(np.isnan(v), np.uint16(0x7FC0), out).astype(np.uint16)

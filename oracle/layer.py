@@ -48,8 +48,8 @@ import math
 
 import numpy as np
 
-from .formats import (E4M3_MAX, decode_e2m1, decode_e4m3, decode_ue8m0,
-                      encode_e4m3_rne_satfinite, unpack_e2m1_pairs)
+from .formats import (E4M3_MAX, decode_bf16, decode_e2m1, decode_e4m3, decode_ue8m0,
+                      encode_bf16_rne, encode_e4m3_rne_satfinite, unpack_e2m1_pairs)
 
 BLOCK = 128          # activation / FP8-weight scale block along K (and N for weights)
 FP4_BLOCK = 32       # MXFP4 weight scale block along K
@@ -211,6 +211,45 @@ def layer(x, x_scales, topk_idx, topk_w, w1, w1_scales, w2, w2_scales,
     return out
 
 
+def layer_bf16(x, topk_idx, topk_w, w1, w2, alpha=1.0, up_bias=0.0, limit=math.inf,
+               keep=False):
+    """The BF16 variant of the layer (fw-ai/DeepGEMM PR #16 "Overview": BF16 and
+    FP8/FP4 Mega MoE share the scheduler) in float64: x [T,H], w1 [E,2I,H] and
+    w2 [E,H,I] are BF16 bit patterns (uint16), no block scales.  Reading (the
+    pages name the variant only): the activation a goes to FC2 as BF16 (round to
+    nearest even) instead of FP8 + 1x128 scales; everything else as in layer()."""
+    T, k = np.asarray(topk_idx).shape
+    E = w1.shape[0]
+    H = x.shape[1]
+    I = w2.shape[2]
+    counts, offsets, perm, inv = route(topk_idx, E)
+    xh = decode_bf16(x)
+    S = T * k
+    y = np.zeros((S, H), dtype=np.float64)
+    inter = {"h": {}, "a": {}, "ab": {}}
+    for e in range(E):
+        slots = perm[offsets[e]:offsets[e + 1]]
+        if slots.shape[0] == 0:
+            continue
+        tokens = slots // k
+        h = xh[tokens] @ decode_bf16(w1[e]).T                   # [n_e, 2I]
+        a = swiglu(h[:, :I], h[:, I:], alpha, up_bias, limit)   # [n_e, I]
+        ab = encode_bf16_rne(a)
+        y[slots] = decode_bf16(ab) @ decode_bf16(w2[e]).T        # [n_e, H]
+        if keep:
+            inter["h"][e], inter["a"][e], inter["ab"][e] = h, a, ab
+    w = np.asarray(topk_w, dtype=np.float64)
+    out = np.zeros((T, H), dtype=np.float64)
+    for t in range(T):
+        for j in range(k):
+            if inv[t * k + j] >= 0:
+                out[t] += w[t, j] * y[t * k + j]
+    if keep:
+        inter.update(counts=counts, offsets=offsets, perm=perm, inv=inv, y=y)
+        return out, inter
+    return out
+
+
 # ------------------------------------------------------------- brute-force tier (tiny)
 def _e4m3_scalar(b):
     s = -1.0 if b & 0x80 else 1.0
@@ -289,3 +328,51 @@ def _rne_e4m3_scalar(v):
             best, best_code = d, code
     r = _e4m3_scalar(best_code)
     return -r if v < 0 else r
+
+
+def _bf16_scalar(bits):
+    """BF16 pattern -> float via the binary32 bytes (struct, not numpy)."""
+    import struct
+    return struct.unpack("<f", struct.pack("<I", (int(bits) & 0xFFFF) << 16))[0]
+
+
+def _rne_bf16_scalar(v):
+    """Nearest BF16 value to v, ties to even mantissa, past the top -> inf:
+    Python's round() (half to even) on v scaled by the spacing at v."""
+    if v == 0.0 or math.isinf(v) or math.isnan(v):
+        return v
+    m, ex = math.frexp(abs(v))            # |v| = m * 2^ex, m in [0.5, 1)
+    e = max(ex - 1, -126)
+    r = round(abs(v) / 2.0 ** (e - 7)) * 2.0 ** (e - 7)
+    if r > (2.0 - 2.0 ** -7) * 2.0 ** 127:
+        r = math.inf
+    return -r if v < 0 else r
+
+
+def layer_bf16_bruteforce(x, topk_idx, topk_w, w1, w2, alpha=1.0, up_bias=0.0,
+                          limit=math.inf):
+    """Element-by-element pure-Python statement of layer_bf16 (tiny shapes)."""
+    T, k = np.asarray(topk_idx).shape
+    H = x.shape[1]
+    I = w2.shape[2]
+    E = w1.shape[0]
+    out = [[0.0] * H for _ in range(T)]
+    for t in range(T):
+        xh = [_bf16_scalar(x[t, c]) for c in range(H)]
+        for j in range(k):
+            e = int(topk_idx[t, j])
+            if e < 0 or e >= E:
+                continue
+            ab = []
+            for i in range(I):
+                g = sum(xh[c] * _bf16_scalar(w1[e, i, c]) for c in range(H))
+                u = sum(xh[c] * _bf16_scalar(w1[e, I + i, c]) for c in range(H))
+                gc = min(g, limit)
+                uc = max(-limit, min(u, limit))
+                a = (gc / (1.0 + math.exp(-alpha * gc)) * (uc + up_bias)
+                     if -alpha * gc < 700 else 0.0)
+                ab.append(_rne_bf16_scalar(a))
+            for c in range(H):
+                yc = sum(ab[i] * _bf16_scalar(w2[e, c, i]) for i in range(I))
+                out[t][c] += float(topk_w[t, j]) * yc
+    return np.array(out)
