@@ -141,8 +141,11 @@ def algorithmic_bytes(wl, d):
     import torch
     counts = torch.bincount(d["topk_idx"].reshape(-1).long(), minlength=wl.E)[:wl.E]
     active = int((counts > 0).sum())
-    per_expert_w = sum(d[k][0].numel() for k in ("w1", "w1_scales", "w2", "w2_scales"))
-    act_bytes = (d["x"].numel() + d["x_scales"].numel() + d["topk_idx"].numel() * 4 +
+    def nbytes(t):
+        return 0 if t is None else t.numel() * t.element_size()
+    per_expert_w = sum(nbytes(d[k][0]) if d[k] is not None else 0
+                       for k in ("w1", "w1_scales", "w2", "w2_scales"))
+    act_bytes = (nbytes(d["x"]) + nbytes(d["x_scales"]) + d["topk_idx"].numel() * 4 +
                  d["topk_w"].numel() * 4 + wl.T * wl.H * 2)
     return active * per_expert_w + act_bytes, active * per_expert_w, active
 
@@ -168,7 +171,7 @@ def run_b200(args, wl):
     d = make_inputs(wl, device=dev)
     # FP8 weights are rearranged once into the tensor-core tile layout (as at
     # model load); the timed steps read them in that layout.
-    tiled = wl.w_dtype == "e4m3" and not args.row_major_weights
+    tiled = wl.w_dtype in ("e4m3", "bf16") and not args.row_major_weights
     lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype=wl.w_dtype, act=wl.act,
                        alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit, device=dev,
                        tiled_weights=tiled, cta_pairs=args.cta_pairs if tiled else None)
@@ -282,7 +285,8 @@ def run_b200(args, wl):
     total_ms = sum(step_ms)
 
     # ---- e2e through the host-buffer entry point
-    host = {k: d[k].cpu().pin_memory() for k in ("x", "x_scales", "topk_idx", "topk_w")}
+    host = {k: (None if d[k] is None else d[k].cpu().pin_memory())
+            for k in ("x", "x_scales", "topk_idx", "topk_w")}
     out_h = torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory()
     for _ in range(args.warmup):
         moe.moe_forward_hostio(lay.plan, host["x"], host["x_scales"], host["topk_idx"],
@@ -313,21 +317,27 @@ def run_b200(args, wl):
     hbm, bf16, bf16_sus, peak_src = _peaks()
     flops = 6.0 * wl.S * wl.H * wl.I
     gemm_ms = statistics.mean(split["fc1_fc2"])
-    hbm_bound = alg_bytes / (hbm * 1e9) > flops / (2 * bf16 * 1e12)
+    # Tensor peak of the GEMM's own input type: the measured bf16 burst for
+    # BF16 weights, twice it for FP8 (and E4M3 x E2M1) operands.
+    tc_mult = 1.0 if wl.w_dtype == "bf16" else 2.0
+    hbm_bound = alg_bytes / (hbm * 1e9) > flops / (tc_mult * bf16 * 1e12)
     if hbm_bound:
         roof = {"bound": "hbm", "achieved": round(w_bytes / (gemm_ms * 1e-3) / 1e9, 1),
                 "peak": hbm, "unit": "GB/s"}
     else:
         roof = {"bound": "tensor", "achieved": round(flops / (gemm_ms * 1e-3) / 1e12, 1),
-                "peak": round(2 * bf16, 1), "unit": "TFLOP/s"}
+                "peak": round(tc_mult * bf16, 1), "unit": "TFLOP/s"}
     roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
     roof["traffic"] = measured_traffic(wl.name)
     roof["kernel"] = (("moe_gemm_pair_kernel (CTA pairs, 2-SM MMA; with its weight-scale "
                        "expansion launch)" if pairs else "moe_gemm_kernel") +
-                      ": FC1 + SwiGLU + FP8 requant and FC2 in one persistent launch")
+                      ": FC1 + SwiGLU + " + ("bf16 activation" if wl.w_dtype == "bf16"
+                                              else "FP8 requant") +
+                      " and FC2 in one persistent launch")
     roof["per_launch"] = (f"{w_bytes} B of expert weights+scales ({active} active experts)"
                           if hbm_bound else f"{flops:.4g} FLOP (6*S*H*I)")
     roof["peak_source"] = f"{peak_src}" + ("" if roof["unit"] == "GB/s" else
+                                           " bf16 burst" if tc_mult == 1.0 else
                                            " bf16 burst x2 (FP8 = 2x bf16 nominal)")
 
     tokens = wl.T * world
@@ -336,7 +346,8 @@ def run_b200(args, wl):
         "metric": METRIC, "value": round(tokens / (total_ms * 1e-3 / args.steps), 1),
         "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "fp8_e4m3" if wl.w_dtype == "e4m3" else "fp8_e4m3xe2m1",
+        "vs_baseline": None, "dtype": {"e4m3": "fp8_e4m3", "e2m1": "fp8_e4m3xe2m1",
+                                       "bf16": "bf16"}[wl.w_dtype],
         "data": "synthetic (seeded; random-init weights)",
         "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
                    "w_dtype": wl.w_dtype, "routing": wl.routing, "act": wl.act,
@@ -351,7 +362,8 @@ def run_b200(args, wl):
         "timing": "CUDA-graph replay of moe_forward, events on the launching stream",
         "roofline": roof,
         "e2e": {"value": round(tokens / (e2e_total * 1e-3 / args.steps), 1), "unit": "tokens/s",
-                "h2d_bytes_per_step": int(sum(v.numel() * v.element_size() for v in host.values())),
+                "h2d_bytes_per_step": int(sum(v.numel() * v.element_size() for v in host.values()
+                                              if v is not None)),
                 "d2h_bytes_per_step": int(out_h.numel() * 2)},
         "gpu_launches": moe.moe_forward_launch_count(lay.plan) * args.steps,
         "clocks": clk,
@@ -369,7 +381,11 @@ def _oracle_sample(wl, dn, tokens):
     from oracle import layer as L
     sub = dict(dn)
     for key in ("x", "x_scales", "topk_idx", "topk_w"):
-        sub[key] = dn[key][tokens]
+        if dn[key] is not None:
+            sub[key] = dn[key][tokens]
+    if wl.w_dtype == "bf16":
+        return L.layer_bf16(sub["x"], sub["topk_idx"], sub["topk_w"], dn["w1"], dn["w2"],
+                            alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit)
     return L.layer(sub["x"], sub["x_scales"], sub["topk_idx"], sub["topk_w"], dn["w1"],
                    dn["w1_scales"], dn["w2"], dn["w2_scales"], w_dtype=wl.w_dtype,
                    alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit)

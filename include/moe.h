@@ -64,13 +64,20 @@ typedef enum {
   MOE_ERR_BAD_ROUTING = 6     /* a topk_idx entry was outside [0, E)            */
 } moe_status;
 
-/* Weight formats.  Activations x are always E4M3 with one UE8M0 per 1x128. */
+/* Weight formats.  With the two block-scaled formats the activations x are
+ * E4M3 with one UE8M0 per 1x128 and the FC1 activation is requantised to that
+ * format.  MOE_W_BF16 is the BF16 variant the pages name next to FP8/FP4
+ * (fw-ai/DeepGEMM PR #16, Overview): x is bf16 [T,H] and x_scales is unused
+ * (may be NULL), W1 bf16 [E,2I,H] and W2 bf16 [E,H,I] with no scales (NULL
+ * allowed), and the FC1 activation goes to FC2 as bf16 (round to nearest
+ * even), fp32 accumulation throughout.                                       */
 typedef enum {
   MOE_W_E4M3_UE8M0_128x128 = 0, /* W1 u8 [E,2I,H], scales u8 [E,2I/128,H/128]  */
-  MOE_W_E2M1_UE8M0_1x32 = 1     /* W1 u8 [E,2I,H/2] (two E2M1 codes per byte,
+  MOE_W_E2M1_UE8M0_1x32 = 1,    /* W1 u8 [E,2I,H/2] (two E2M1 codes per byte,
                                    element 2i in the low nibble),
                                    scales u8 [E,2I,H/32]; W2 likewise [E,H,I/2],
                                    [E,H,I/32]                                   */
+  MOE_W_BF16 = 2                /* W1 bf16 [E,2I,H], W2 bf16 [E,H,I], no scales */
 } moe_wdtype;
 
 typedef struct {
@@ -107,8 +114,8 @@ size_t moe_workspace_bytes(moe_plan_t plan);
 
 /* The whole layer: route -> gather -> FC1 (+ activation + FP8 requant) -> FC2
  * -> combine, enqueued on `stream`.
- *   x          u8 [T,H]      E4M3 codes of the activations
- *   x_scales   u8 [T,H/128]  UE8M0 scale bytes
+ *   x          u8 [T,H]      E4M3 codes of the activations (MOE_W_BF16: bf16 [T,H])
+ *   x_scales   u8 [T,H/128]  UE8M0 scale bytes (MOE_W_BF16: unused, may be NULL)
  *   topk_idx   i32 [T,k]     expert ids
  *   topk_w     f32 [T,k]     combine weights
  *   w1, w1_scales, w2, w2_scales   weights in the plan's moe_wdtype layout
@@ -235,8 +242,9 @@ typedef struct {
   int32_t *perm;        /* [S]                                        */
   int32_t *inv;         /* [S]                                        */
   int32_t *pad_offsets; /* [E+1]  row offsets, multiples of 128       */
-  uint8_t *act;         /* FP8 E4M3 activation (FC1 output), tiled:
-                           read it row-major with moe_copy_act()      */
+  uint8_t *act;         /* FC1 output activation (E4M3, or bf16 for
+                           MOE_W_BF16), tiled: read it row-major with
+                           moe_copy_act()                             */
   float *act_f32;       /* [rows, I]  the activation before requant,
                            written only when debug capture is on      */
   uint16_t *y;          /* [S, H] bf16, slot order (FC2 output)       */
@@ -250,7 +258,8 @@ moe_status moe_workspace_view(moe_plan_t plan, void *workspace,
 /* FP8 scale bytes of the activation (FC1 output) for padded row r and block
  * b = column / 128 are stored inside the workspace in the layout the FC2
  * tensor cores read; this copies them out as a plain u8 [rows, I/128] array
- * (device pointer `dst`), enqueued on `stream`.                              */
+ * (device pointer `dst`), enqueued on `stream`.  MOE_ERR_UNSUPPORTED for
+ * MOE_W_BF16 plans (no scales).                                              */
 moe_status moe_copy_act_scales(moe_plan_t plan, const void *workspace,
                                uint8_t *dst, moe_stream_t stream);
 
@@ -258,8 +267,8 @@ moe_status moe_copy_act_scales(moe_plan_t plan, const void *workspace,
  * moe_forward, read by 2-D TMA tiles.  MOE_WEIGHTS_TILED: W1/W2 are the output
  * of moe_prepack_weights() -- the same bytes rearranged into 128 x 128-byte
  * tiles that the tensor cores consume directly, streamed by linear bulk copies
- * (faster; FP8 weights only, MOE_ERR_UNSUPPORTED for MXFP4).  Weight scales
- * keep their layout in both cases.                                          */
+ * (faster; FP8 and BF16 weights, MOE_ERR_UNSUPPORTED for MXFP4).  Weight
+ * scales keep their layout in both cases.                                   */
 typedef enum { MOE_WEIGHTS_ROW_MAJOR = 0, MOE_WEIGHTS_TILED = 1 } moe_weight_layout;
 moe_status moe_plan_set_weight_layout(moe_plan_t plan, int layout);
 
@@ -278,19 +287,21 @@ moe_status moe_plan_set_cta_pairs(moe_plan_t plan, int mode);
  * current settings, 0 if not (or plan is NULL).                             */
 int moe_plan_cta_pairs_active(moe_plan_t plan);
 
-/* Rearrange row-major FP8 weights w1 [E,2I,H] and w2 [E,H,I] (device) into
- * the tiled layout (w1_tiled, w2_tiled: device buffers of the same sizes,
- * 16-byte aligned; must not overlap the inputs).  Tile (b, kb) -- rows
- * 128b..128b+127 of the [E*2I, H] (or [E*H, I]) matrix, bytes 128kb..128kb+127
- * of each row -- is 16384 bytes at offset (b * K/128 + kb) * 16384, and byte c
- * of tile row r lies at r*128 + ((c/16) XOR (r%8))*16 + c%16.  Done once per
- * weight set (e.g. at model load), enqueued on `stream`.                    */
+/* Rearrange row-major FP8 or BF16 weights w1 [E,2I,H] and w2 [E,H,I] (device)
+ * into the tiled layout (w1_tiled, w2_tiled: device buffers of the same sizes,
+ * 16-byte aligned; must not overlap the inputs).  With KB = the bytes of one
+ * row (K for FP8, 2K for BF16), tile (b, kb) -- rows 128b..128b+127 of the
+ * [E*2I, H] (or [E*H, I]) matrix, bytes 128kb..128kb+127 of each row -- is
+ * 16384 bytes at offset (b * KB/128 + kb) * 16384, and byte c of tile row r
+ * lies at r*128 + ((c/16) XOR (r%8))*16 + c%16.  Done once per weight set
+ * (e.g. at model load), enqueued on `stream`.                               */
 moe_status moe_prepack_weights(moe_plan_t plan, const void *w1, const void *w2,
                                void *w1_tiled, void *w2_tiled, moe_stream_t stream);
 
 /* Copy the FC1 activation codes out of the workspace as a row-major u8
- * [rows, I] array (device pointer `dst`, 16-byte aligned), enqueued on
- * `stream`; inside the workspace they are kept in the tiled layout.        */
+ * [rows, I] array (MOE_W_BF16: bf16 [rows, I]; device pointer `dst`, 16-byte
+ * aligned), enqueued on `stream`; inside the workspace they are kept in the
+ * tiled layout.                                                             */
 moe_status moe_copy_act(moe_plan_t plan, const void *workspace, uint8_t *dst,
                         moe_stream_t stream);
 

@@ -19,7 +19,7 @@ MOE_OK = 0
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                 3: "MOE_ERR_ALIGNMENT", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_TIMEOUT",
                 6: "MOE_ERR_BAD_ROUTING"}
-W_DTYPES = {"e4m3": 0, "e2m1": 1}
+W_DTYPES = {"e4m3": 0, "e2m1": 1, "bf16": 2}
 ACT_KINDS = {"swiglu": 0, "swiglu_oai": 1}
 
 
@@ -293,7 +293,7 @@ class MoELayer:
         return out
 
     def prepack(self, w1, w2):
-        """Tiled copies of row-major FP8 weights for a plan with tiled_weights."""
+        """Tiled copies of row-major FP8 or BF16 weights for a plan with tiled_weights."""
         import torch
         w1t, w2t = torch.empty_like(w1), torch.empty_like(w2)
         moe_prepack_weights(self.plan, w1, w2, w1t, w2t)

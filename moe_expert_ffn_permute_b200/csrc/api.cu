@@ -32,10 +32,13 @@ void compute_layout(moe_plan_s* p) {
   L.perm = take(S * 4);
   L.inv = take(S * 4);
   L.row_token = take(rows * 4);
-  L.xg = take(rows * p->H);
-  L.xg_sf = take(rows / kTileM * (p->H / 128) * 512);
-  L.act = take(rows * p->I);
-  L.act_sf = take(rows / kTileM * (p->I / 128) * 512);
+  // BF16 plans keep 2-byte activations and no scale chunks.
+  const bool bf16 = p->w_dtype == MOE_W_BF16;
+  const size_t elem = bf16 ? 2 : 1;
+  L.xg = take(rows * p->H * elem);
+  L.xg_sf = take(bf16 ? 0 : rows / kTileM * (p->H / 128) * 512);
+  L.act = take(rows * p->I * elem);
+  L.act_sf = take(bf16 ? 0 : rows / kTileM * (p->I / 128) * 512);
   L.act_f32 = take(p->debug_act_f32 ? rows * p->I * 4 : 0);
   L.y = take(S * p->H * 2);
   // One 1 KB record per (expert, n-tile, k-block) of each GEMM: the two 128-row
@@ -43,8 +46,8 @@ void compute_layout(moe_plan_s* p) {
   const bool fp8 = p->w_dtype == MOE_W_E4M3_UE8M0_128x128;
   L.pair_sf1 = take(fp8 ? E * (p->I / 128) * (p->H / 128) * 1024 : 0);
   L.pair_sf2 = take(fp8 ? E * (p->H / 256) * (p->I / 128) * 1024 : 0);
-  L.in_x = take(static_cast<size_t>(p->T) * p->H);
-  L.in_xs = take(static_cast<size_t>(p->T) * (p->H / 128));
+  L.in_x = take(static_cast<size_t>(p->T) * p->H * elem);
+  L.in_xs = take(bf16 ? 0 : static_cast<size_t>(p->T) * (p->H / 128));
   L.in_idx = take(S * 4);
   L.in_w = take(S * 4);
   L.out_stage = take(static_cast<size_t>(p->T) * p->H * 2);
@@ -77,8 +80,14 @@ static moe_status check_ws(moe_plan_t plan, const void* workspace) {
   return MOE_OK;
 }
 
+// x_scales is required except for BF16 plans (BF16 activations carry no scales).
+static bool x_scales_ok(moe_plan_t plan, const uint8_t* x_scales) {
+  return x_scales != nullptr || plan->w_dtype == MOE_W_BF16;
+}
+
 static moe_status check_weights(moe_plan_t plan, const void* w, const uint8_t* ws) {
-  if (w == nullptr || ws == nullptr) return MOE_ERR_INVALID_ARG;
+  if (w == nullptr) return MOE_ERR_INVALID_ARG;
+  if (ws == nullptr && plan->w_dtype != MOE_W_BF16) return MOE_ERR_INVALID_ARG;
   const size_t wa = plan->w_dtype == MOE_W_E2M1_UE8M0_1x32 ? 32 : 16;
   if (!aligned(w, wa)) return MOE_ERR_ALIGNMENT;
   if (plan->w_dtype == MOE_W_E2M1_UE8M0_1x32 && !aligned(ws, 4)) return MOE_ERR_ALIGNMENT;
@@ -96,7 +105,8 @@ moe_status moe_plan(int T, int H, int I, int E, int k, moe_dtypes dtypes, moe_ac
   if (H % 128 != 0 || I % 128 != 0) return MOE_ERR_UNSUPPORTED;
   if (H % 256 != 0) return MOE_ERR_UNSUPPORTED;   // FC2 tiles are 256 columns wide
   if (static_cast<long long>(T) * k >= (1ll << 31)) return MOE_ERR_INVALID_ARG;
-  if (dtypes.w_dtype != MOE_W_E4M3_UE8M0_128x128 && dtypes.w_dtype != MOE_W_E2M1_UE8M0_1x32)
+  if (dtypes.w_dtype != MOE_W_E4M3_UE8M0_128x128 && dtypes.w_dtype != MOE_W_E2M1_UE8M0_1x32 &&
+      dtypes.w_dtype != MOE_W_BF16)
     return MOE_ERR_INVALID_ARG;
   if (act.kind != MOE_ACT_SWIGLU && act.kind != MOE_ACT_SWIGLU_OAI) return MOE_ERR_INVALID_ARG;
   if (act.kind == MOE_ACT_SWIGLU_OAI) {
@@ -137,7 +147,7 @@ size_t moe_workspace_bytes(moe_plan_t plan) { return plan ? plan->ws.total : 0; 
 moe_status moe_plan_set_weight_layout(moe_plan_t plan, int layout) {
   if (plan == nullptr) return MOE_ERR_INVALID_ARG;
   if (layout != MOE_WEIGHTS_ROW_MAJOR && layout != MOE_WEIGHTS_TILED) return MOE_ERR_INVALID_ARG;
-  if (layout == MOE_WEIGHTS_TILED && plan->w_dtype != MOE_W_E4M3_UE8M0_128x128)
+  if (layout == MOE_WEIGHTS_TILED && plan->w_dtype == MOE_W_E2M1_UE8M0_1x32)
     return MOE_ERR_UNSUPPORTED;
   plan->w_tiled = layout == MOE_WEIGHTS_TILED ? 1 : 0;
   return MOE_OK;
@@ -156,16 +166,17 @@ moe_status moe_prepack_weights(moe_plan_t plan, const void* w1, const void* w2, 
   if (plan == nullptr || w1 == nullptr || w2 == nullptr || w1_tiled == nullptr ||
       w2_tiled == nullptr)
     return MOE_ERR_INVALID_ARG;
-  if (plan->w_dtype != MOE_W_E4M3_UE8M0_128x128) return MOE_ERR_UNSUPPORTED;
+  if (plan->w_dtype == MOE_W_E2M1_UE8M0_1x32) return MOE_ERR_UNSUPPORTED;
   if (!aligned(w1, 16) || !aligned(w2, 16) || !aligned(w1_tiled, 16) || !aligned(w2_tiled, 16))
     return MOE_ERR_ALIGNMENT;
   auto st = reinterpret_cast<cudaStream_t>(stream);
   const long long E = plan->E;
-  if (moe::launch_prepack(static_cast<const uint8_t*>(w1), E * 2 * plan->I, plan->H,
+  const int elem = plan->w_dtype == MOE_W_BF16 ? 2 : 1;   // bytes per weight
+  if (moe::launch_prepack(static_cast<const uint8_t*>(w1), E * 2 * plan->I, plan->H * elem,
                           static_cast<uint8_t*>(w1_tiled), st) != cudaSuccess)
     return MOE_ERR_CUDA;
-  return cuda_status(moe::launch_prepack(static_cast<const uint8_t*>(w2), E * plan->H, plan->I,
-                                         static_cast<uint8_t*>(w2_tiled), st));
+  return cuda_status(moe::launch_prepack(static_cast<const uint8_t*>(w2), E * plan->H,
+                                         plan->I * elem, static_cast<uint8_t*>(w2_tiled), st));
 }
 
 moe_status moe_copy_act(moe_plan_t plan, const void* workspace, uint8_t* dst,
@@ -212,7 +223,7 @@ moe_status moe_gather(moe_plan_t plan, const void* x, const uint8_t* x_scales, v
                       moe_stream_t stream) {
   moe_status s = check_ws(plan, workspace);
   if (s != MOE_OK) return s;
-  if (x == nullptr || x_scales == nullptr) return MOE_ERR_INVALID_ARG;
+  if (x == nullptr || !x_scales_ok(plan, x_scales)) return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16)) return MOE_ERR_ALIGNMENT;
   return cuda_status(moe::launch_gather(plan, static_cast<const uint8_t*>(x), x_scales,
                                         static_cast<uint8_t*>(workspace),
@@ -223,7 +234,8 @@ moe_status moe_route_gather(moe_plan_t plan, const int32_t* topk_idx, const void
                             const uint8_t* x_scales, void* workspace, moe_stream_t stream) {
   moe_status s = check_ws(plan, workspace);
   if (s != MOE_OK) return s;
-  if (topk_idx == nullptr || x == nullptr || x_scales == nullptr) return MOE_ERR_INVALID_ARG;
+  if (topk_idx == nullptr || x == nullptr || !x_scales_ok(plan, x_scales))
+    return MOE_ERR_INVALID_ARG;
   if (!aligned(topk_idx, 4) || !aligned(x, 16)) return MOE_ERR_ALIGNMENT;
   if (plan->S > moe::kFusedMaxSlots) {
     if ((s = moe_route(plan, topk_idx, workspace, stream)) != MOE_OK) return s;
@@ -282,7 +294,7 @@ moe_status moe_forward(moe_plan_t plan, const void* x, const uint8_t* x_scales,
   // Validate everything before the first launch.
   moe_status s = check_ws(plan, workspace);
   if (s != MOE_OK) return s;
-  if (x == nullptr || x_scales == nullptr || topk_idx == nullptr || topk_w == nullptr ||
+  if (x == nullptr || !x_scales_ok(plan, x_scales) || topk_idx == nullptr || topk_w == nullptr ||
       out == nullptr)
     return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(topk_idx, 4) || !aligned(topk_w, 4) || !aligned(out, 16))
@@ -304,7 +316,7 @@ moe_status moe_forward_hostio(moe_plan_t plan, const void* x_host, const uint8_t
                               moe_stream_t stream) {
   moe_status s = check_ws(plan, workspace);
   if (s != MOE_OK) return s;
-  if (x_host == nullptr || x_scales_host == nullptr || topk_idx_host == nullptr ||
+  if (x_host == nullptr || !x_scales_ok(plan, x_scales_host) || topk_idx_host == nullptr ||
       topk_w_host == nullptr || out_host == nullptr)
     return MOE_ERR_INVALID_ARG;
   if ((s = check_weights(plan, w1, w1_scales)) != MOE_OK) return s;
@@ -313,16 +325,19 @@ moe_status moe_forward_hostio(moe_plan_t plan, const void* x_host, const uint8_t
   auto st = reinterpret_cast<cudaStream_t>(stream);
   const auto& L = plan->ws;
   const size_t T = plan->T, H = plan->H, S = static_cast<size_t>(plan->S);
-  if (cudaMemcpyAsync(ws + L.in_x, x_host, T * H, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(ws + L.in_xs, x_scales_host, T * (H / 128), cudaMemcpyHostToDevice, st) !=
+  const bool bf16 = plan->w_dtype == MOE_W_BF16;
+  if (cudaMemcpyAsync(ws + L.in_x, x_host, T * H * (bf16 ? 2 : 1), cudaMemcpyHostToDevice, st) !=
           cudaSuccess ||
+      (!bf16 && cudaMemcpyAsync(ws + L.in_xs, x_scales_host, T * (H / 128),
+                                cudaMemcpyHostToDevice, st) != cudaSuccess) ||
       cudaMemcpyAsync(ws + L.in_idx, topk_idx_host, S * 4, cudaMemcpyHostToDevice, st) !=
           cudaSuccess ||
       cudaMemcpyAsync(ws + L.in_w, topk_w_host, S * 4, cudaMemcpyHostToDevice, st) !=
           cudaSuccess)
     return MOE_ERR_CUDA;
   uint8_t* out_dev = ws + L.out_stage;
-  s = moe_forward(plan, ws + L.in_x, ws + L.in_xs, reinterpret_cast<const int32_t*>(ws + L.in_idx),
+  s = moe_forward(plan, ws + L.in_x, bf16 ? nullptr : ws + L.in_xs,
+                  reinterpret_cast<const int32_t*>(ws + L.in_idx),
                   reinterpret_cast<const float*>(ws + L.in_w), w1, w1_scales, w2, w2_scales,
                   out_dev, workspace, stream);
   if (s != MOE_OK) return s;
@@ -355,6 +370,7 @@ moe_status moe_copy_act_scales(moe_plan_t plan, const void* workspace, uint8_t* 
   moe_status s = check_ws(plan, workspace);
   if (s != MOE_OK) return s;
   if (dst == nullptr) return MOE_ERR_INVALID_ARG;
+  if (plan->w_dtype == MOE_W_BF16) return MOE_ERR_UNSUPPORTED;
   return cuda_status(moe::launch_unpack_act_scales(plan, static_cast<const uint8_t*>(workspace),
                                                    dst, reinterpret_cast<cudaStream_t>(stream)));
 }

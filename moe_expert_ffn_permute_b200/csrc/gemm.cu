@@ -172,12 +172,19 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   return v;
 }
 
-template <bool kFp4>
+// Weight formats: E4M3 with 128x128 UE8M0 scales, E2M1 with 1x32 UE8M0 scales
+// (both with E4M3 activations, block-scaled MMA), or BF16 (BF16 activations,
+// kind::f16 MMA, no scales).
+enum : int { kWFp8 = 0, kWFp4 = 1, kWBf16 = 2 };
+
+template <int kW>
 __global__ void __launch_bounds__(kThreads, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a1,
                     const __grid_constant__ CUtensorMap tmap_b1,
                     const __grid_constant__ CUtensorMap tmap_a2,
                     const __grid_constant__ CUtensorMap tmap_b2, const Params p) {
+  constexpr bool kFp4 = kW == kWFp4;
+  constexpr bool kBf16 = kW == kWBf16;
   extern __shared__ uint8_t smem_raw[];
   griddep_launch_dependents();
   Smem& sm = *reinterpret_cast<Smem*>(
@@ -188,7 +195,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       // operand producer's expect-tx arrive + one arrive per scale-factor lane
-      mbar_init(&sm.full[s], 33);
+      // (BF16: the expect-tx arrive alone)
+      mbar_init(&sm.full[s], kBf16 ? 1 : 33);
       mbar_init(&sm.empty[s], 1);
     }
     mbar_init(&sm.tmem_full, 1);
@@ -267,6 +275,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool operands = warp == 0;
     int slot = 0, stage = 0;
     uint32_t sphase = 0, phase = 0;
+    if (kBf16 && !operands) {
+      // No scale factors: the scale warp only releases its task slots.
+      Task t;
+      while (get_task(sm, slot, sphase, t, p.err)) {
+        if (t.e < 0) break;
+      }
+    } else {
     // A tiles are re-read by every n-tile of their m-tile: keep them in L2.
     // Weight tiles are re-read only when the expert has several m-tiles;
     // otherwise they stream through L2 once and go first.
@@ -391,6 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    }   // BF16 scale warp / producers
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     // One lane issues everything: a warp-wide wait + fence + __syncwarp per
@@ -410,23 +426,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             aborted = true;
             break;
           }
-          // MXFP4 weight scales land by cp.async (generic proxy): order them
-          // before the tensor core's (async proxy) reads of shared memory.
-          if (kFp4) fence_proxy_async_smem();
-          const uint32_t sfa = tmem + kSfaCol + sfset * kSfSetStride;
-          const uint32_t sfb = tmem + kSfbCol + sfset * kSfSetStride;
-          tmem_cp_32x128b_warpx4(sfa, sf_desc(smem_u32(sm.sfa[stage])));
-          tmem_cp_32x128b_warpx4(sfb, sf_desc(smem_u32(sm.sfb[stage])));
-          tmem_cp_32x128b_warpx4(sfb + 4, sf_desc(smem_u32(sm.sfb[stage] + 512)));
           const uint32_t a_base = smem_u32(sm.a[stage]);
           const uint32_t b_base = smem_u32(sm.b[stage]);
+          if (kBf16) {
+            // 128 bytes of K = 64 BF16 values: four MMAs of K = 16 (32 bytes each).
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint32_t idesc = mxf8f6f4_idesc(kFp4 ? 5u : 0u, BN, ks);
-            mma_mxf8f6f4(tmem + kAccCol, umma_desc_sw128(a_base + ks * 32),
-                         umma_desc_sw128(b_base + ks * 32), idesc,
-                         sfa | (static_cast<uint32_t>(ks) << 30),
-                         sfb | (static_cast<uint32_t>(ks) << 30), (kb > 0 || ks > 0) ? 1u : 0u);
+            for (int ks = 0; ks < 4; ++ks)
+              mma_bf16(tmem + kAccCol, umma_desc_sw128(a_base + ks * 32),
+                       umma_desc_sw128(b_base + ks * 32), bf16_idesc(BN),
+                       (kb > 0 || ks > 0) ? 1u : 0u);
+          } else {
+            // MXFP4 weight scales land by cp.async (generic proxy): order them
+            // before the tensor core's (async proxy) reads of shared memory.
+            if (kFp4) fence_proxy_async_smem();
+            const uint32_t sfa = tmem + kSfaCol + sfset * kSfSetStride;
+            const uint32_t sfb = tmem + kSfbCol + sfset * kSfSetStride;
+            tmem_cp_32x128b_warpx4(sfa, sf_desc(smem_u32(sm.sfa[stage])));
+            tmem_cp_32x128b_warpx4(sfb, sf_desc(smem_u32(sm.sfb[stage])));
+            tmem_cp_32x128b_warpx4(sfb + 4, sf_desc(smem_u32(sm.sfb[stage] + 512)));
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint32_t idesc = mxf8f6f4_idesc(kFp4 ? 5u : 0u, BN, ks);
+              mma_mxf8f6f4(tmem + kAccCol, umma_desc_sw128(a_base + ks * 32),
+                           umma_desc_sw128(b_base + ks * 32), idesc,
+                           sfa | (static_cast<uint32_t>(ks) << 30),
+                           sfb | (static_cast<uint32_t>(ks) << 30), (kb > 0 || ks > 0) ? 1u : 0u);
+            }
           }
           tc_commit(&sm.empty[stage]);
           sfset ^= 1u;
@@ -487,6 +512,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           g[i] = __float_as_uint(a);
           amax = fmaxf(amax, fabsf(a));
+        }
+        if (kBf16) {
+          // BF16 activation (round to nearest even): this warp's 64 columns are
+          // exactly one 128-byte row of activation tile (m-tile, 2 * nt + half).
+          uint8_t* tile = p.act + (static_cast<size_t>(t.mt) * (p.I / 64) + 2 * t.nt + half) *
+                                      kTileBytes;
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const int i0 = v * 8;
+            *reinterpret_cast<uint4*>(tile + swz128(row, v)) = make_uint4(
+                pack_bf16x2(__uint_as_float(g[i0]), __uint_as_float(g[i0 + 1])),
+                pack_bf16x2(__uint_as_float(g[i0 + 2]), __uint_as_float(g[i0 + 3])),
+                pack_bf16x2(__uint_as_float(g[i0 + 4]), __uint_as_float(g[i0 + 5])),
+                pack_bf16x2(__uint_as_float(g[i0 + 6]), __uint_as_float(g[i0 + 7])));
+          }
+          if (p.act_f32 != nullptr) {
+            const size_t prow = static_cast<size_t>(t.mt) * BM + row;
+            float4* fd =
+                reinterpret_cast<float4*>(p.act_f32 + prow * p.I + t.nt * 128 + half * 64);
+#pragma unroll
+            for (int v = 0; v < 16; ++v)
+              fd[v] = make_float4(__uint_as_float(g[4 * v]), __uint_as_float(g[4 * v + 1]),
+                                  __uint_as_float(g[4 * v + 2]), __uint_as_float(g[4 * v + 3]));
+          }
+          if (p.phases & 2) {
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) atomicAdd(p.fc1_done + t.mt, 1u);
+          }
+          acc_phase ^= 1u;
+          continue;
         }
         // Combine the two halves' amax of this row (the other warp of the pair).
         sm.amax[tile_par][half][row] = amax;
@@ -622,7 +678,7 @@ int num_sms() {
   return n;
 }
 
-template <bool kFp4>
+template <int kW>
 cudaError_t launch_gemm(const moe_plan_s* pl, int phases, bool dynamic, const void* w1,
                         const uint8_t* w1s, const void* w2, const uint8_t* w2s, uint8_t* ws,
                         cudaStream_t st) {
@@ -637,22 +693,30 @@ cudaError_t launch_gemm(const moe_plan_s* pl, int phases, bool dynamic, const vo
   p.dynamic = dynamic ? 1 : 0;
   long long max_tiles = 0;
   const bool tiled = pl->w_tiled != 0;
+  constexpr bool kFp4 = kW == kWFp4;
+  constexpr bool kBf16 = kW == kWBf16;
+  // Bytes of one weight row of K elements, and the map's inner extent: FP4 maps
+  // count 4-bit elements (the copy widens them), the others count bytes.
+  auto row_bytes = [](int K) { return kFp4 ? K / 2 : (kBf16 ? 2 * K : K); };
+  auto inner = [](int K) { return kBf16 ? 2 * K : K; };
+  // K-blocks of 128 bytes in shared memory (128 elements for FP8/FP4, 64 BF16).
+  auto k_blocks = [](int K) { return kBf16 ? K / 64 : K / 128; };
   if (phases & 1) {
     const int K = pl->H;
-    if (!tiled && !make_map(&maps[1], w1, K, static_cast<uint64_t>(pl->E) * 2 * pl->I,
-                            kFp4 ? K / 2 : K, 128, kFp4))
+    if (!tiled && !make_map(&maps[1], w1, inner(K), static_cast<uint64_t>(pl->E) * 2 * pl->I,
+                            row_bytes(K), 128, kFp4))
       return cudaErrorInvalidValue;
-    p.ph[0] = Phase{pl->I / 128, K / 128, 2 * pl->I, ws + L.xg_sf, w1s, ws + L.xg,
-                    tiled ? static_cast<const uint8_t*>(w1) : nullptr};
+    p.ph[0] = Phase{pl->I / 128, k_blocks(K), 2 * pl->I, kBf16 ? nullptr : ws + L.xg_sf, w1s,
+                    ws + L.xg, tiled ? static_cast<const uint8_t*>(w1) : nullptr};
     max_tiles += (pl->rows_cap / BM) * p.ph[0].n_tiles;
   }
   if (phases & 2) {
     const int K = pl->I;
-    if (!tiled && !make_map(&maps[3], w2, K, static_cast<uint64_t>(pl->E) * pl->H,
-                            kFp4 ? K / 2 : K, 256, kFp4))
+    if (!tiled && !make_map(&maps[3], w2, inner(K), static_cast<uint64_t>(pl->E) * pl->H,
+                            row_bytes(K), 256, kFp4))
       return cudaErrorInvalidValue;
-    p.ph[1] = Phase{pl->H / 256, K / 128, pl->H, ws + L.act_sf, w2s, ws + L.act,
-                    tiled ? static_cast<const uint8_t*>(w2) : nullptr};
+    p.ph[1] = Phase{pl->H / 256, k_blocks(K), pl->H, kBf16 ? nullptr : ws + L.act_sf, w2s,
+                    ws + L.act, tiled ? static_cast<const uint8_t*>(w2) : nullptr};
     max_tiles += (pl->rows_cap / BM) * p.ph[1].n_tiles;
   }
   p.tile_off = reinterpret_cast<const int32_t*>(ws + L.tile_off);
@@ -671,7 +735,7 @@ cudaError_t launch_gemm(const moe_plan_s* pl, int phases, bool dynamic, const vo
   p.y = reinterpret_cast<uint16_t*>(ws + L.y);
   p.err = reinterpret_cast<uint32_t*>(ws + L.err);
   const size_t smem = sizeof(Smem) + 1024;
-  auto kern = moe_gemm_kernel<kFp4>;
+  auto kern = moe_gemm_kernel<kW>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e =
@@ -688,25 +752,34 @@ cudaError_t launch_gemm(const moe_plan_s* pl, int phases, bool dynamic, const vo
 
 size_t gemm_smem_bytes() { return sizeof(Smem) + 1024; }
 
+// phases: 1 FC1 only, 2 FC2 only, 3 both in one launch (dynamic scheduling).
+static cudaError_t launch_phases(const moe_plan_s* p, int phases, const void* w1,
+                                 const uint8_t* w1s, const void* w2, const uint8_t* w2s,
+                                 uint8_t* ws, cudaStream_t st) {
+  const bool dyn = phases == 3;
+  switch (p->w_dtype) {
+    case MOE_W_E2M1_UE8M0_1x32:
+      return launch_gemm<kWFp4>(p, phases, dyn, w1, w1s, w2, w2s, ws, st);
+    case MOE_W_BF16:
+      return launch_gemm<kWBf16>(p, phases, dyn, w1, w1s, w2, w2s, ws, st);
+    default:
+      return launch_gemm<kWFp8>(p, phases, dyn, w1, w1s, w2, w2s, ws, st);
+  }
+}
+
 cudaError_t launch_fc1(const moe_plan_s* p, const void* w1, const uint8_t* w1s, uint8_t* ws,
                        cudaStream_t st) {
-  if (p->w_dtype == MOE_W_E2M1_UE8M0_1x32)
-    return launch_gemm<true>(p, 1, false, w1, w1s, nullptr, nullptr, ws, st);
-  return launch_gemm<false>(p, 1, false, w1, w1s, nullptr, nullptr, ws, st);
+  return launch_phases(p, 1, w1, w1s, nullptr, nullptr, ws, st);
 }
 
 cudaError_t launch_fc2(const moe_plan_s* p, const void* w2, const uint8_t* w2s, uint8_t* ws,
                        cudaStream_t st) {
-  if (p->w_dtype == MOE_W_E2M1_UE8M0_1x32)
-    return launch_gemm<true>(p, 2, false, nullptr, nullptr, w2, w2s, ws, st);
-  return launch_gemm<false>(p, 2, false, nullptr, nullptr, w2, w2s, ws, st);
+  return launch_phases(p, 2, nullptr, nullptr, w2, w2s, ws, st);
 }
 
 cudaError_t launch_fc12(const moe_plan_s* p, const void* w1, const uint8_t* w1s, const void* w2,
                         const uint8_t* w2s, uint8_t* ws, cudaStream_t st) {
-  if (p->w_dtype == MOE_W_E2M1_UE8M0_1x32)
-    return launch_gemm<true>(p, 3, true, w1, w1s, w2, w2s, ws, st);
-  return launch_gemm<false>(p, 3, true, w1, w1s, w2, w2s, ws, st);
+  return launch_phases(p, 3, w1, w1s, w2, w2s, ws, st);
 }
 
 }  // namespace moe

@@ -61,8 +61,9 @@ cudaError_t launch_prepack(const uint8_t* src, long long rows, int K, uint8_t* d
 
 cudaError_t launch_unpack_act(const moe_plan_s* p, const uint8_t* ws, uint8_t* dst,
                               cudaStream_t st) {
-  const long long n = p->rows_cap * (p->I / 16);
-  unpack_kernel<<<blocks_for(n), 256, 0, st>>>(ws + p->ws.act, p->rows_cap, p->I,
+  const int row_bytes = p->I * (p->w_dtype == MOE_W_BF16 ? 2 : 1);
+  const long long n = p->rows_cap * (row_bytes / 16);
+  unpack_kernel<<<blocks_for(n), 256, 0, st>>>(ws + p->ws.act, p->rows_cap, row_bytes,
                                                reinterpret_cast<uint4*>(dst));
   return cudaGetLastError();
 }

@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
 constexpr int kGatherWarps = 8;
 
 __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(
-    const uint8_t* __restrict__ x, const uint8_t* __restrict__ xs, int H, int E,
+    const uint8_t* __restrict__ x, const uint8_t* __restrict__ xs, int row_bytes, int E,
     const int32_t* __restrict__ pad_off, const int32_t* __restrict__ row_token,
     uint8_t* __restrict__ xg, uint8_t* __restrict__ xg_sf) {
   griddep_launch_dependents();
@@ -212,14 +212,16 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(
   if (t < 0) return;   // padding row
   const int tile = static_cast<int>(P / kTileM);
   const int r = static_cast<int>(P % kTileM);
-  const int vec = H / 16;
-  const int kb_n = H / 128;
-  const uint4* __restrict__ src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
+  const int vec = row_bytes / 16;
+  const int kb_n = row_bytes / 128;
+  const uint4* __restrict__ src =
+      reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * row_bytes);
   // Destination: pre-swizzled 128 x 128-byte tiles [tile][k-block][16 KB].
   uint8_t* __restrict__ dst = xg + static_cast<size_t>(tile) * kb_n * kTileBytes;
   for (int c = lane; c < vec; c += 32)
     *reinterpret_cast<uint4*>(dst + static_cast<size_t>(c >> 3) * kTileBytes + swz128(r, c & 7)) =
         __ldg(&src[c]);
+  if (xs == nullptr) return;   // BF16 activations: no scales
   uint8_t* chunk = xg_sf + static_cast<size_t>(tile) * kb_n * 512 + (r & 31) * 16 + (r >> 5) * 4;
   for (int kb = lane; kb < kb_n; kb += 32) {
     const uint32_t b = __ldg(&xs[static_cast<size_t>(t) * kb_n + kb]);
@@ -240,7 +242,7 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(
 // launches.
 __global__ void __launch_bounds__(kRouteThreads) route_gather_kernel(
     const int32_t* __restrict__ idx, int S, int E, int k, const uint8_t* __restrict__ x,
-    const uint8_t* __restrict__ xs, int H, int32_t* __restrict__ counts,
+    const uint8_t* __restrict__ xs, int row_bytes, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ tile_off, int32_t* __restrict__ pad_off,
     int32_t* __restrict__ pair_off, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
     uint32_t* err, uint32_t* __restrict__ sched, int sched_words,
@@ -355,8 +357,9 @@ __global__ void __launch_bounds__(kRouteThreads) route_gather_kernel(
   }
   // Gather: one warp per routed row; all loads of a row are issued before its
   // stores.
-  const int kb_n = H / 128;
-  const int vec = H / 16;
+  const int kb_n = row_bytes / 128;   // 128-byte k-blocks per row (scale blocks when FP8)
+  const int vec = row_bytes / 16;
+  const bool scales = xs != nullptr;  // BF16 activations carry none
   for (int q = blockIdx.x * kWarps + warp; q < routed; q += gridDim.x * kWarps) {
     int lo = 0, hi = E - 1;   // expert of sorted position q: largest e with scan[e] <= q
     while (lo < hi) {
@@ -368,10 +371,11 @@ __global__ void __launch_bounds__(kRouteThreads) route_gather_kernel(
     const int t = sorted[q] / k;
     const int tile = static_cast<int>(P / kTileM);
     const int r = static_cast<int>(P % kTileM);
-    const uint4* __restrict__ src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
+    const uint4* __restrict__ src =
+        reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * row_bytes);
     uint8_t* __restrict__ dst = xg + static_cast<size_t>(tile) * kb_n * kTileBytes;
-    // Rows of up to 8192 bytes (H <= 8192) move in one batch of loads; the
-    // scale bytes (up to 64 per row) are loaded with them.
+    // Rows of up to 8192 bytes move in one batch of loads; the scale bytes (up
+    // to 64 per row) are loaded with them.
     constexpr int kBatch = 16;
     uint8_t* chunk = xg_sf + static_cast<size_t>(tile) * kb_n * 512 + (r & 31) * 16 + (r >> 5) * 4;
     for (int c0 = lane; c0 < vec; c0 += 32 * kBatch) {
@@ -382,7 +386,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_gather_kernel(
         if (c < vec) xv[u] = __ldg(&src[c]);
       }
       uint32_t sb[2] = {0u, 0u};
-      if (c0 == lane) {
+      if (scales && c0 == lane) {
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int kb = lane + 32 * u;
@@ -396,7 +400,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_gather_kernel(
           *reinterpret_cast<uint4*>(dst + static_cast<size_t>(c >> 3) * kTileBytes +
                                     swz128(r, c & 7)) = xv[u];
       }
-      if (c0 == lane) {
+      if (scales && c0 == lane) {
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int kb = lane + 32 * u;
@@ -406,7 +410,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_gather_kernel(
         }
       }
     }
-    for (int kb = lane + 64; kb < kb_n; kb += 32) {   // H > 8192
+    for (int kb = lane + 64; scales && kb < kb_n; kb += 32) {   // rows > 8192 bytes
       const uint32_t b = __ldg(&xs[static_cast<size_t>(t) * kb_n + kb]);
       *reinterpret_cast<uint32_t*>(chunk + static_cast<size_t>(kb) * 512) = b * 0x01010101u;
     }
@@ -454,8 +458,9 @@ cudaError_t launch_gather(const moe_plan_s* p, const uint8_t* x, const uint8_t* 
                           cudaStream_t st) {
   const auto& L = p->ws;
   const int blocks = static_cast<int>(p->rows_cap / kGatherWarps);
-  return launch_pdl(gather_kernel, dim3(blocks), dim3(kGatherWarps * 32), 0, st, x, xs, p->H,
-                    p->E, reinterpret_cast<const int32_t*>(ws + L.pad_off),
+  const bool bf16 = p->w_dtype == MOE_W_BF16;   // 2-byte activations, no scales
+  return launch_pdl(gather_kernel, dim3(blocks), dim3(kGatherWarps * 32), 0, st, x,
+                    bf16 ? nullptr : xs, p->H * (bf16 ? 2 : 1), p->E, reinterpret_cast<const int32_t*>(ws + L.pad_off),
                     reinterpret_cast<const int32_t*>(ws + L.row_token), ws + L.xg, ws + L.xg_sf);
 }
 
@@ -470,11 +475,13 @@ cudaError_t launch_route_gather(const moe_plan_s* p, const int32_t* topk_idx, co
     if (cudaGetDevice(&dev) == cudaSuccess)
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   }
+  const bool bf16 = p->w_dtype == MOE_W_BF16;   // 2-byte activations, no scales
   const int want = (S + kRouteThreads / 32 - 1) / (kRouteThreads / 32);
   const int blocks = std::max(1, std::min(want, 2 * sms));
   return launch_pdl(
       route_gather_kernel, dim3(blocks), dim3(kRouteThreads), 2 * S * sizeof(int32_t), st,
-      topk_idx, S, p->E, p->k, x, xs, p->H, reinterpret_cast<int32_t*>(ws + L.counts),
+      topk_idx, S, p->E, p->k, x, bf16 ? nullptr : xs, p->H * (bf16 ? 2 : 1),
+      reinterpret_cast<int32_t*>(ws + L.counts),
       reinterpret_cast<int32_t*>(ws + L.offsets), reinterpret_cast<int32_t*>(ws + L.tile_off),
       reinterpret_cast<int32_t*>(ws + L.pad_off), reinterpret_cast<int32_t*>(ws + L.pair_off),
       reinterpret_cast<int32_t*>(ws + L.perm), reinterpret_cast<int32_t*>(ws + L.inv),

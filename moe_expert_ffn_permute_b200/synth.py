@@ -35,7 +35,7 @@ class Workload:
     I: int
     E: int
     k: int
-    w_dtype: str = "e4m3"          # "e4m3" or "e2m1"
+    w_dtype: str = "e4m3"          # "e4m3", "e2m1" or "bf16" (then x is bf16 too)
     routing: str = "gaussian"      # "gaussian" or "zipf"
     act: str = "swiglu"            # "swiglu" or "swiglu_oai"
     alpha: float = 1.0
@@ -61,6 +61,8 @@ WORKLOADS = {
     "oai": Workload("oai", 2048, 3072, 1536, 64, 4, act="swiglu_oai",
                     alpha=1.702, up_bias=1.0, limit=7.0, cfg_id=3),
     "mxfp4": Workload("mxfp4", 128, 7168, 3072, 48, 6, w_dtype="e2m1", cfg_id=4),
+    # The BF16 variant at the decode layer's shape and routing.
+    "bf16": Workload("bf16", 128, 7168, 2048, 32, 8, w_dtype="bf16", routing="zipf", cfg_id=5),
 }
 MXFP4_TOKEN_SWEEP = (128, 512, 1024, 2048, 4096, 8192, 16384, 32768)
 
@@ -142,12 +144,14 @@ def make_weights(wl, device="cpu", seed=None):
             v = torch.randn(R, C, generator=gen, device=device, dtype=torch.float32) * 0.02
             if wl.w_dtype == "e4m3":
                 q, s = _quant_e4m3_blocks(v, 128, 128)
-            else:
+            elif wl.w_dtype == "e2m1":
                 q, s = _quant_e2m1_rows(v)
+            else:
+                q, s = v.to(torch.bfloat16), None
             codes.append(q)
             scales.append(s)
         out[name] = torch.stack(codes)
-        out[name + "_scales"] = torch.stack(scales)
+        out[name + "_scales"] = None if scales[0] is None else torch.stack(scales)
     return out
 
 
@@ -156,8 +160,11 @@ def make_activations(wl, device="cpu", seed=None):
     gen = torch.Generator(device=device)
     gen.manual_seed((1000 + wl.cfg_id) * 7919 + wl.T if seed is None else seed)
     x = torch.randn(wl.T, wl.H, generator=gen, device=device, dtype=torch.float32)
-    x = x.to(torch.bfloat16).to(torch.float32)
-    xq, xs = _quant_e4m3_blocks(x, 1, 128)
+    x = x.to(torch.bfloat16)
+    if wl.w_dtype == "bf16":
+        xq, xs = x, None
+    else:
+        xq, xs = _quant_e4m3_blocks(x.to(torch.float32), 1, 128)
     idx, w = _routing(wl, gen, device)
     return {"x": xq, "x_scales": xs, "topk_idx": idx, "topk_w": w}
 
@@ -169,4 +176,11 @@ def make_inputs(wl, device="cpu", seed=None):
 
 
 def to_numpy(d):
-    return {k: v.cpu().numpy() for k, v in d.items()}
+    """Tensors -> numpy (bf16 as its uint16 bit patterns; None stays None)."""
+    def conv(v):
+        if v is None:
+            return None
+        if v.dtype == torch.bfloat16:
+            return v.cpu().view(torch.int16).numpy().view("uint16")
+        return v.cpu().numpy()
+    return {k: conv(v) for k, v in d.items()}

@@ -60,13 +60,22 @@ def oracle_kw(wl):
     return dict(w_dtype=wl.w_dtype, alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit)
 
 
+def oracle_layer(wl, dn, keep=False):
+    """The oracle for the workload's weight format (numpy inputs)."""
+    if wl.w_dtype == "bf16":
+        return L.layer_bf16(dn["x"], dn["topk_idx"], dn["topk_w"], dn["w1"], dn["w2"],
+                            alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit, keep=keep)
+    return L.layer(*oracle_args(dn), **oracle_kw(wl), keep=keep)
+
+
 def oracle_tokens(wl, dn, tokens, keep=False):
     """Oracle output for a subset of tokens (rows of the full-layer output:
     every token's output depends only on its own inputs)."""
     sub = dict(dn)
     for key in ("x", "x_scales", "topk_idx", "topk_w"):
-        sub[key] = dn[key][tokens]
-    return L.layer(*oracle_args(sub), **oracle_kw(wl), keep=keep)
+        if dn[key] is not None:
+            sub[key] = dn[key][tokens]
+    return oracle_layer(wl, sub, keep=keep)
 
 
 def inputs(wl, device="cuda", seed=None):

@@ -138,3 +138,28 @@ def test_cta_pair_mode_selection_and_launch_count():
     assert not moe.moe_plan_cta_pairs_active(q)
     moe.moe_plan_destroy(q)
     assert not moe.moe_plan_cta_pairs_active(None)
+
+
+def test_bf16_plans_take_no_scales_and_tiled_weights():
+    g = 1 << 20                          # aligned fake addresses: never dereferenced
+    p = moe.moe_plan(64, 512, 256, 8, 2, w_dtype="bf16")
+    q = moe.moe_plan(64, 512, 256, 8, 2)
+    # Without scales a BF16 plan gets as far as the alignment check of x (no
+    # launch happens); an FP8 plan stops at the missing x_scales.
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_forward(p, g + 4, None, g, g, g, None, g, None, g, g, stream=0)
+    assert ei.value.status == 3
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_forward(q, g + 4, None, g, g, g, g, g, g, g, g, stream=0)
+    assert ei.value.status == 1
+    with pytest.raises(moe.MoEError) as ei:          # no activation scales to copy
+        moe.moe_copy_act_scales(p, g, g, stream=0)
+    assert ei.value.status == 2
+    moe.moe_plan_set_weight_layout(p, True)           # tiled BF16 weights are fine
+    with pytest.raises(moe.MoEError) as ei:          # the 2-SM kernel is FP8 only
+        moe.moe_plan_set_cta_pairs(p, 2)
+    assert ei.value.status == 2
+    # 2-byte activations: the workspace is larger than the FP8 plan's.
+    assert moe.moe_workspace_bytes(p) > moe.moe_workspace_bytes(q)
+    moe.moe_plan_destroy(p)
+    moe.moe_plan_destroy(q)
