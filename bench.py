@@ -150,6 +150,23 @@ def algorithmic_bytes(wl, d):
     return active * per_expert_w + act_bytes, active * per_expert_w, active
 
 
+def max_over_ranks(values, world, device):
+    """Element-wise max of per-rank times (each rank gets the result): a
+    replica job is as fast as its slowest rank."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def replica_throughput(tokens_per_rank, world, total_ms, steps):
+    """Whole-job tokens/s of `world` independent replicas (weak scaling), each
+    processing tokens_per_rank per step, timed by the slowest rank."""
+    return tokens_per_rank * world / (total_ms * 1e-3 / steps)
+
+
 def run_b200(args, wl):
     import torch
     import torch.distributed as dist
@@ -308,10 +325,7 @@ def run_b200(args, wl):
         raise RuntimeError("device error during timing")
 
     # ---- max over ranks
-    vals = torch.tensor([total_ms, sum(e2e_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    total_ms, e2e_total = float(vals[0]), float(vals[1])
+    total_ms, e2e_total = max_over_ranks([total_ms, sum(e2e_ms)], world, dev)
 
     alg_bytes, w_bytes, active = algorithmic_bytes(wl, d)
     hbm, bf16, bf16_sus, peak_src = _peaks()
@@ -340,10 +354,9 @@ def run_b200(args, wl):
                                            " bf16 burst" if tc_mult == 1.0 else
                                            " bf16 burst x2 (FP8 = 2x bf16 nominal)")
 
-    tokens = wl.T * world
     ms_per_step = total_ms / args.steps
     res = {
-        "metric": METRIC, "value": round(tokens / (total_ms * 1e-3 / args.steps), 1),
+        "metric": METRIC, "value": round(replica_throughput(wl.T, world, total_ms, args.steps), 1),
         "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": {"e4m3": "fp8_e4m3", "e2m1": "fp8_e4m3xe2m1",
@@ -361,7 +374,8 @@ def run_b200(args, wl):
         "eager_ms_per_step": round(sum(eager_ms) / args.steps, 4),
         "timing": "CUDA-graph replay of moe_forward, events on the launching stream",
         "roofline": roof,
-        "e2e": {"value": round(tokens / (e2e_total * 1e-3 / args.steps), 1), "unit": "tokens/s",
+        "e2e": {"value": round(replica_throughput(wl.T, world, e2e_total, args.steps), 1),
+                "unit": "tokens/s",
                 "h2d_bytes_per_step": int(sum(v.numel() * v.element_size() for v in host.values()
                                               if v is not None)),
                 "d2h_bytes_per_step": int(out_h.numel() * 2)},
@@ -405,7 +419,8 @@ def cpu_baseline(wl, d, args, ntok=None):
     """The float64 oracle, as it stands, on a bounded sample of the workload's
     tokens (the oracle's cost is dominated by dequantising the touched experts'
     weights, so a few tokens already take seconds)."""
-    dn = {k: v.cpu().numpy() for k, v in d.items()}
+    from moe_expert_ffn_permute_b200.synth import to_numpy
+    dn = to_numpy(d)
     ntok = ntok or args.cpu_tokens
     t0 = time.perf_counter()
     _oracle_sample(wl, dn, list(range(ntok)))
@@ -420,9 +435,9 @@ def run_reference(args, wl):
     if rank != 0:
         return
     import torch
-    from moe_expert_ffn_permute_b200.synth import make_inputs
+    from moe_expert_ffn_permute_b200.synth import make_inputs, to_numpy
     d = make_inputs(wl, device="cuda" if torch.cuda.is_available() else "cpu")
-    dn = {k: v.cpu().numpy() for k, v in d.items()}
+    dn = to_numpy(d)
     ntok = args.cpu_tokens
     for i in range(args.warmup):
         _oracle_sample(wl, dn, [i % wl.T])
