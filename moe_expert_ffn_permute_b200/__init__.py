@@ -68,6 +68,8 @@ _SIGS = {
     "moe_plan_set_weight_layout": (ctypes.c_int, [_P, ctypes.c_int]),
     "moe_plan_set_cta_pairs": (ctypes.c_int, [_P, ctypes.c_int]),
     "moe_plan_cta_pairs_active": (ctypes.c_int, [_P]),
+    "moe_plan_set_swap_ab": (ctypes.c_int, [_P, ctypes.c_int]),
+    "moe_plan_swap_ab_active": (ctypes.c_int, [_P]),
     "moe_prepack_weights": (ctypes.c_int, [_P] * 6),
     "moe_copy_act": (ctypes.c_int, [_P] * 4),
     "moe_clear_device_error": (ctypes.c_int, [_P] * 3),
@@ -237,6 +239,15 @@ def moe_plan_cta_pairs_active(plan):
     return bool(lib().moe_plan_cta_pairs_active(plan))
 
 
+def moe_plan_set_swap_ab(plan, mode):
+    """0: automatic, 1: never, 2: always use token-major (swap-AB) GEMM tiles."""
+    _check(lib().moe_plan_set_swap_ab(plan, int(mode)), "moe_plan_set_swap_ab")
+
+
+def moe_plan_swap_ab_active(plan):
+    return bool(lib().moe_plan_swap_ab_active(plan))
+
+
 def moe_prepack_weights(plan, w1, w2, w1_tiled, w2_tiled, stream=None):
     _check(lib().moe_prepack_weights(plan, *map(_ptr, (w1, w2, w1_tiled, w2_tiled)),
                                      _stream(stream)), "moe_prepack_weights")
@@ -269,7 +280,7 @@ class MoELayer:
 
     def __init__(self, T, H, I, E, k, w_dtype="e4m3", act="swiglu", alpha=1.0, up_bias=0.0,
                  limit=math.inf, device="cuda", debug=False, tiled_weights=False,
-                 cta_pairs=None):
+                 cta_pairs=None, swap_ab=None):
         import torch
         self.T, self.H, self.I, self.E, self.k = T, H, I, E, k
         self.plan = moe_plan(T, H, I, E, k, w_dtype, act, alpha, up_bias, limit)
@@ -277,6 +288,8 @@ class MoELayer:
             moe_plan_set_weight_layout(self.plan, True)
         if cta_pairs is not None:
             moe_plan_set_cta_pairs(self.plan, cta_pairs)
+        if swap_ab is not None:
+            moe_plan_set_swap_ab(self.plan, swap_ab)
         if debug:
             moe_plan_set_debug(self.plan, True)
         nbytes = moe_workspace_bytes(self.plan)

@@ -73,6 +73,19 @@ static bool use_pairs(const moe_plan_s* p) {
   return p->pair_mode == 2;
 }
 
+namespace moe {
+// Token-major (swap-AB) MMAs: the block-scaled MMA has M = 128, so with few
+// tokens per expert a token-row tile computes mostly padding; with the weights
+// as A and the tile's tokens as B (N = their count rounded up to 16) the
+// tensor work follows the tokens.  Chosen automatically when experts hold at
+// most 64 slots on average; not with CTA pairs or BF16 weights.
+bool use_swap(const moe_plan_s* p) {
+  if (p->w_dtype == MOE_W_BF16 || use_pairs(p) || p->swap_mode == 1) return false;
+  if (p->swap_mode == 2) return true;
+  return p->S <= 64ll * p->E;
+}
+}  // namespace moe
+
 static moe_status check_ws(moe_plan_t plan, const void* workspace) {
   if (plan == nullptr) return MOE_ERR_INVALID_ARG;
   if (workspace == nullptr) return MOE_ERR_INVALID_ARG;
@@ -130,6 +143,7 @@ moe_status moe_plan(int T, int H, int I, int E, int k, moe_dtypes dtypes, moe_ac
   p->debug_act_f32 = 0;
   p->w_tiled = 0;
   p->pair_mode = 0;
+  p->swap_mode = 0;
   p->S = static_cast<long long>(T) * k;
   // Sum over experts of ceil(n_e / 128) <= floor((S + 127 E) / 128).
   p->rows_cap = ((p->S + 127ll * E) / kTileM) * kTileM;
@@ -194,6 +208,17 @@ moe_status moe_plan_set_debug(moe_plan_t plan, int capture_act_f32) {
   plan->debug_act_f32 = capture_act_f32 ? 1 : 0;
   moe::compute_layout(plan);
   return MOE_OK;
+}
+
+moe_status moe_plan_set_swap_ab(moe_plan_t plan, int mode) {
+  if (plan == nullptr || mode < 0 || mode > 2) return MOE_ERR_INVALID_ARG;
+  if (mode == 2 && plan->w_dtype == MOE_W_BF16) return MOE_ERR_UNSUPPORTED;
+  plan->swap_mode = mode;
+  return MOE_OK;
+}
+
+int moe_plan_swap_ab_active(moe_plan_t plan) {
+  return plan != nullptr && moe::use_swap(plan) ? 1 : 0;
 }
 
 int moe_plan_cta_pairs_active(moe_plan_t plan) {

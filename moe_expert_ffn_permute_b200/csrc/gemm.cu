@@ -70,6 +70,8 @@ struct __align__(1024) Smem {
   int4 task[SCHED_DEPTH];          // kind | reuse << 1 | expert << 2, m-tile, n-tile, rows
   int task_pos[SCHED_DEPTH];       // position (unpadded) of the tile's first row
   float amax[2][2][BM];            // [tile parity][half][row]
+  float swap_red[2][4][64];        // token-major FC1: per-warp amax [half][sub-partition][token]
+  float swap_inv[2][64];           // token-major FC1: 1 / 2^n per token [half][token]
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -91,6 +93,7 @@ struct Params {
   int E, I, H;
   int phases;                // bit 0: FC1 tiles, bit 1: FC2 tiles
   int dynamic;               // tiles from a global counter (else round-robin)
+  int swap;                  // token-major MMAs (weights as A, the tile's tokens as B)
   Phase ph[2];
   const int32_t* tile_off;
   const int32_t* counts;
@@ -444,13 +447,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_cp_32x128b_warpx4(sfa, sf_desc(smem_u32(sm.sfa[stage])));
             tmem_cp_32x128b_warpx4(sfb, sf_desc(smem_u32(sm.sfb[stage])));
             tmem_cp_32x128b_warpx4(sfb + 4, sf_desc(smem_u32(sm.sfb[stage] + 512)));
+            if (p.swap) {
+              // Token-major: each 128-row half of the weight tile is the A
+              // operand (its scales: the weight chunk), the tile's tokens are B
+              // with N = their count rounded up to 16 (scales: the token chunk).
+              // D0 (columns 0..) holds the first half, D1 (columns 128..) the second.
+              const uint32_t n = static_cast<uint32_t>(min(128, max(16, (t.rows + 15) & ~15)));
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              const uint32_t idesc = mxf8f6f4_idesc(kFp4 ? 5u : 0u, BN, ks);
-              mma_mxf8f6f4(tmem + kAccCol, umma_desc_sw128(a_base + ks * 32),
-                           umma_desc_sw128(b_base + ks * 32), idesc,
-                           sfa | (static_cast<uint32_t>(ks) << 30),
-                           sfb | (static_cast<uint32_t>(ks) << 30), (kb > 0 || ks > 0) ? 1u : 0u);
+              for (int ks = 0; ks < 4; ++ks) {
+                const uint32_t idesc = mxf8f6f4_idesc_ab(kFp4 ? 5u : 0u, 0u, n, ks);
+                const uint32_t ksh = static_cast<uint32_t>(ks) << 30;
+                const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
+                mma_mxf8f6f4(tmem + kAccCol, umma_desc_sw128(b_base + ks * 32),
+                             umma_desc_sw128(a_base + ks * 32), idesc, sfb | ksh, sfa | ksh, acc);
+                mma_mxf8f6f4(tmem + kAccCol + 128, umma_desc_sw128(b_base + 128 * BK + ks * 32),
+                             umma_desc_sw128(a_base + ks * 32), idesc, (sfb + 4) | ksh,
+                             sfa | ksh, acc);
+              }
+            } else {
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks) {
+                const uint32_t idesc = mxf8f6f4_idesc(kFp4 ? 5u : 0u, BN, ks);
+                mma_mxf8f6f4(tmem + kAccCol, umma_desc_sw128(a_base + ks * 32),
+                             umma_desc_sw128(b_base + ks * 32), idesc,
+                             sfa | (static_cast<uint32_t>(ks) << 30),
+                             sfb | (static_cast<uint32_t>(ks) << 30), (kb > 0 || ks > 0) ? 1u : 0u);
+              }
             }
           }
           tc_commit(&sm.empty[stage]);
@@ -484,6 +506,134 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (t.e < 0) break;
       if (!mbar_wait(&sm.tmem_full, acc_phase, p.err, &sm.abort_flag)) break;
       tc_fence_after();
+      if (!kBf16 && p.swap) {
+        // Token-major tile: TMEM lane = feature, column = token.  This warp
+        // owns feature f of the tile for the tokens of its half.
+        const int f = q * 32 + lane;
+        if (t.kind == 0) {
+          const int tok0 = half * 64;
+          const int ntok = min(64, t.rows - tok0);   // uniform over the half's warps
+          // (Loaded unconditionally: TMEM columns are always addressable, and a
+          // conditional load would move the arrays to local memory.)
+          uint32_t g[64], u[64];
+          tmem_ld_32x32b_x32(t_row + kAccCol + tok0, *reinterpret_cast<uint32_t(*)[32]>(g));
+          tmem_ld_32x32b_x32(t_row + kAccCol + tok0 + 32,
+                             *reinterpret_cast<uint32_t(*)[32]>(g + 32));
+          tmem_ld_32x32b_x32(t_row + kAccCol + 128 + tok0, *reinterpret_cast<uint32_t(*)[32]>(u));
+          tmem_ld_32x32b_x32(t_row + kAccCol + 128 + tok0 + 32,
+                             *reinterpret_cast<uint32_t(*)[32]>(u + 32));
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.tmem_empty);
+          if (ntok > 0) {
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+              float gv = __uint_as_float(g[j]);
+              float uv = __uint_as_float(u[j]);
+              float a;
+              if (p.oai) {
+                gv = fminf(gv, p.limit);
+                uv = fminf(fmaxf(uv, -p.limit), p.limit);
+                a = gv * sigmoidf_fast(p.alpha * gv) * (uv + p.up_bias);
+              } else {
+                a = gv * sigmoidf_fast(gv) * uv;
+              }
+              g[j] = __float_as_uint(j < ntok ? a : 0.0f);
+            }
+            // amax of every token over this warp's 32 features (lanes), then
+            // over the half's four warps (128 features = one requant block).
+            // Transpose-reduction per 32 tokens: at the step with lane offset o
+            // a lane keeps the o tokens of its side of bit o and trades the
+            // other o with its partner, so after 31 shuffles lane l holds the
+            // maximum of token l.
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              if (32 * r < ntok) {
+                float m[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) m[i] = fabsf(__uint_as_float(g[32 * r + i]));
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) {
+                  const bool upper = (lane & o) != 0;
+#pragma unroll
+                  for (int i = 0; i < o; ++i) {
+                    const float send = upper ? m[i] : m[i + o];
+                    const float keep = upper ? m[i + o] : m[i];
+                    m[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, o));
+                  }
+                }
+                sm.swap_red[half][q][32 * r + lane] = m[0];
+              }
+            }
+            named_barrier_sync(1 + half, 128);
+            const int nb = p.I / 128;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const int j = lane + 32 * c;
+              if (j < ntok) {
+                const float m = fmaxf(fmaxf(sm.swap_red[half][0][j], sm.swap_red[half][1][j]),
+                                      fmaxf(sm.swap_red[half][2][j], sm.swap_red[half][3][j]));
+                const int n = ue8m0_exponent(m);
+                if (q == 0) sm.swap_inv[half][j] = __uint_as_float(static_cast<uint32_t>(127 - n) << 23);
+                if (q == 0) {
+                  const int rr = tok0 + j;   // row of the m-tile
+                  *reinterpret_cast<uint32_t*>(
+                      p.act_sf_chunks + (static_cast<size_t>(t.mt) * nb + t.nt) * 512 +
+                      (rr & 31) * 16 + (rr >> 5) * 4) = (static_cast<uint32_t>(n + 127) & 0xFFu) * 0x01010101u;
+                }
+              }
+            }
+            named_barrier_sync(1 + half, 128);
+            uint8_t* tile = p.act + (static_cast<size_t>(t.mt) * nb + t.nt) * kTileBytes;
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+              if (j < ntok) {
+                const float av = __uint_as_float(g[j]);
+                const int rr = tok0 + j;
+                tile[swz128(rr, f >> 4) + (f & 15)] =
+                    static_cast<uint8_t>(cvt_e4m3x2(av * sm.swap_inv[half][j], 0.0f) & 0xFFu);
+                if (p.act_f32 != nullptr)
+                  p.act_f32[(static_cast<size_t>(t.mt) * BM + rr) * p.I + t.nt * 128 + f] = av;
+              }
+            }
+          }
+          if (p.phases & 2) {
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) atomicAdd(p.fc1_done + t.mt, 1u);
+          }
+        } else {
+          uint32_t v[128];
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            tmem_ld_32x32b_x32(t_row + kAccCol + half * 128 + c * 32,
+                               *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c));
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.tmem_empty);
+          const int h = t.nt * 256 + half * 128 + f;   // output column
+          int pl[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int j = lane + 32 * c;
+            pl[c] = j < t.rows ? p.perm[t.pos + j] : 0;
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+              const int sl = __shfl_sync(0xffffffffu, pl[c], jj);
+              if (c * 32 + jj < t.rows)
+                p.y[static_cast<size_t>(sl) * p.H + h] =
+                    static_cast<uint16_t>(pack_bf16x2(__uint_as_float(v[c * 32 + jj]), 0.0f) & 0xFFFFu);
+            }
+          }
+        }
+        acc_phase ^= 1u;
+        continue;
+      }
       if (t.kind == 0) {
         uint32_t g[64], u[64];
         tmem_ld_32x32b_x32(t_row + kAccCol + half * 64, *reinterpret_cast<uint32_t(*)[32]>(g));
@@ -691,6 +841,7 @@ cudaError_t launch_gemm(const moe_plan_s* pl, int phases, bool dynamic, const vo
   p.H = pl->H;
   p.phases = phases;
   p.dynamic = dynamic ? 1 : 0;
+  p.swap = use_swap(pl) ? 1 : 0;
   long long max_tiles = 0;
   const bool tiled = pl->w_tiled != 0;
   constexpr bool kFp4 = kW == kWFp4;

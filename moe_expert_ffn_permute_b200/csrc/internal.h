@@ -41,6 +41,7 @@ struct moe_plan_s {
   int debug_act_f32;
   int w_tiled;           // weights given as pre-swizzled tiles (moe_prepack_weights)
   int pair_mode;         // 2-SM GEMM: 0 automatic, 1 never, 2 always
+  int swap_mode;         // token-major MMAs: 0 automatic, 1 never, 2 always
   long long S;           // T*k
   long long rows_cap;    // padded row capacity (multiple of 128)
   int route_blocks;
@@ -50,6 +51,7 @@ struct moe_plan_s {
 namespace moe {
 
 void compute_layout(moe_plan_s* p);
+bool use_swap(const moe_plan_s* p);   // token-major (swap-AB) MMAs in the GEMM
 
 // Launch with programmatic stream serialization: the kernel may start while its
 // predecessor in the stream finishes; it must execute griddep_wait() before

@@ -260,6 +260,14 @@ __host__ __device__ constexpr uint32_t mxf8f6f4_idesc(uint32_t b_format, uint32_
          ((128u >> 4) << 24) | (sf_id << 29);
 }
 
+// Block-scaled descriptor with both operand formats given (E4M3 = 0, E2M1 =
+// 5): used when the weights are the A operand (token-major "swap AB" tiles).
+__host__ __device__ constexpr uint32_t mxf8f6f4_idesc_ab(uint32_t a_format, uint32_t b_format,
+                                                         uint32_t n, uint32_t sf_id) {
+  return (sf_id << 4) | (a_format << 7) | (b_format << 10) | ((n >> 3) << 17) | (1u << 23) |
+         ((128u >> 4) << 24) | (sf_id << 29);
+}
+
 __device__ __forceinline__ void mma_mxf8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                              uint32_t idesc, uint32_t sfa_tmem,
                                              uint32_t sfb_tmem, uint32_t accumulate) {
@@ -335,6 +343,12 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
       "}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// Barrier among `threads` threads (whole warps) of the CTA, id 1..15 (0 is
+// __syncthreads).
+__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -163,3 +163,30 @@ def test_bf16_plans_take_no_scales_and_tiled_weights():
     assert moe.moe_workspace_bytes(p) > moe.moe_workspace_bytes(q)
     moe.moe_plan_destroy(p)
     moe.moe_plan_destroy(q)
+
+
+def test_swap_ab_selection():
+    """Token-major tiles: automatic at <= 64 slots per expert on average, never
+    with BF16 weights or CTA pairs, forced on or off by the mode."""
+    p = moe.moe_plan(128, 7168, 2048, 32, 8)            # 1024 slots, 32 experts
+    assert moe.moe_plan_swap_ab_active(p)
+    moe.moe_plan_set_swap_ab(p, 1)
+    assert not moe.moe_plan_swap_ab_active(p)
+    moe.moe_plan_set_weight_layout(p, True)
+    moe.moe_plan_set_swap_ab(p, 2)
+    assert moe.moe_plan_swap_ab_active(p)
+    moe.moe_plan_set_cta_pairs(p, 2)                    # pairs take precedence
+    assert not moe.moe_plan_swap_ab_active(p)
+    moe.moe_plan_destroy(p)
+    q = moe.moe_plan(8192, 7168, 2048, 32, 8)           # 65536 slots: token-row tiles
+    assert not moe.moe_plan_swap_ab_active(q)
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_plan_set_swap_ab(q, 3)
+    assert ei.value.status == 1
+    moe.moe_plan_destroy(q)
+    b = moe.moe_plan(128, 512, 256, 8, 2, w_dtype="bf16")
+    assert not moe.moe_plan_swap_ab_active(b)
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_plan_set_swap_ab(b, 2)
+    assert ei.value.status == 2
+    moe.moe_plan_destroy(b)

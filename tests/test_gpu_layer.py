@@ -258,9 +258,10 @@ def test_tiled_weights_full_size_parity(name, ntok):
 
 
 def _run_mode(wl, d, pairs, debug=False):
+    # The pair kernel computes token-row tiles; its single-CTA reference does too.
     lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype=wl.w_dtype, act=wl.act,
                        alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit, tiled_weights=True,
-                       cta_pairs=pairs, debug=debug)
+                       cta_pairs=pairs, swap_ab=1, debug=debug)
     w1t, w2t = lay.prepack(d["w1"], d["w2"])
     out = lay.forward(d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], w1t, d["w1_scales"],
                       w2t, d["w2_scales"])
@@ -377,3 +378,95 @@ def test_fused_route_gather_writes_the_same_bytes(case):
         else:
             assert diff.numel() == 0, how
         assert lay.check() == (6 if case == "bad-ids" else 0)
+
+
+
+SWAP_CASES = [RAGGED, RAGGED_FP4, RAGGED_OAI, WORKLOADS["tiny"], SINGLE]
+
+
+def _layer_swap(wl, swap, debug=False, tiled=False):
+    return moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype=wl.w_dtype, act=wl.act,
+                        alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit, debug=debug,
+                        tiled_weights=tiled, swap_ab=swap)
+
+
+@pytest.mark.parametrize("wl", SWAP_CASES, ids=lambda w: w.name)
+def test_token_major_tiles_match_oracle(wl):
+    """Swap-AB GEMM tiles (weights as A, tokens as B) forced on: parity with the
+    oracle, including experts with more than 64 and more than 128 rows."""
+    d = inputs(wl)
+    lay = _layer_swap(wl, 2)
+    assert moe.moe_plan_swap_ab_active(lay.plan)
+    out = lay.forward(d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], d["w1"],
+                      d["w1_scales"], d["w2"], d["w2_scales"])
+    torch.cuda.synchronize()
+    assert lay.check() == 0
+    ref = L.layer(*oracle_args(to_numpy(d)), **oracle_kw(wl))
+    assert_parity(out.float().cpu().numpy(), ref, f"swap {wl.name}")
+
+
+@pytest.mark.parametrize("wl", [RAGGED, RAGGED_FP4], ids=lambda w: w.name)
+def test_token_major_requant_bytes_exact(wl):
+    """With swap-AB tiles the FC1 epilogue reduces each token's amax across
+    lanes; its FP8 codes and scales equal the oracle quantiser applied to the
+    GPU's own fp32 activation, byte for byte."""
+    d = inputs(wl)
+    lay = _layer_swap(wl, 2, debug=True)
+    lay.forward(d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], d["w1"], d["w1_scales"],
+                d["w2"], d["w2_scales"])
+    torch.cuda.synchronize()
+    v = lay.view()
+    rows = v.rows
+    act_t = torch.empty(rows, wl.I, dtype=torch.uint8, device="cuda")
+    moe.moe_copy_act(lay.plan, lay.workspace, act_t)
+    a32 = _ws_bytes(lay, v.act_f32, rows * wl.I * 4).view(torch.float32).view(rows, wl.I)
+    sf = torch.empty(rows, wl.I // 128, dtype=torch.uint8, device="cuda")
+    moe.moe_copy_act_scales(lay.plan, lay.workspace, sf)
+    counts = _ws_bytes(lay, v.counts, 4 * wl.E).view(torch.int32).cpu().numpy()
+    pad = _ws_bytes(lay, v.pad_offsets, 4 * (wl.E + 1)).view(torch.int32).cpu().numpy()
+    act, a32, sf = act_t.cpu().numpy(), a32.cpu().numpy(), sf.cpu().numpy()
+    for e in range(wl.E):
+        r = slice(pad[e], pad[e] + counts[e])
+        q_ref, s_ref = L.requant_1x128(a32[r].astype(np.float64))
+        np.testing.assert_array_equal(act[r], q_ref, err_msg=f"codes, expert {e}")
+        np.testing.assert_array_equal(sf[r], s_ref, err_msg=f"scales, expert {e}")
+
+
+def test_token_major_fused_equals_separate_and_tiled_equals_row_major():
+    wl = RAGGED
+    d = inputs(wl)
+    outs = []
+    for tiled in (False, True):
+        lay = _layer_swap(wl, 2, tiled=tiled)
+        w1, w2 = lay.prepack(d["w1"], d["w2"]) if tiled else (d["w1"], d["w2"])
+        outs.append(lay.forward(d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], w1,
+                                d["w1_scales"], w2, d["w2_scales"]))
+        torch.cuda.synchronize()
+        if not tiled:
+            v = lay.view()
+            n = wl.T * wl.k * wl.H * 2
+            off = v.y - lay.workspace.data_ptr()
+            y_fused = lay.workspace[off:off + n].clone()
+            moe.moe_route(lay.plan, d["topk_idx"], lay.workspace)
+            moe.moe_gather(lay.plan, d["x"], d["x_scales"], lay.workspace)
+            moe.moe_fc1(lay.plan, w1, d["w1_scales"], lay.workspace)
+            moe.moe_fc2(lay.plan, w2, d["w2_scales"], lay.workspace)
+            torch.cuda.synchronize()
+            assert torch.equal(lay.workspace[off:off + n], y_fused)
+    assert torch.equal(outs[0], outs[1])
+
+
+def test_token_major_decode_full_size():
+    """The decode layer (T=128, E=32, k=8) picks swap-AB tiles automatically."""
+    wl = WORKLOADS["decode"]
+    d = inputs(wl)
+    lay = _layer_swap(wl, None, tiled=True)
+    assert moe.moe_plan_swap_ab_active(lay.plan)
+    w1, w2 = lay.prepack(d["w1"], d["w2"])
+    out = lay.forward(d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], w1, d["w1_scales"],
+                      w2, d["w2_scales"])
+    torch.cuda.synchronize()
+    assert lay.check() == 0
+    tokens = np.sort(np.random.default_rng(4).choice(wl.T, size=8, replace=False))
+    ref = oracle_tokens(wl, to_numpy(d), tokens)
+    assert_parity(out.float().cpu().numpy()[tokens], ref, "decode swap")
