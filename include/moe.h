@@ -289,14 +289,14 @@ int moe_plan_cta_pairs_active(moe_plan_t plan);
 
 /* Token-major ("swap AB") GEMM tiles, the swapAB variant of the Mega MoE
  * kernels (DeepGEMM PR #445, Summary and its calc_diff table).  The
- * block-scaled tensor-core MMA has M = 128; with few tokens per expert a tile
+ * tensor-core MMAs used here have M = 128; with few tokens per expert a tile
  * of 128 token rows is mostly padding.  With swap AB each 128-row weight block
  * is the A operand and the tile's tokens are B, with N = their count rounded
  * up to 16, so the tensor work follows the tokens.  mode 0: automatic (when
  * T*k <= 64*E, i.e. at most 64 slots per expert on average), 1: never,
- * 2: always (MOE_ERR_UNSUPPORTED for BF16 weights).  Not combined with CTA
- * pairs.  Results agree with the token-row tiles within rounding (the sums run
- * in a different order inside the MMA).                                      */
+ * 2: always.  All weight formats; not combined with CTA pairs.  Results
+ * agree with the token-row tiles within rounding (the sums run in a different
+ * order inside the MMA).                                                     */
 moe_status moe_plan_set_swap_ab(moe_plan_t plan, int mode);
 
 /* 1 if the GEMMs use token-major tiles with the plan's current settings.     */

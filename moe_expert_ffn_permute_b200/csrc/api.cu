@@ -74,13 +74,13 @@ static bool use_pairs(const moe_plan_s* p) {
 }
 
 namespace moe {
-// Token-major (swap-AB) MMAs: the block-scaled MMA has M = 128, so with few
+// Token-major (swap-AB) MMAs: the MMAs used here have M = 128, so with few
 // tokens per expert a token-row tile computes mostly padding; with the weights
 // as A and the tile's tokens as B (N = their count rounded up to 16) the
 // tensor work follows the tokens.  Chosen automatically when experts hold at
-// most 64 slots on average; not with CTA pairs or BF16 weights.
+// most 64 slots on average; not with CTA pairs.
 bool use_swap(const moe_plan_s* p) {
-  if (p->w_dtype == MOE_W_BF16 || use_pairs(p) || p->swap_mode == 1) return false;
+  if (use_pairs(p) || p->swap_mode == 1) return false;
   if (p->swap_mode == 2) return true;
   return p->S <= 64ll * p->E;
 }
@@ -212,7 +212,6 @@ moe_status moe_plan_set_debug(moe_plan_t plan, int capture_act_f32) {
 
 moe_status moe_plan_set_swap_ab(moe_plan_t plan, int mode) {
   if (plan == nullptr || mode < 0 || mode > 2) return MOE_ERR_INVALID_ARG;
-  if (mode == 2 && plan->w_dtype == MOE_W_BF16) return MOE_ERR_UNSUPPORTED;
   plan->swap_mode = mode;
   return MOE_OK;
 }

@@ -433,11 +433,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t b_base = smem_u32(sm.b[stage]);
           if (kBf16) {
             // 128 bytes of K = 64 BF16 values: four MMAs of K = 16 (32 bytes each).
+            if (p.swap) {
+              // Token-major, as for the block-scaled formats below.
+              const uint32_t n = static_cast<uint32_t>(min(128, max(16, (t.rows + 15) & ~15)));
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-              mma_bf16(tmem + kAccCol, umma_desc_sw128(a_base + ks * 32),
-                       umma_desc_sw128(b_base + ks * 32), bf16_idesc(BN),
-                       (kb > 0 || ks > 0) ? 1u : 0u);
+              for (int ks = 0; ks < 4; ++ks) {
+                const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
+                mma_bf16(tmem + kAccCol, umma_desc_sw128(b_base + ks * 32),
+                         umma_desc_sw128(a_base + ks * 32), bf16_idesc(n), acc);
+                mma_bf16(tmem + kAccCol + 128, umma_desc_sw128(b_base + 128 * BK + ks * 32),
+                         umma_desc_sw128(a_base + ks * 32), bf16_idesc(n), acc);
+              }
+            } else {
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tmem + kAccCol, umma_desc_sw128(a_base + ks * 32),
+                         umma_desc_sw128(b_base + ks * 32), bf16_idesc(BN),
+                         (kb > 0 || ks > 0) ? 1u : 0u);
+            }
           } else {
             // MXFP4 weight scales land by cp.async (generic proxy): order them
             // before the tensor core's (async proxy) reads of shared memory.
@@ -506,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (t.e < 0) break;
       if (!mbar_wait(&sm.tmem_full, acc_phase, p.err, &sm.abort_flag)) break;
       tc_fence_after();
-      if (!kBf16 && p.swap) {
+      if (p.swap) {
         // Token-major tile: TMEM lane = feature, column = token.  This warp
         // owns feature f of the tile for the tokens of its half.
         const int f = q * 32 + lane;
@@ -541,6 +554,25 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               g[j] = __float_as_uint(j < ntok ? a : 0.0f);
             }
+          }
+          if (kBf16 && ntok > 0) {
+            // BF16 activation, token-major: feature f of n-tile nt is column
+            // 128 * nt + f, i.e. byte 2 * (f % 64) of a row of activation tile
+            // (m-tile, 2 * nt + f / 64).
+            uint8_t* tile = p.act + (static_cast<size_t>(t.mt) * (p.I / 64) + 2 * t.nt + (f >> 6)) *
+                                        kTileBytes;
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+              if (j < ntok) {
+                const float av = __uint_as_float(g[j]);
+                const int rr = tok0 + j;
+                *reinterpret_cast<uint16_t*>(tile + swz128(rr, (f & 63) >> 3) + (f & 7) * 2) =
+                    static_cast<uint16_t>(pack_bf16x2(av, 0.0f) & 0xFFFFu);
+                if (p.act_f32 != nullptr)
+                  p.act_f32[(static_cast<size_t>(t.mt) * BM + rr) * p.I + t.nt * 128 + f] = av;
+              }
+            }
+          } else if (ntok > 0) {
             // amax of every token over this warp's 32 features (lanes), then
             // over the half's four warps (128 features = one requant block).
             // Transpose-reduction per 32 tokens: at the step with lane offset o

@@ -24,36 +24,38 @@ def _built():
     ensure_built()
 
 
-def _layer(wl, tiled=False, debug=False):
+def _layer(wl, tiled=False, debug=False, swap=None):
     return moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype="bf16", act=wl.act,
                         alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit, debug=debug,
-                        tiled_weights=tiled)
+                        tiled_weights=tiled, swap_ab=swap)
 
 
-def _run(wl, d, tiled=False, debug=False):
-    lay = _layer(wl, tiled, debug)
+def _run(wl, d, tiled=False, debug=False, swap=None):
+    lay = _layer(wl, tiled, debug, swap)
     w1, w2 = (lay.prepack(d["w1"], d["w2"]) if tiled else (d["w1"], d["w2"]))
     out = lay.forward(d["x"], None, d["topk_idx"], d["topk_w"], w1, None, w2, None)
     torch.cuda.synchronize()
     return out, lay
 
 
+@pytest.mark.parametrize("swap", [1, 2], ids=["token-rows", "swap-ab"])
 @pytest.mark.parametrize("wl", [RAGGED_BF16, OAI_BF16, SINGLE_BF16], ids=lambda w: w.name)
-def test_layer_matches_oracle(wl):
+def test_layer_matches_oracle(wl, swap):
     d = inputs(wl)
-    out, lay = _run(wl, d)
+    out, lay = _run(wl, d, swap=swap)
     assert lay.check() == 0
     ref = oracle_layer(wl, to_numpy(d))
     assert_parity(out.float().cpu().numpy(), ref, wl.name)
 
 
-def test_activation_is_bf16_rne_of_the_fp32_activation():
+@pytest.mark.parametrize("swap", [1, 2], ids=["token-rows", "swap-ab"])
+def test_activation_is_bf16_rne_of_the_fp32_activation(swap):
     """The FC1 epilogue's bf16 activation equals the oracle's round-to-nearest-
     even of the GPU's own fp32 activation (debug capture), bit for bit, on every
     routed row; and that fp32 activation matches the oracle's float64 one."""
     wl = RAGGED_BF16
     d = inputs(wl)
-    out, lay = _run(wl, d, debug=True)
+    out, lay = _run(wl, d, debug=True, swap=swap)
     v = lay.view()
     rows = v.rows
     act = torch.empty(rows, wl.I, dtype=torch.bfloat16, device="cuda")
