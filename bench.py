@@ -191,7 +191,8 @@ def run_b200(args, wl):
     tiled = wl.w_dtype in ("e4m3", "bf16") and not args.row_major_weights
     lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype=wl.w_dtype, act=wl.act,
                        alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit, device=dev,
-                       tiled_weights=tiled, cta_pairs=args.cta_pairs if tiled else None)
+                       tiled_weights=tiled, cta_pairs=args.cta_pairs if tiled else None,
+                       swap_ab=args.swap_ab)
     pairs = moe.moe_plan_cta_pairs_active(lay.plan)
     d_row_major = dict(d)          # the oracle reads the original layout
     if tiled:
@@ -368,6 +369,9 @@ def run_b200(args, wl):
                    "w_dtype": wl.w_dtype, "routing": wl.routing, "act": wl.act,
                    "active_experts": active, "l2": "flushed (256 MiB write) before each step",
                    "weights": "tiled (moe_prepack_weights, once)" if tiled else "row-major",
+                   "gemm_tiles": {0: "token rows", 1: "token-major (swap AB)",
+                                  2: "token-major for tiles of <= 96 tokens, else token rows"}[
+                       moe.moe_plan_swap_ab_active(lay.plan)],
                    "parallelism": f"replicas x{world}"},
         "achieved": {"tflops": round(flops / (ms_per_step * 1e-3) / 1e12, 2),
                      "hbm_gbs": round(alg_bytes / (ms_per_step * 1e-3) / 1e9, 1),
@@ -477,6 +481,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cta-pairs", type=int, default=0, choices=[0, 1, 2],
                     help="GEMM on CTA pairs: 0 automatic, 1 never, 2 always (tiled FP8 only)")
+    ap.add_argument("--swap-ab", type=int, default=0, choices=[0, 1, 2],
+                    help="token-major GEMM tiles: 0 tile by tile (automatic), 1 never, 2 always")
     ap.add_argument("--row-major-weights", action="store_true",
                     help="read FP8 weights row-major via 2-D TMA instead of prepacked tiles")
     args = ap.parse_args()

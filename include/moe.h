@@ -289,17 +289,18 @@ int moe_plan_cta_pairs_active(moe_plan_t plan);
 
 /* Token-major ("swap AB") GEMM tiles, the swapAB variant of the Mega MoE
  * kernels (DeepGEMM PR #445, Summary and its calc_diff table).  The
- * tensor-core MMAs used here have M = 128; with few tokens per expert a tile
- * of 128 token rows is mostly padding.  With swap AB each 128-row weight block
- * is the A operand and the tile's tokens are B, with N = their count rounded
- * up to 16, so the tensor work follows the tokens.  mode 0: automatic (when
- * T*k <= 64*E, i.e. at most 64 slots per expert on average), 1: never,
- * 2: always.  All weight formats; not combined with CTA pairs.  Results
- * agree with the token-row tiles within rounding (the sums run in a different
- * order inside the MMA).                                                     */
+ * tensor-core MMAs used here have M = 128; a tile with few token rows (an
+ * expert's last, ragged tile; every tile at decode sizes) is mostly padding.
+ * With swap AB each 128-row weight block is the A operand and the tile's
+ * tokens are B, with N = their count rounded up to 16, so the tensor work
+ * follows the tokens.  mode 0: automatic, tile by tile (token-major for tiles
+ * of at most 96 tokens), 1: never, 2: every tile.  All weight formats; not
+ * combined with CTA pairs.  Results agree with token-row tiles within rounding
+ * (the sums run in a different order inside the MMA) and are deterministic. */
 moe_status moe_plan_set_swap_ab(moe_plan_t plan, int mode);
 
-/* 1 if the GEMMs use token-major tiles with the plan's current settings.     */
+/* 0: the GEMMs use token-row tiles only; 1: token-major tiles throughout;
+ * 2: chosen tile by tile (automatic mode).                                   */
 int moe_plan_swap_ab_active(moe_plan_t plan);
 
 /* Rearrange row-major FP8 or BF16 weights w1 [E,2I,H] and w2 [E,H,I] (device)

@@ -245,7 +245,8 @@ def moe_plan_set_swap_ab(plan, mode):
 
 
 def moe_plan_swap_ab_active(plan):
-    return bool(lib().moe_plan_swap_ab_active(plan))
+    """0: token-row tiles only, 1: token-major throughout, 2: tile by tile."""
+    return int(lib().moe_plan_swap_ab_active(plan))
 
 
 def moe_prepack_weights(plan, w1, w2, w1_tiled, w2_tiled, stream=None):

@@ -74,15 +74,14 @@ static bool use_pairs(const moe_plan_s* p) {
 }
 
 namespace moe {
-// Token-major (swap-AB) MMAs: the MMAs used here have M = 128, so with few
-// tokens per expert a token-row tile computes mostly padding; with the weights
-// as A and the tile's tokens as B (N = their count rounded up to 16) the
-// tensor work follows the tokens.  Chosen automatically when experts hold at
-// most 64 slots on average; not with CTA pairs.
-bool use_swap(const moe_plan_s* p) {
-  if (use_pairs(p) || p->swap_mode == 1) return false;
-  if (p->swap_mode == 2) return true;
-  return p->S <= 64ll * p->E;
+// Token-major (swap-AB) MMAs: the MMAs used here have M = 128, so a tile with
+// few token rows computes mostly padding; with the weights as A and the tile's
+// tokens as B (N = their count rounded up to 16) the tensor work follows the
+// tokens.  Returns the kernel's mode: 0 never (mode 1, or CTA pairs), 1 every
+// tile (mode 2), 2 tile by tile from its row count (mode 0, automatic).
+int use_swap(const moe_plan_s* p) {
+  if (use_pairs(p) || p->swap_mode == 1) return 0;
+  return p->swap_mode == 2 ? 1 : 2;
 }
 }  // namespace moe
 
@@ -217,7 +216,7 @@ moe_status moe_plan_set_swap_ab(moe_plan_t plan, int mode) {
 }
 
 int moe_plan_swap_ab_active(moe_plan_t plan) {
-  return plan != nullptr && moe::use_swap(plan) ? 1 : 0;
+  return plan == nullptr ? 0 : moe::use_swap(plan);
 }
 
 int moe_plan_cta_pairs_active(moe_plan_t plan) {

@@ -53,6 +53,10 @@ constexpr uint32_t kAccCol = 0, kSfaCol = 256, kSfbCol = 264, kSfSetStride = 16;
 constexpr int kEpiWarps = 8;
 constexpr int kSchedConsumers = 3 + kEpiWarps;   // 2 producers, MMA, epilogue warps
 constexpr uint64_t kDepWaitLimitNs = 2000000000ull;
+// Automatic swap-AB: a tile of r token rows costs 2 x 128 x round16(r) MMA
+// work token-major against 128 x 256 token-row, but its FC1 epilogue does more
+// (a cross-lane amax, a barrier, byte stores); token-major from this size down.
+constexpr int kSwapRows = 96;
 
 struct __align__(1024) Smem {
   uint8_t a[STAGES][BM * BK];
@@ -93,7 +97,8 @@ struct Params {
   int E, I, H;
   int phases;                // bit 0: FC1 tiles, bit 1: FC2 tiles
   int dynamic;               // tiles from a global counter (else round-robin)
-  int swap;                  // token-major MMAs (weights as A, the tile's tokens as B)
+  int swap;                  // token-major MMAs (weights as A, the tile's tokens as B):
+                             // 0 never, 1 always, 2 for tiles of at most kSwapRows rows
   Phase ph[2];
   const int32_t* tile_off;
   const int32_t* counts;
@@ -163,6 +168,10 @@ __device__ __forceinline__ bool get_task_single(Smem& sm, int& slot, uint32_t& p
     phase ^= 1u;
   }
   return true;
+}
+
+__device__ __forceinline__ bool swap_tile(const Params& p, int rows) {
+  return p.swap == 1 || (p.swap == 2 && rows <= kSwapRows);
 }
 
 __device__ __forceinline__ float sigmoidf_fast(float z) {
@@ -433,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t b_base = smem_u32(sm.b[stage]);
           if (kBf16) {
             // 128 bytes of K = 64 BF16 values: four MMAs of K = 16 (32 bytes each).
-            if (p.swap) {
+            if (swap_tile(p, t.rows)) {
               // Token-major, as for the block-scaled formats below.
               const uint32_t n = static_cast<uint32_t>(min(128, max(16, (t.rows + 15) & ~15)));
 #pragma unroll
@@ -460,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_cp_32x128b_warpx4(sfa, sf_desc(smem_u32(sm.sfa[stage])));
             tmem_cp_32x128b_warpx4(sfb, sf_desc(smem_u32(sm.sfb[stage])));
             tmem_cp_32x128b_warpx4(sfb + 4, sf_desc(smem_u32(sm.sfb[stage] + 512)));
-            if (p.swap) {
+            if (swap_tile(p, t.rows)) {
               // Token-major: each 128-row half of the weight tile is the A
               // operand (its scales: the weight chunk), the tile's tokens are B
               // with N = their count rounded up to 16 (scales: the token chunk).
@@ -519,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (t.e < 0) break;
       if (!mbar_wait(&sm.tmem_full, acc_phase, p.err, &sm.abort_flag)) break;
       tc_fence_after();
-      if (p.swap) {
+      if (swap_tile(p, t.rows)) {
         // Token-major tile: TMEM lane = feature, column = token.  This warp
         // owns feature f of the tile for the tokens of its half.
         const int f = q * 32 + lane;
@@ -873,7 +882,7 @@ cudaError_t launch_gemm(const moe_plan_s* pl, int phases, bool dynamic, const vo
   p.H = pl->H;
   p.phases = phases;
   p.dynamic = dynamic ? 1 : 0;
-  p.swap = use_swap(pl) ? 1 : 0;
+  p.swap = use_swap(pl);
   long long max_tiles = 0;
   const bool tiled = pl->w_tiled != 0;
   constexpr bool kFp4 = kW == kWFp4;

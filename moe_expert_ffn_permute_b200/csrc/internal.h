@@ -51,7 +51,7 @@ struct moe_plan_s {
 namespace moe {
 
 void compute_layout(moe_plan_s* p);
-bool use_swap(const moe_plan_s* p);   // token-major (swap-AB) MMAs in the GEMM
+int use_swap(const moe_plan_s* p);    // token-major (swap-AB) MMAs: 0 never, 1 all, 2 by tile
 
 // Launch with programmatic stream serialization: the kernel may start while its
 // predecessor in the stream finishes; it must execute griddep_wait() before

@@ -166,26 +166,23 @@ def test_bf16_plans_take_no_scales_and_tiled_weights():
 
 
 def test_swap_ab_selection():
-    """Token-major tiles: automatic at <= 64 slots per expert on average (any
-    weight format), never with CTA pairs, forced on or off by the mode."""
-    p = moe.moe_plan(128, 7168, 2048, 32, 8)            # 1024 slots, 32 experts
-    assert moe.moe_plan_swap_ab_active(p)
+    """Token-major tiles: tile by tile in automatic mode (any weight format),
+    forced on or off by the mode, never with CTA pairs."""
+    p = moe.moe_plan(128, 7168, 2048, 32, 8)
+    assert moe.moe_plan_swap_ab_active(p) == 2
     moe.moe_plan_set_swap_ab(p, 1)
-    assert not moe.moe_plan_swap_ab_active(p)
+    assert moe.moe_plan_swap_ab_active(p) == 0
     moe.moe_plan_set_weight_layout(p, True)
     moe.moe_plan_set_swap_ab(p, 2)
-    assert moe.moe_plan_swap_ab_active(p)
+    assert moe.moe_plan_swap_ab_active(p) == 1
     moe.moe_plan_set_cta_pairs(p, 2)                    # pairs take precedence
-    assert not moe.moe_plan_swap_ab_active(p)
-    moe.moe_plan_destroy(p)
-    q = moe.moe_plan(8192, 7168, 2048, 32, 8)           # 65536 slots: token-row tiles
-    assert not moe.moe_plan_swap_ab_active(q)
+    assert moe.moe_plan_swap_ab_active(p) == 0
     with pytest.raises(moe.MoEError) as ei:
-        moe.moe_plan_set_swap_ab(q, 3)
+        moe.moe_plan_set_swap_ab(p, 3)
     assert ei.value.status == 1
-    moe.moe_plan_destroy(q)
-    b = moe.moe_plan(128, 512, 256, 8, 2, w_dtype="bf16")   # 256 slots, 8 experts: 32 each
-    assert moe.moe_plan_swap_ab_active(b)
-    moe.moe_plan_set_swap_ab(b, 1)
-    assert not moe.moe_plan_swap_ab_active(b)
+    moe.moe_plan_destroy(p)
+    b = moe.moe_plan(128, 512, 256, 8, 2, w_dtype="bf16")
+    assert moe.moe_plan_swap_ab_active(b) == 2
+    moe.moe_plan_set_swap_ab(b, 2)
+    assert moe.moe_plan_swap_ab_active(b) == 1
     moe.moe_plan_destroy(b)

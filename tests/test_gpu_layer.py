@@ -396,7 +396,7 @@ def test_token_major_tiles_match_oracle(wl):
     oracle, including experts with more than 64 and more than 128 rows."""
     d = inputs(wl)
     lay = _layer_swap(wl, 2)
-    assert moe.moe_plan_swap_ab_active(lay.plan)
+    assert moe.moe_plan_swap_ab_active(lay.plan) == 1
     out = lay.forward(d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], d["w1"],
                       d["w1_scales"], d["w2"], d["w2_scales"])
     torch.cuda.synchronize()
@@ -457,11 +457,12 @@ def test_token_major_fused_equals_separate_and_tiled_equals_row_major():
 
 
 def test_token_major_decode_full_size():
-    """The decode layer (T=128, E=32, k=8) picks swap-AB tiles automatically."""
+    """The decode layer (T=128, E=32, k=8) in automatic mode: token-major tiles
+    wherever an expert's tile holds at most 96 tokens."""
     wl = WORKLOADS["decode"]
     d = inputs(wl)
     lay = _layer_swap(wl, None, tiled=True)
-    assert moe.moe_plan_swap_ab_active(lay.plan)
+    assert moe.moe_plan_swap_ab_active(lay.plan) == 2
     w1, w2 = lay.prepack(d["w1"], d["w2"])
     out = lay.forward(d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], w1, d["w1_scales"],
                       w2, d["w2_scales"])
