@@ -471,3 +471,31 @@ def test_token_major_decode_full_size():
     tokens = np.sort(np.random.default_rng(4).choice(wl.T, size=8, replace=False))
     ref = oracle_tokens(wl, to_numpy(d), tokens)
     assert_parity(out.float().cpu().numpy()[tokens], ref, "decode swap")
+
+
+
+@pytest.mark.parametrize("swap", [1, 2], ids=["token-rows", "swap-ab"])
+def test_tokens_without_routed_slots_get_zero_rows(swap):
+    """A token whose slots are all masked or invalid gets a zero row (no FC2
+    row reaches it); moe_forward equals the step calls byte for byte and the
+    oracle within tolerance, with either tile orientation."""
+    wl = RAGGED
+    d = inputs(wl)
+    d["topk_idx"][3, :] = -1
+    d["topk_idx"][10, :] = wl.E + 5
+    d["topk_idx"][11, 1:] = -1
+    lay = _layer_swap(wl, swap)
+    out = torch.full((wl.T, wl.H), 7.0, dtype=torch.bfloat16, device="cuda")
+    moe.moe_forward(lay.plan, d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], d["w1"],
+                    d["w1_scales"], d["w2"], d["w2_scales"], out, lay.workspace)
+    torch.cuda.synchronize()
+    assert lay.check() == 6
+    assert not out[3].any() and not out[10].any()
+    sep = torch.full_like(out, 7.0)
+    moe.moe_route_gather(lay.plan, d["topk_idx"], d["x"], d["x_scales"], lay.workspace)
+    moe.moe_fc1_fc2(lay.plan, d["w1"], d["w1_scales"], d["w2"], d["w2_scales"], lay.workspace)
+    moe.moe_combine(lay.plan, d["topk_w"], sep, lay.workspace)
+    torch.cuda.synchronize()
+    assert torch.equal(out, sep)
+    ref = L.layer(*oracle_args(to_numpy(d)), **oracle_kw(wl))
+    assert_parity(out.float().cpu().numpy(), ref, "zero rows")
