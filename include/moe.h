@@ -321,9 +321,14 @@ moe_status moe_prepack_weights(moe_plan_t plan, const void *w1, const void *w2,
 moe_status moe_copy_act(moe_plan_t plan, const void *workspace, uint8_t *dst,
                         moe_stream_t stream);
 
-/* Debug capture: when on, moe_fc1 also writes the fp32 activation before
- * requantisation to act_f32 (costs bandwidth; off by default).              */
-moe_status moe_plan_set_debug(moe_plan_t plan, int capture_act_f32);
+/* Debug flags (0 by default).  Bit 0: FC1 also writes the fp32 activation
+ * before requantisation to act_f32 (costs bandwidth).  Bit 1: test hook for
+ * the failure path -- in the fused FC1+FC2 launch (moe_fc1_fc2, moe_forward
+ * without CTA pairs) every FC2 tile waits for one FC1 completion more than its
+ * m-tile can provide, so that bounded wait runs out (about 2 s): the launch
+ * stops, the error word gets MOE_ERR_DEVICE_TIMEOUT, nothing traps or hangs,
+ * and the output is undefined.  Other bits: MOE_ERR_INVALID_ARG.            */
+moe_status moe_plan_set_debug(moe_plan_t plan, int flags);
 
 /* Zero the workspace's device error word (enqueued on `stream`). */
 moe_status moe_clear_device_error(moe_plan_t plan, void *workspace,

@@ -144,8 +144,10 @@ def moe_workspace_bytes(plan):
     return lib().moe_workspace_bytes(plan)
 
 
-def moe_plan_set_debug(plan, capture_act_f32):
-    _check(lib().moe_plan_set_debug(plan, int(bool(capture_act_f32))), "moe_plan_set_debug")
+def moe_plan_set_debug(plan, flags):
+    """Bit 0 (or True): capture the fp32 FC1 activation; bit 1: the failure-path
+    test hook (the fused launch's FC2 dependency wait runs out)."""
+    _check(lib().moe_plan_set_debug(plan, int(flags)), "moe_plan_set_debug")
 
 
 def moe_forward(plan, x, x_scales, topk_idx, topk_w, w1, w1_scales, w2, w2_scales, out,

@@ -140,6 +140,7 @@ moe_status moe_plan(int T, int H, int I, int E, int k, moe_dtypes dtypes, moe_ac
   p->w_dtype = dtypes.w_dtype;
   p->act = act;
   p->debug_act_f32 = 0;
+  p->debug_fault = 0;
   p->w_tiled = 0;
   p->pair_mode = 0;
   p->swap_mode = 0;
@@ -202,9 +203,11 @@ moe_status moe_copy_act(moe_plan_t plan, const void* workspace, uint8_t* dst,
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
-moe_status moe_plan_set_debug(moe_plan_t plan, int capture_act_f32) {
+moe_status moe_plan_set_debug(moe_plan_t plan, int flags) {
   if (plan == nullptr) return MOE_ERR_INVALID_ARG;
-  plan->debug_act_f32 = capture_act_f32 ? 1 : 0;
+  if (flags & ~3) return MOE_ERR_INVALID_ARG;
+  plan->debug_act_f32 = flags & 1;
+  plan->debug_fault = (flags >> 1) & 1;
   moe::compute_layout(plan);
   return MOE_OK;
 }

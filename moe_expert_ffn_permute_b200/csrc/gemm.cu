@@ -75,6 +75,7 @@ struct __align__(1024) Smem {
   int task_pos[SCHED_DEPTH];       // position (unpadded) of the tile's first row
   float amax[2][2][BM];            // [tile parity][half][row]
   float swap_red[2][4][64];        // token-major FC1: per-warp amax [half][sub-partition][token]
+  uint64_t swap_bar[2];            // token-major FC1: the four warps of a half (bounded waits)
   float swap_inv[2][64];           // token-major FC1: 1 / 2^n per token [half][token]
   uint32_t tmem_base;
   int abort_flag;
@@ -99,6 +100,7 @@ struct Params {
   int dynamic;               // tiles from a global counter (else round-robin)
   int swap;                  // token-major MMAs (weights as A, the tile's tokens as B):
                              // 0 never, 1 always, 2 for tiles of at most kSwapRows rows
+  int dep_extra;             // test hook: FC2 waits for this many FC1 completions more
   Phase ph[2];
   const int32_t* tile_off;
   const int32_t* counts;
@@ -219,6 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.sched_empty[r], kSchedConsumers);
     }
     for (int q = 0; q < 4; ++q) mbar_init(&sm.pair[q], 2);
+    for (int h = 0; h < 2; ++h) mbar_init(&sm.swap_bar[h], 4);
     sm.abort_flag = 0;
     fence_mbarrier_init();
     if ((p.phases & 1) && p.ph[0].w_tiles == nullptr) tma_prefetch_desc(&tmap_b1);
@@ -301,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t pol_b_once = l2_policy_evict_first();
     const uint64_t pol_b_reused = l2_policy_evict_normal();
     const uint32_t ab_bytes = BM * BK + (kFp4 ? BN * BK / 2 : BN * BK);
-    const uint32_t fc1_target = static_cast<uint32_t>(kEpiWarps * p.ph[0].n_tiles);
+    const uint32_t fc1_target = static_cast<uint32_t>(kEpiWarps * p.ph[0].n_tiles + p.dep_extra);
     Task t;
     bool aborted = false;
     while (!aborted && get_task(sm, slot, sphase, t, p.err)) {
@@ -521,9 +524,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = q * 32 + lane;
     const uint32_t t_row = tmem + (static_cast<uint32_t>(q * 32) << 16);
     int slot = 0;
-    uint32_t sphase = 0, acc_phase = 0, pair_phase = 0;
+    uint32_t sphase = 0, acc_phase = 0, pair_phase = 0, swap_phase = 0;
     int tile_par = 0;
     Task t;
+    // Token-major FC1: the four warps of this half meet on an mbarrier (a
+    // bounded wait, so an aborting CTA cannot leave a warp waiting forever).
+    auto half_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.swap_bar[half]);
+      const bool ok = mbar_wait(&sm.swap_bar[half], swap_phase, p.err, &sm.abort_flag);
+      swap_phase ^= 1u;
+      return ok;
+    };
     while (get_task(sm, slot, sphase, t, p.err)) {
       if (t.e < 0) break;
       if (!mbar_wait(&sm.tmem_full, acc_phase, p.err, &sm.abort_flag)) break;
@@ -607,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 sm.swap_red[half][q][32 * r + lane] = m[0];
               }
             }
-            named_barrier_sync(1 + half, 128);
+            if (!half_sync()) break;
             const int nb = p.I / 128;
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
@@ -625,7 +637,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
               }
             }
-            named_barrier_sync(1 + half, 128);
+            if (!half_sync()) break;
             uint8_t* tile = p.act + (static_cast<size_t>(t.mt) * nb + t.nt) * kTileBytes;
 #pragma unroll
             for (int j = 0; j < 64; ++j) {
@@ -883,6 +895,7 @@ cudaError_t launch_gemm(const moe_plan_s* pl, int phases, bool dynamic, const vo
   p.phases = phases;
   p.dynamic = dynamic ? 1 : 0;
   p.swap = use_swap(pl);
+  p.dep_extra = pl->debug_fault ? 1 : 0;
   long long max_tiles = 0;
   const bool tiled = pl->w_tiled != 0;
   constexpr bool kFp4 = kW == kWFp4;

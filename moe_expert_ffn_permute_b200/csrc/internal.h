@@ -39,6 +39,7 @@ struct moe_plan_s {
   int w_dtype;
   moe_act_params act;
   int debug_act_f32;
+  int debug_fault;       // test hook: the fused GEMM's FC2 dependency can never be met
   int w_tiled;           // weights given as pre-swizzled tiles (moe_prepack_weights)
   int pair_mode;         // 2-SM GEMM: 0 automatic, 1 never, 2 always
   int swap_mode;         // token-major MMAs: 0 automatic, 1 never, 2 always

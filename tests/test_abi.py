@@ -186,3 +186,16 @@ def test_swap_ab_selection():
     moe.moe_plan_set_swap_ab(b, 2)
     assert moe.moe_plan_swap_ab_active(b) == 1
     moe.moe_plan_destroy(b)
+
+
+def test_debug_flags():
+    p = moe.moe_plan(64, 512, 256, 8, 2)
+    a = moe.moe_workspace_bytes(p)
+    moe.moe_plan_set_debug(p, 2)                 # failure-path hook only: no capture buffer
+    assert moe.moe_workspace_bytes(p) == a
+    moe.moe_plan_set_debug(p, 3)
+    assert moe.moe_workspace_bytes(p) > a
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_plan_set_debug(p, 4)
+    assert ei.value.status == 1
+    moe.moe_plan_destroy(p)
