@@ -61,10 +61,11 @@ class Clocks:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix=f"moe_clocks_gpu{gpu_index}_", suffix=".csv")
+        os.close(fd)
 
     def start(self):
-        os.makedirs(os.path.dirname(self.path), exist_ok=True)
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
@@ -97,11 +98,15 @@ class Clocks:
             for name, val in zip(names, parts[5:9]):
                 if val.lower() == "active":
                     reasons.add(name)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None,
                 "reasons": sorted(reasons), "samples": len(sm),
-                "window": "continuous steps of the same layer, 0.6 s before and after "
-                          "the timed steps"}
+                "window": "continuous steps of the same layer around the timed steps, the "
+                          "eager steps and the per-kernel split"}
 
 
 KERNEL_SOURCES = ("moe_expert_ffn_permute_b200/csrc/gemm.cu",
