@@ -194,14 +194,18 @@ def run_b200(args, wl):
     # FP8 weights are rearranged once into the tensor-core tile layout (as at
     # model load); the timed steps read them in that layout.
     tiled = wl.w_dtype in ("e4m3", "bf16") and not args.row_major_weights
+    chunked = wl.w_dtype == "e2m1" and not args.row_major_weights
     lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype=wl.w_dtype, act=wl.act,
                        alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit, device=dev,
                        tiled_weights=tiled, cta_pairs=args.cta_pairs if tiled else None,
-                       swap_ab=args.swap_ab)
+                       swap_ab=args.swap_ab, chunked_scales=chunked)
     pairs = moe.moe_plan_cta_pairs_active(lay.plan)
     d_row_major = dict(d)          # the oracle reads the original layout
     if tiled:
         d["w1"], d["w2"] = lay.prepack(d["w1"], d["w2"])
+        torch.cuda.synchronize()
+    if chunked:
+        d["w1_scales"], d["w2_scales"] = lay.prepack_scales(d["w1_scales"], d["w2_scales"])
         torch.cuda.synchronize()
     out = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
@@ -373,7 +377,9 @@ def run_b200(args, wl):
         "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
                    "w_dtype": wl.w_dtype, "routing": wl.routing, "act": wl.act,
                    "active_experts": active, "l2": "flushed (256 MiB write) before each step",
-                   "weights": "tiled (moe_prepack_weights, once)" if tiled else "row-major",
+                   "weights": ("tiled (moe_prepack_weights, once)" if tiled else
+                               "row-major codes, chunked scales (moe_prepack_weight_scales, once)"
+                               if chunked else "row-major"),
                    "gemm_tiles": {0: "token rows", 1: "token-major (swap AB)",
                                   2: "token-major for tiles of <= 96 tokens, else token rows"}[
                        moe.moe_plan_swap_ab_active(lay.plan)],
@@ -489,7 +495,8 @@ def main():
     ap.add_argument("--swap-ab", type=int, default=0, choices=[0, 1, 2],
                     help="token-major GEMM tiles: 0 tile by tile (automatic), 1 never, 2 always")
     ap.add_argument("--row-major-weights", action="store_true",
-                    help="read FP8 weights row-major via 2-D TMA instead of prepacked tiles")
+                    help="weights as given (row-major, 2-D TMA; MXFP4 scales unchunked) "
+                         "instead of prepacked")
     args = ap.parse_args()
     from moe_expert_ffn_permute_b200.synth import WORKLOADS
     wl = WORKLOADS[args.workload]

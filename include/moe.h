@@ -269,8 +269,29 @@ moe_status moe_copy_act_scales(moe_plan_t plan, const void *workspace,
  * tiles that the tensor cores consume directly, streamed by linear bulk copies
  * (faster; FP8 and BF16 weights, MOE_ERR_UNSUPPORTED for MXFP4).  Weight
  * scales keep their layout in both cases.                                   */
-typedef enum { MOE_WEIGHTS_ROW_MAJOR = 0, MOE_WEIGHTS_TILED = 1 } moe_weight_layout;
+typedef enum {
+  MOE_WEIGHTS_ROW_MAJOR = 0,
+  MOE_WEIGHTS_TILED = 1,
+  /* MXFP4 only: the E2M1 codes stay row-major (read by TMA, which widens them),
+   * w1_scales / w2_scales are the output of moe_prepack_weight_scales(),
+   * 16-byte aligned.                                                          */
+  MOE_WEIGHTS_SCALES_CHUNKED = 2
+} moe_weight_layout;
 moe_status moe_plan_set_weight_layout(moe_plan_t plan, int layout);
+
+/* Rearrange MXFP4 weight scales w1_scales u8 [E,2I,H/32] and w2_scales u8
+ * [E,H,I/32] (device, 4-byte aligned) into 512-byte chunks (outputs: device
+ * buffers of the same sizes, 16-byte aligned, not overlapping the inputs):
+ * with K the row length (H, or I) and rows counted across experts, the chunk
+ * of row block b (rows 128b..128b+127) and k-block kb (elements 128kb..+127) is
+ * at (b * K/128 + kb) * 512 and holds row r's four scale bytes at
+ * (r % 32) * 16 + (r / 32) * 4 -- the layout the tensor core's scale copy
+ * reads, so a pipeline stage needs two contiguous 512-byte copies instead of
+ * 256 scattered 4-byte reads.  Done once per weight set, on `stream`.
+ * MOE_ERR_UNSUPPORTED for other weight formats.                             */
+moe_status moe_prepack_weight_scales(moe_plan_t plan, const uint8_t *w1_scales,
+                                     const uint8_t *w2_scales, uint8_t *w1_scales_chunked,
+                                     uint8_t *w2_scales_chunked, moe_stream_t stream);
 
 /* GEMM variant for moe_fc1_fc2 / moe_forward.  With tiled FP8 weights the two
  * GEMMs can run on CTA pairs with the 2-SM tensor-core MMA (each pair computes

@@ -69,6 +69,7 @@ _SIGS = {
     "moe_plan_set_cta_pairs": (ctypes.c_int, [_P, ctypes.c_int]),
     "moe_plan_cta_pairs_active": (ctypes.c_int, [_P]),
     "moe_plan_set_swap_ab": (ctypes.c_int, [_P, ctypes.c_int]),
+    "moe_prepack_weight_scales": (ctypes.c_int, [_P] * 6),
     "moe_plan_swap_ab_active": (ctypes.c_int, [_P]),
     "moe_prepack_weights": (ctypes.c_int, [_P] * 6),
     "moe_copy_act": (ctypes.c_int, [_P] * 4),
@@ -228,8 +229,15 @@ def moe_copy_act_scales(plan, workspace, dst, stream=None):
            "moe_copy_act_scales")
 
 
-def moe_plan_set_weight_layout(plan, tiled):
-    _check(lib().moe_plan_set_weight_layout(plan, 1 if tiled else 0), "moe_plan_set_weight_layout")
+def moe_plan_set_weight_layout(plan, layout):
+    """0 / False: row-major, 1 / True: tiled (FP8, BF16), 2: MXFP4 scales chunked."""
+    _check(lib().moe_plan_set_weight_layout(plan, int(layout)), "moe_plan_set_weight_layout")
+
+
+def moe_prepack_weight_scales(plan, w1_scales, w2_scales, w1s_chunked, w2s_chunked, stream=None):
+    _check(lib().moe_prepack_weight_scales(plan, *map(_ptr, (w1_scales, w2_scales, w1s_chunked,
+                                                              w2s_chunked)), _stream(stream)),
+           "moe_prepack_weight_scales")
 
 
 def moe_plan_set_cta_pairs(plan, mode):
@@ -283,12 +291,14 @@ class MoELayer:
 
     def __init__(self, T, H, I, E, k, w_dtype="e4m3", act="swiglu", alpha=1.0, up_bias=0.0,
                  limit=math.inf, device="cuda", debug=False, tiled_weights=False,
-                 cta_pairs=None, swap_ab=None):
+                 cta_pairs=None, swap_ab=None, chunked_scales=False):
         import torch
         self.T, self.H, self.I, self.E, self.k = T, H, I, E, k
         self.plan = moe_plan(T, H, I, E, k, w_dtype, act, alpha, up_bias, limit)
         if tiled_weights:
-            moe_plan_set_weight_layout(self.plan, True)
+            moe_plan_set_weight_layout(self.plan, 1)
+        if chunked_scales:
+            moe_plan_set_weight_layout(self.plan, 2)
         if cta_pairs is not None:
             moe_plan_set_cta_pairs(self.plan, cta_pairs)
         if swap_ab is not None:
@@ -314,6 +324,13 @@ class MoELayer:
         w1t, w2t = torch.empty_like(w1), torch.empty_like(w2)
         moe_prepack_weights(self.plan, w1, w2, w1t, w2t)
         return w1t, w2t
+
+    def prepack_scales(self, w1_scales, w2_scales):
+        """Chunked copies of MXFP4 weight scales for a plan with chunked_scales."""
+        import torch
+        a, b = torch.empty_like(w1_scales), torch.empty_like(w2_scales)
+        moe_prepack_weight_scales(self.plan, w1_scales, w2_scales, a, b)
+        return a, b
 
     def view(self):
         return moe_workspace_view(self.plan, self.workspace)

@@ -102,7 +102,8 @@ static moe_status check_weights(moe_plan_t plan, const void* w, const uint8_t* w
   if (ws == nullptr && plan->w_dtype != MOE_W_BF16) return MOE_ERR_INVALID_ARG;
   const size_t wa = plan->w_dtype == MOE_W_E2M1_UE8M0_1x32 ? 32 : 16;
   if (!aligned(w, wa)) return MOE_ERR_ALIGNMENT;
-  if (plan->w_dtype == MOE_W_E2M1_UE8M0_1x32 && !aligned(ws, 4)) return MOE_ERR_ALIGNMENT;
+  if (plan->w_dtype == MOE_W_E2M1_UE8M0_1x32 && !aligned(ws, plan->w_sf_chunked ? 16 : 4))
+    return MOE_ERR_ALIGNMENT;
   return MOE_OK;
 }
 
@@ -142,6 +143,7 @@ moe_status moe_plan(int T, int H, int I, int E, int k, moe_dtypes dtypes, moe_ac
   p->debug_act_f32 = 0;
   p->debug_fault = 0;
   p->w_tiled = 0;
+  p->w_sf_chunked = 0;
   p->pair_mode = 0;
   p->swap_mode = 0;
   p->S = static_cast<long long>(T) * k;
@@ -160,11 +162,34 @@ size_t moe_workspace_bytes(moe_plan_t plan) { return plan ? plan->ws.total : 0; 
 
 moe_status moe_plan_set_weight_layout(moe_plan_t plan, int layout) {
   if (plan == nullptr) return MOE_ERR_INVALID_ARG;
-  if (layout != MOE_WEIGHTS_ROW_MAJOR && layout != MOE_WEIGHTS_TILED) return MOE_ERR_INVALID_ARG;
-  if (layout == MOE_WEIGHTS_TILED && plan->w_dtype == MOE_W_E2M1_UE8M0_1x32)
-    return MOE_ERR_UNSUPPORTED;
+  if (layout != MOE_WEIGHTS_ROW_MAJOR && layout != MOE_WEIGHTS_TILED &&
+      layout != MOE_WEIGHTS_SCALES_CHUNKED)
+    return MOE_ERR_INVALID_ARG;
+  const bool fp4 = plan->w_dtype == MOE_W_E2M1_UE8M0_1x32;
+  if (layout == MOE_WEIGHTS_TILED && fp4) return MOE_ERR_UNSUPPORTED;
+  if (layout == MOE_WEIGHTS_SCALES_CHUNKED && !fp4) return MOE_ERR_UNSUPPORTED;
   plan->w_tiled = layout == MOE_WEIGHTS_TILED ? 1 : 0;
+  plan->w_sf_chunked = layout == MOE_WEIGHTS_SCALES_CHUNKED ? 1 : 0;
   return MOE_OK;
+}
+
+moe_status moe_prepack_weight_scales(moe_plan_t plan, const uint8_t* w1_scales,
+                                     const uint8_t* w2_scales, uint8_t* w1_scales_chunked,
+                                     uint8_t* w2_scales_chunked, moe_stream_t stream) {
+  if (plan == nullptr || w1_scales == nullptr || w2_scales == nullptr ||
+      w1_scales_chunked == nullptr || w2_scales_chunked == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (plan->w_dtype != MOE_W_E2M1_UE8M0_1x32) return MOE_ERR_UNSUPPORTED;
+  if (!aligned(w1_scales, 4) || !aligned(w2_scales, 4) || !aligned(w1_scales_chunked, 16) ||
+      !aligned(w2_scales_chunked, 16))
+    return MOE_ERR_ALIGNMENT;
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  const long long E = plan->E;
+  if (moe::launch_prepack_fp4_scales(w1_scales, E * 2 * plan->I, plan->H, w1_scales_chunked,
+                                     st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return cuda_status(
+      moe::launch_prepack_fp4_scales(w2_scales, E * plan->H, plan->I, w2_scales_chunked, st));
 }
 
 moe_status moe_plan_set_cta_pairs(moe_plan_t plan, int mode) {

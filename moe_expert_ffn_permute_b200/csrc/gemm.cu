@@ -101,6 +101,7 @@ struct Params {
   int swap;                  // token-major MMAs (weights as A, the tile's tokens as B):
                              // 0 never, 1 always, 2 for tiles of at most kSwapRows rows
   int dep_extra;             // test hook: FC2 waits for this many FC1 completions more
+  int sf_chunked;            // MXFP4 weight scales prepacked into 512-byte chunks
   Phase ph[2];
   const int32_t* tile_off;
   const int32_t* counts;
@@ -392,7 +393,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                       ph.sfa_chunks + (static_cast<size_t>(t.mt) * ph.k_blocks + kb) * 512, 512,
                       &sm.full[stage]);
           }
-          if (kFp4) {
+          if (kFp4 && p.sf_chunked) {
+            // Prepacked scales: the stage's two 512-byte chunks (128 weight rows
+            // each) are contiguous, so two bulk copies replace 256 scattered
+            // 4-byte reads.
+            if (lane == 0) {
+              mbar_expect_tx(&sm.full[stage], 1024);
+              bulk_load(sm.sfb[stage],
+                        ph.w_sf + (static_cast<size_t>(brow0 / 128) * ph.k_blocks + kb) * 512,
+                        512, &sm.full[stage]);
+              bulk_load(sm.sfb[stage] + 512,
+                        ph.w_sf + (static_cast<size_t>(brow1 / 128) * ph.k_blocks + kb) * 512,
+                        512, &sm.full[stage]);
+            }
+            __syncwarp();
+            mbar_arrive(&sm.full[stage]);
+          } else if (kFp4) {
             // One 32-bit word = the four 1x32 scales of this 128-wide k-block.
             const int kw = ph.k_blocks * 4;   // scale bytes per weight row
 #pragma unroll
@@ -896,6 +912,7 @@ cudaError_t launch_gemm(const moe_plan_s* pl, int phases, bool dynamic, const vo
   p.dynamic = dynamic ? 1 : 0;
   p.swap = use_swap(pl);
   p.dep_extra = pl->debug_fault ? 1 : 0;
+  p.sf_chunked = pl->w_sf_chunked;
   long long max_tiles = 0;
   const bool tiled = pl->w_tiled != 0;
   constexpr bool kFp4 = kW == kWFp4;

@@ -41,6 +41,7 @@ struct moe_plan_s {
   int debug_act_f32;
   int debug_fault;       // test hook: the fused GEMM's FC2 dependency can never be met
   int w_tiled;           // weights given as pre-swizzled tiles (moe_prepack_weights)
+  int w_sf_chunked;      // MXFP4 scales given in 512-byte chunks (moe_prepack_weight_scales)
   int pair_mode;         // 2-SM GEMM: 0 automatic, 1 never, 2 always
   int swap_mode;         // token-major MMAs: 0 automatic, 1 never, 2 always
   long long S;           // T*k
@@ -80,6 +81,9 @@ cudaError_t launch_route(const moe_plan_s* p, const int32_t* topk_idx, uint8_t* 
 constexpr int kFusedMaxSlots = 4096;
 cudaError_t launch_route_gather(const moe_plan_s* p, const int32_t* topk_idx, const uint8_t* x,
                                 const uint8_t* xs, uint8_t* ws, cudaStream_t st);
+// MXFP4 weight scales [rows, K/32] -> 512-byte tensor-core chunks.
+cudaError_t launch_prepack_fp4_scales(const uint8_t* src, long long rows, int K, uint8_t* dst,
+                                      cudaStream_t st);
 cudaError_t launch_gather(const moe_plan_s* p, const uint8_t* x, const uint8_t* xs, uint8_t* ws,
                           cudaStream_t st);
 cudaError_t launch_fc1(const moe_plan_s* p, const void* w1, const uint8_t* w1s, uint8_t* ws,

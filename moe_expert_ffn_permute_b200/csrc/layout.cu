@@ -45,6 +45,24 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__
   }
 }
 
+// MXFP4 weight scales [rows, K/32] (four bytes per row per 128-wide k-block)
+// -> chunks: for row block b and k-block kb, 512 bytes at (b * K/128 + kb) * 512
+// holding row r's four bytes at (r % 32) * 16 + (r / 32) * 4 -- the layout the
+// tensor core's scale copy (32x128b.warpx4) reads.  One thread per 4-byte word.
+__global__ void __launch_bounds__(256) prepack_fp4_scales_kernel(
+    const uint32_t* __restrict__ src, long long rows, int kb_n, uint8_t* __restrict__ dst) {
+  const long long n = rows * kb_n;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long row = i / kb_n;
+    const int kb = static_cast<int>(i - row * kb_n);
+    const long long b = row / 128;
+    const int r = static_cast<int>(row - b * 128);
+    *reinterpret_cast<uint32_t*>(dst + (b * kb_n + kb) * 512 + (r & 31) * 16 + (r >> 5) * 4) =
+        __ldg(&src[i]);
+  }
+}
+
 int blocks_for(long long n) {
   const long long b = (n + 255) / 256;
   return static_cast<int>(b < 148 * 16 ? b : 148 * 16);
@@ -56,6 +74,14 @@ cudaError_t launch_prepack(const uint8_t* src, long long rows, int K, uint8_t* d
                            cudaStream_t st) {
   const long long n = rows * (K / 16);
   prepack_kernel<<<blocks_for(n), 256, 0, st>>>(reinterpret_cast<const uint4*>(src), rows, K, dst);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prepack_fp4_scales(const uint8_t* src, long long rows, int K, uint8_t* dst,
+                                      cudaStream_t st) {
+  const int kb_n = K / 128;
+  prepack_fp4_scales_kernel<<<blocks_for(rows * kb_n), 256, 0, st>>>(
+      reinterpret_cast<const uint32_t*>(src), rows, kb_n, dst);
   return cudaGetLastError();
 }
 

@@ -199,3 +199,25 @@ def test_debug_flags():
         moe.moe_plan_set_debug(p, 4)
     assert ei.value.status == 1
     moe.moe_plan_destroy(p)
+
+
+
+def test_fp4_chunked_scale_layout_rules():
+    g = 1 << 20
+    p = moe.moe_plan(64, 512, 256, 8, 2, w_dtype="e2m1")
+    q = moe.moe_plan(64, 512, 256, 8, 2)
+    moe.moe_plan_set_weight_layout(p, 2)
+    with pytest.raises(moe.MoEError) as ei:          # chunked scales: MXFP4 only
+        moe.moe_plan_set_weight_layout(q, 2)
+    assert ei.value.status == 2
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_prepack_weight_scales(q, g, g, g, g, stream=0)
+    assert ei.value.status == 2
+    with pytest.raises(moe.MoEError) as ei:          # chunk copies need 16-byte alignment
+        moe.moe_prepack_weight_scales(p, g, g, g + 4, g, stream=0)
+    assert ei.value.status == 3
+    with pytest.raises(moe.MoEError) as ei:          # and so do the kernels' reads of them
+        moe.moe_fc2(p, g, g + 4, g, stream=0)
+    assert ei.value.status == 3
+    moe.moe_plan_destroy(p)
+    moe.moe_plan_destroy(q)

@@ -499,3 +499,53 @@ def test_tokens_without_routed_slots_get_zero_rows(swap):
     assert torch.equal(out, sep)
     ref = L.layer(*oracle_args(to_numpy(d)), **oracle_kw(wl))
     assert_parity(out.float().cpu().numpy(), ref, "zero rows")
+
+
+def test_fp4_scale_chunk_layout_matches_its_definition():
+    """moe_prepack_weight_scales: chunk (b, kb) at (b * K/128 + kb) * 512 holds
+    row r of block b's four k-block scale bytes at (r % 32) * 16 + (r / 32) * 4."""
+    wl = RAGGED_FP4
+    d = inputs(wl)
+    lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype="e2m1", chunked_scales=True)
+    c1, c2 = lay.prepack_scales(d["w1_scales"], d["w2_scales"])
+    torch.cuda.synchronize()
+    for src, got, K in ((d["w1_scales"], c1, wl.H), (d["w2_scales"], c2, wl.I)):
+        s = src.reshape(-1, K // 32).cpu().numpy()          # [rows, K/32]
+        rows, kbn = s.shape[0], K // 128
+        ref = np.zeros(rows * K // 32, dtype=np.uint8)
+        for row in range(rows):
+            b, r = divmod(row, 128)
+            for kb in range(kbn):
+                o = (b * kbn + kb) * 512 + (r % 32) * 16 + (r // 32) * 4
+                ref[o:o + 4] = s[row, 4 * kb:4 * kb + 4]
+        np.testing.assert_array_equal(got.reshape(-1).cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("swap", [1, 2], ids=["token-rows", "swap-ab"])
+def test_fp4_chunked_scales_give_the_same_bytes(swap):
+    wl = RAGGED_FP4
+    d = inputs(wl)
+    outs = []
+    for chunked in (False, True):
+        lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype="e2m1", swap_ab=swap,
+                           chunked_scales=chunked)
+        s1, s2 = (lay.prepack_scales(d["w1_scales"], d["w2_scales"]) if chunked
+                  else (d["w1_scales"], d["w2_scales"]))
+        outs.append(lay.forward(d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], d["w1"], s1,
+                                d["w2"], s2))
+        torch.cuda.synchronize()
+        assert lay.check() == 0
+    assert torch.equal(outs[0], outs[1])
+
+
+def test_fp4_chunked_scales_full_size_128_tokens():
+    wl = WORKLOADS["mxfp4"]
+    d = inputs(wl)
+    lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype="e2m1", chunked_scales=True)
+    s1, s2 = lay.prepack_scales(d["w1_scales"], d["w2_scales"])
+    out = lay.forward(d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], d["w1"], s1, d["w2"], s2)
+    torch.cuda.synchronize()
+    assert lay.check() == 0
+    tokens = np.sort(np.random.default_rng(6).choice(wl.T, size=6, replace=False))
+    ref = oracle_tokens(wl, to_numpy(d), tokens)
+    assert_parity(out.float().cpu().numpy()[tokens], ref, "mxfp4 chunked scales")
