@@ -116,12 +116,23 @@ KERNEL_SOURCES = ("moe_expert_ffn_permute_b200/csrc/gemm.cu",
                   "moe_expert_ffn_permute_b200/csrc/internal.h")
 
 
+def _strip_comments(src):
+    """C++ source without comments and blank lines (string literals in these
+    kernel sources hold no comment markers)."""
+    import re
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+
+
 def kernel_source_hash():
+    """Hash of the GEMM kernel sources' code (comments and blank lines do not
+    count), which the recorded DRAM traffic is valid for."""
     import hashlib
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            h.update(_strip_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 

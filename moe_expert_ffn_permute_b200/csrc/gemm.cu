@@ -1,23 +1,35 @@
-// gemm.cu -- FC1 and FC2 grouped GEMMs on the 5th-generation tensor cores.
+// gemm.cu -- FC1 and FC2 grouped GEMMs on the 5th-generation tensor cores, in
+// one persistent launch (FC2 tiles of an m-tile start as soon as that m-tile's
+// FC1 tiles have published their rows) or as separate launches.
 //
-// One persistent CTA per SM computes 128 x 256 output tiles of one expert:
-//   FC1: A = gathered x rows [128 x H] (E4M3), B = 128 gate rows + 128 up rows of
-//        W1[e] (E4M3 or E2M1), D = fp32 [128 x 256] in tensor memory; the
-//        epilogue applies the (OAI-)SwiGLU and requantises the 128-wide
-//        activation block to E4M3 + one UE8M0 scale per row.
-//   FC2: A = FP8 activation rows [128 x I], B = 256 rows of W2[e]; the epilogue
+// One persistent CTA per SM computes tiles of one expert.  Token-row tiles are
+// 128 tokens x 256 columns:
+//   FC1: A = gathered x rows [128 x H], B = 128 gate rows + 128 up rows of W1[e],
+//        D = fp32 [128 x 256] in tensor memory; the epilogue applies the
+//        (OAI-)SwiGLU and requantises the 128-wide activation block to E4M3 +
+//        one UE8M0 scale per row (BF16 weights: rounds it to bf16).
+//   FC2: A = activation rows [128 x I], B = 256 rows of W2[e]; the epilogue
 //        writes bf16 rows to their slot (t*k + j) for the combine.
-// Block scales (1x128 for activations, 128x128 or 1x32 for weights, all UE8M0)
-// are applied by the MMA itself (tcgen05.mma.kind::mxf8f6f4.block_scale, one
-// scale per 32-wide K sub-block; the coarser blocks are replicated).
+// Token-major ("swap AB") tiles, used for tiles with few tokens, make each
+// 128-row half of the weight tile the A operand and the tile's tokens B
+// (N = their count rounded up to 16), so the tensor work follows the tokens;
+// the epilogue then owns one feature per TMEM lane.
+// Weights: E4M3 with 128x128 or E2M1 with 1x32 UE8M0 scales, applied by the
+// MMA itself (tcgen05.mma.kind::mxf8f6f4.block_scale, one scale per 32-wide K
+// sub-block; coarser blocks are replicated), with E4M3 activations; or BF16
+// weights and activations (kind::f16, no scales).
 //
 // Warp roles (12 warps):
-//   warp 0   operand producer: bulk copies of the A/B tiles
-//   warp 1   MMA issuer; owns the tensor-memory allocation
+//   warp 0   operand producer: bulk copies of pre-swizzled A/B tiles (2-D TMA
+//            for row-major and MXFP4 weights)
+//   warp 1   MMA issuer (one lane); owns the tensor-memory allocation
 //   warp 2   tile scheduler: writes task infos into a ring of shared-memory slots
-//   warp 3   scale-factor producer: A scale chunks (bulk copy), B scales
-//            (shared-memory stores or cp.async)
+//   warp 3   scale-factor producer: A scale chunks and prepacked MXFP4 scale
+//            chunks (bulk copies), FP8 B scales (shared-memory stores) or
+//            unchunked MXFP4 scales (cp.async)
 //   warps 4-11 epilogue: two warps per 32-lane TMEM sub-partition
+// Every wait is bounded (mbarrier waits and the FC1->FC2 dependency): on expiry
+// the error word gets MOE_ERR_DEVICE_TIMEOUT and the CTA winds down.
 //
 // Scheduler slot release (fw-ai/DeepGEMM PR #16 "Sync upstream through PR #441:
 // fix Mega MoE scheduler ordering", Overview): a consumer copies the task info
@@ -27,7 +39,8 @@
 //
 // Activation (DeepGEMM PR #445 "fix(sm90): support parameterized SwiGLU in FP8
 // MegaMoE", Summary): gate = min(gate, limit), up = clamp(up, -limit, limit),
-// a = gate * sigmoid(alpha * gate) * (up + up_bias).
+// a = gate * sigmoid(alpha * gate) * (up + up_bias); its swapAB variant (the
+// same PR's calc_diff table) for the token-major tiles.
 // Requantisation (TensorRT-LLM PR #16346 "DSV4 o_proj: fuse fp8/UE8M0 quantize
 // ...", Description): per 1x128 block, amax -> UE8M0 exponent -> E4M3 codes,
 // done in the producing GEMM's epilogue.
