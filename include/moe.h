@@ -10,6 +10,10 @@
  *   y[t,j]  = (q * sq) @ W2[e]^T,  W2[e] = [H, I]
  *   out[t]  = bf16( sum_j topk_w[t,j] * y[t,j] )     (fp32 sum, j ascending)
  *
+ * with W1, W2 in E4M3 (128x128 UE8M0 blocks) or E2M1 (1x32 UE8M0 blocks).  The
+ * BF16 variant (MOE_W_BF16) takes bf16 x and weights without scales and passes
+ * a to FC2 rounded to bf16 instead of q * sq.
+ *
  * Sources (web pages, by title and section):
  *   - DeepGEMM PR #445 "fix(sm90): support parameterized SwiGLU in FP8 MegaMoE",
  *     Summary / Compatibility: the activation and its parameters (defaults
@@ -19,14 +23,17 @@
  *     scales consumed natively and the direct weighted combine to token order.
  *   - fw-ai/DeepGEMM PR #16 "Sync upstream through PR #441: fix Mega MoE
  *     scheduler ordering", Overview: the persistent tile scheduler's task-info
- *     slots and their release ordering (used inside moe_fc1 / moe_fc2).
+ *     slots and their release ordering (used inside moe_fc1 / moe_fc2 /
+ *     moe_fc1_fc2), and the BF16 / FP8 / FP4 Mega MoE variants.
  *   - TensorRT-LLM PR #16346 "DSV4 o_proj: fuse fp8/UE8M0 quantize ...",
  *     Description: BF16/FP32 -> FP8 + 1x128 UE8M0 quantisation fused into a
  *     GEMM epilogue (the FC1 epilogue here).
  *
  * Conventions for every entry point:
- *   - All tensors are row-major and contiguous; all device pointers must be
- *     16-byte aligned (MXFP4 weight pointers 32-byte aligned).
+ *   - Tensors are row-major and contiguous unless a layout call says otherwise
+ *     (moe_plan_set_weight_layout); device pointers must be 16-byte aligned
+ *     (MXFP4 weight codes 32-byte, their scales 4-byte, or 16-byte when
+ *     chunked).
  *   - Ownership: the caller owns every buffer, host or device.  The library
  *     never allocates or frees device memory; a plan is a small host object.
  *   - Errors are returned as moe_status; nothing is thrown across the ABI.

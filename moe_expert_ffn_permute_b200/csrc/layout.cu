@@ -1,7 +1,8 @@
-// layout.cu -- conversions between row-major operands and the pre-swizzled
-// tile layout the grouped GEMMs stream with linear bulk copies: a 128-row x
-// 128-byte tile is 16 KB, tiles ordered [row block][k-block], and byte c of
-// row r sits at r * 128 + (((c / 16) ^ (r % 8)) * 16) + c % 16.
+// layout.cu -- conversions between row-major operands and the layouts the
+// grouped GEMMs stream with linear bulk copies: pre-swizzled tiles (a 128-row x
+// 128-byte tile is 16 KB, tiles ordered [row block][k-block], and byte c of row
+// r sits at r * 128 + (((c / 16) ^ (r % 8)) * 16) + c % 16), and MXFP4 weight
+// scales in the tensor core's 512-byte scale chunks.
 #include <cuda_runtime.h>
 
 #include "internal.h"

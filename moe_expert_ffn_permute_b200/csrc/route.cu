@@ -1,4 +1,5 @@
-// route.cu -- step 1 (routing) and the FC1 operand gather.
+// route.cu -- step 1 (routing) and the FC1 operand gather, as separate launches
+// or, for up to 4096 slots, as one (route_gather_kernel).
 //
 // Routing groups the T*k slots (slot s = t*k + j holds expert topk_idx[t, j]) by
 // expert: a per-expert histogram, an exclusive scan, and a stable scatter that
