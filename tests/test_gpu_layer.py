@@ -549,3 +549,23 @@ def test_fp4_chunked_scales_full_size_128_tokens():
     tokens = np.sort(np.random.default_rng(6).choice(wl.T, size=6, replace=False))
     ref = oracle_tokens(wl, to_numpy(d), tokens)
     assert_parity(out.float().cpu().numpy()[tokens], ref, "mxfp4 chunked scales")
+
+
+def test_token_rows_are_independent_of_the_batch():
+    """With token-row tiles a token's output does not depend on the other tokens
+    of the batch: the layer on a subset of tokens gives those tokens' rows of
+    the full run byte for byte."""
+    wl = RAGGED
+    d = inputs(wl)
+    full = _layer_swap(wl, 1)
+    out_full = full.forward(d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], d["w1"],
+                            d["w1_scales"], d["w2"], d["w2_scales"])
+    tokens = torch.arange(5, wl.T, 7, device="cuda")
+    sub = Workload("ragged-subset", int(tokens.numel()), wl.H, wl.I, wl.E, wl.k, cfg_id=20)
+    part = _layer_swap(sub, 1)
+    out_part = part.forward(d["x"][tokens].contiguous(), d["x_scales"][tokens].contiguous(),
+                            d["topk_idx"][tokens].contiguous(), d["topk_w"][tokens].contiguous(),
+                            d["w1"], d["w1_scales"], d["w2"], d["w2_scales"])
+    torch.cuda.synchronize()
+    assert full.check() == 0 and part.check() == 0
+    assert torch.equal(out_part, out_full[tokens])
