@@ -326,6 +326,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Phase& ph = p.ph[t.kind];
       const uint64_t pol_b = t.reuse ? pol_b_reused : pol_b_once;
       const CUtensorMap* tb = t.kind ? &tmap_b2 : &tmap_b1;
+      // A token-major tile's MMAs read only its first N = round16(rows) token
+      // rows, which are the first N * 128 bytes of the pre-swizzled tile (the
+      // swizzle permutes 16-byte chunks within a row): copy just those.
+      const uint32_t a_bytes =
+          swap_tile(p, t.rows)
+              ? static_cast<uint32_t>(min(128, max(16, (t.rows + 15) & ~15))) * 128u
+              : kTileBytes;
       // Rows of B for this tile: two 128-row halves.
       int brow0, brow1;
       if (t.kind == 0) {
@@ -375,13 +382,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (operands) {
           if (lane == 0) {
-            mbar_arrive_expect_tx(&sm.full[stage], ab_bytes);
+            mbar_arrive_expect_tx(&sm.full[stage], ab_bytes - kTileBytes + a_bytes);
             // Operand tiles are contiguous and pre-swizzled: one linear bulk
             // copy each (row-major weights fall back to 2-D TMA tiles).
             bulk_load_hint(
                 sm.a[stage],
                 ph.a_tiles + (static_cast<size_t>(t.mt) * ph.k_blocks + kb) * kTileBytes,
-                kTileBytes, &sm.full[stage], pol_a);
+                a_bytes, &sm.full[stage], pol_a);
             if (ph.w_tiles != nullptr) {
               bulk_load_hint(
                   sm.b[stage],
