@@ -166,6 +166,27 @@ def algorithmic_bytes(wl, d):
     return active * per_expert_w + act_bytes, active * per_expert_w, active
 
 
+def side_kernel_bytes(wl):
+    """Algorithmic bytes of the launches around the GEMM, per launch.
+    route: topk_idx in; perm, inv, counts and offsets out.  gather: x and its
+    1x128 scales read once, one row (and its scales) written per slot, perm
+    read.  combine: y, topk_w and inv read per slot; out written."""
+    S = wl.S
+    xe = 2 if wl.w_dtype == "bf16" else 1
+    sf = 0 if wl.w_dtype == "bf16" else wl.H // 128
+    route = S * 4 + 2 * S * 4 + (2 * wl.E + 1) * 4
+    gather = (wl.T + S) * (wl.H * xe + sf) + S * 4
+    combine = S * wl.H * 2 + 2 * S * 4 + wl.T * wl.H * 2
+    return {"route_gather": route + gather, "route_alone": route, "gather_alone": gather,
+            "combine": combine}
+
+
+def kernels_gbs(wl, split):
+    """GB/s of the launches around the GEMM from their mean split times (ms)."""
+    return {k: round(b / (statistics.mean(split[k]) * 1e-3) / 1e9, 1)
+            for k, b in side_kernel_bytes(wl).items() if split.get(k)}
+
+
 def max_over_ranks(values, world, device):
     """Element-wise max of per-rank times (each rank gets the result): a
     replica job is as fast as its slowest rank."""
@@ -399,6 +420,7 @@ def run_b200(args, wl):
                      "hbm_gbs": round(alg_bytes / (ms_per_step * 1e-3) / 1e9, 1),
                      "alg_bytes": alg_bytes, "flops": flops},
         "kernels_ms": {k: round(statistics.mean(v), 4) for k, v in split.items()},
+        "kernels_gbs": kernels_gbs(wl, split),
         "eager_ms_per_step": round(sum(eager_ms) / args.steps, 4),
         "timing": "CUDA-graph replay of moe_forward, events on the launching stream",
         "roofline": roof,

@@ -1,0 +1,47 @@
+"""Host-side arithmetic of bench.py that needs no GPU: the algorithmic bytes
+of the launches around the GEMM and their GB/s, checked against sums worked by
+hand for the decode layer (T=128, H=7168, E=32, top-8, FP8 x) and the BF16
+variant of the same shape."""
+import os
+
+import pytest
+
+from moe_expert_ffn_permute_b200.synth import WORKLOADS
+
+ROOT = os.path.abspath(os.path.join(os.path.dirname(__file__), ".."))
+
+
+def _load_bench():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_side_kernel_bytes_decode():
+    b = _load_bench().side_kernel_bytes(WORKLOADS["decode"])
+    # route: 1024 ids in (4 KiB); perm + inv out (8 KiB); 32 counts + 33 offsets.
+    assert b["route_alone"] == 4096 + 8192 + 65 * 4
+    # gather: 128 token rows read + 1024 slot rows written, 7168 B + 56 scale
+    # bytes each; 1024 perm entries read.
+    assert b["gather_alone"] == 1152 * 7224 + 4096
+    assert b["route_gather"] == b["route_alone"] + b["gather_alone"]
+    # combine: 1024 bf16 y rows + weights + inv in, 128 bf16 rows out.
+    assert b["combine"] == 1024 * 14336 + 8192 + 128 * 14336
+
+
+def test_side_kernel_bytes_bf16_has_no_scales():
+    wl = WORKLOADS["bf16"]
+    b = _load_bench().side_kernel_bytes(wl)
+    assert b["gather_alone"] == (wl.T + wl.S) * wl.H * 2 + wl.S * 4
+
+
+def test_kernels_gbs_uses_mean_time_and_skips_missing():
+    bench = _load_bench()
+    wl = WORKLOADS["decode"]
+    split = {"combine": [0.01, 0.03], "fc1_fc2": [0.2], "route_alone": []}
+    g = bench.kernels_gbs(wl, split)
+    assert set(g) == {"combine"}
+    assert g["combine"] == pytest.approx(bench.side_kernel_bytes(wl)["combine"] / 0.02e-3 / 1e9,
+                                         abs=0.05)
