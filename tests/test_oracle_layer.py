@@ -193,3 +193,33 @@ def test_layer_single_expert_hand_example():
     aq = decode_e4m3(encode_e4m3_rne_satfinite(np.array([a / 2 ** n])))[0] * 2 ** n
     np.testing.assert_array_equal(out, np.full((1, H), 0.75 * 128 * aq))
     assert n == -3 and abs(aq - a) < 1.0
+
+
+def test_layer_two_slot_combine_hand_example():
+    """T=2, E=3, k=2, H=I=128, x = 1: expert e has gate codes 1.0 at block scale
+    2^(e-8) (so g_e = 2^(e-1)), up codes 1.0 (u = 128) and W2 = 1, so each
+    expert's output column is 128 * q(a_e) with a_e = g_e * sigmoid(g_e) * 128.
+    Token 0 goes to experts (2, 0) with weights (0.25, 0.75), token 1 to (1, 2)
+    with (0.5, 0.5): the combine must pair each slot's weight with its own
+    expert's rows, in token order."""
+    H = I = 128
+    E = 3
+    x = np.full((2, H), 0x38, np.uint8)
+    xs = np.full((2, 1), 127, np.uint8)
+    w1 = np.full((E, 2 * I, H), 0x38, np.uint8)
+    w1s = np.array([[[127 - 8 + e], [127]] for e in range(E)], np.uint8)
+    w2 = np.full((E, H, I), 0x38, np.uint8)
+    w2s = np.full((E, 1, 1), 127, np.uint8)
+    idx = np.array([[2, 0], [1, 2]], np.int32)
+    w = np.array([[0.25, 0.75], [0.5, 0.5]])
+    out = L.layer(x, xs, idx, w, w1, w1s, w2, w2s)
+
+    def y(e):
+        g = 2.0 ** (e - 1)
+        a = g / (1 + math.exp(-g)) * 128
+        n = math.ceil(math.log2(a / 448))
+        return 128 * decode_e4m3(encode_e4m3_rne_satfinite(np.array([a / 2 ** n])))[0] * 2 ** n
+
+    expect = np.array([[0.25 * y(2) + 0.75 * y(0)] * H, [0.5 * y(1) + 0.5 * y(2)] * H])
+    np.testing.assert_allclose(out, expect, rtol=1e-15)
+    assert len({y(0), y(1), y(2)}) == 3
