@@ -74,6 +74,13 @@ def test_encode_float64_is_one_rounding_of_the_exact_value():
 def test_scalar_and_vector_rounding_agree():
     rng = np.random.default_rng(5)
     x = rng.standard_normal(3000) * 10.0 ** rng.uniform(-38, 38, 3000)
+    # Exact midpoints between consecutive finite BF16 values (normal and
+    # subnormal, both signs, odd and even lower neighbours): the ties.
+    b = np.concatenate([rng.integers(0x0001, 0x7F7F, 2000), np.arange(0x0000, 0x0100)])
+    lo = F.decode_bf16(b.astype(np.uint16))
+    hi = F.decode_bf16((b + 1).astype(np.uint16))
+    ties = (lo + hi) / 2
+    x = np.concatenate([x, ties, -ties])
     vec = F.decode_bf16(F.encode_bf16_rne(x))
     sca = np.array([L._rne_bf16_scalar(float(v)) for v in x])
     assert np.array_equal(vec, sca)

@@ -223,3 +223,15 @@ def test_layer_two_slot_combine_hand_example():
     expect = np.array([[0.25 * y(2) + 0.75 * y(0)] * H, [0.5 * y(1) + 0.5 * y(2)] * H])
     np.testing.assert_allclose(out, expect, rtol=1e-15)
     assert len({y(0), y(1), y(2)}) == 3
+
+
+def test_bruteforce_e4m3_rounding_agrees_with_the_encoder_on_ties():
+    """The brute-force tier's scalar E4M3 rounding (a scan of every code) against
+    the vectorised encoder on every midpoint between consecutive finite E4M3
+    values, both signs, the values themselves and out-of-range magnitudes."""
+    mags = decode_e4m3(np.arange(0x7F, dtype=np.uint8))
+    mids = (mags[:-1] + mags[1:]) / 2
+    vals = np.concatenate([mids, -mids, mags, -mags, [449.0, 464.0, 1e6, -500.0]])
+    vec = decode_e4m3(encode_e4m3_rne_satfinite(vals))
+    sca = np.array([L._rne_e4m3_scalar(float(v)) for v in vals])
+    np.testing.assert_array_equal(sca, vec)
