@@ -21,7 +21,8 @@
 //
 // Warp roles (12 warps):
 //   warp 0   operand producer: bulk copies of pre-swizzled A/B tiles (2-D TMA
-//            for row-major and MXFP4 weights)
+//            for row-major and MXFP4 weights); a token-major tile copies only
+//            the first round16(rows) rows of its token tile
 //   warp 1   MMA issuer (one lane); owns the tensor-memory allocation
 //   warp 2   tile scheduler: writes task infos into a ring of shared-memory slots
 //   warp 3   scale-factor producer: A scale chunks and prepacked MXFP4 scale
