@@ -166,6 +166,14 @@ def algorithmic_bytes(wl, d):
     return active * per_expert_w + act_bytes, active * per_expert_w, active
 
 
+def workload_config(wl, active):
+    """The keys of the line's ``config`` that define the workload; both arms
+    (this library's and the oracle's) report them."""
+    return {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
+            "w_dtype": wl.w_dtype, "routing": wl.routing, "act": wl.act,
+            "active_experts": active}
+
+
 def side_kernel_bytes(wl):
     """Algorithmic bytes of the launches around the GEMM, per launch.
     route: topk_idx in; perm, inv, counts and offsets out.  gather: x and its
@@ -406,9 +414,7 @@ def run_b200(args, wl):
         "vs_baseline": None, "dtype": {"e4m3": "fp8_e4m3", "e2m1": "fp8_e4m3xe2m1",
                                        "bf16": "bf16"}[wl.w_dtype],
         "data": "synthetic (seeded; random-init weights)",
-        "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
-                   "w_dtype": wl.w_dtype, "routing": wl.routing, "act": wl.act,
-                   "active_experts": active, "l2": "flushed (256 MiB write) before each step",
+        "config": {**workload_config(wl, active), "l2": "flushed (256 MiB write) before each step",
                    "weights": ("tiled (moe_prepack_weights, once)" if tiled else
                                "row-major codes, chunked scales (moe_prepack_weight_scales, once)"
                                if chunked else "row-major"),
@@ -503,8 +509,8 @@ def run_reference(args, wl):
            "ms_per_step": round(1e3 * total / args.steps, 2), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
            "impl": "reference",
-           "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E,
-                      "k": wl.k, "w_dtype": wl.w_dtype},
+           "config": {**workload_config(wl, algorithmic_bytes(wl, d)[2]),
+                      "parallelism": "float64 oracle on the host cores (rank 0)"},
            "cpu_baseline": {"value": round(val, 4), "unit": "tokens/s", "cores": _cores(),
                             "kind": "oracle",
                             "sample": f"{ntok} token(s) of {wl.name} per step"},

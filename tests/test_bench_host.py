@@ -45,3 +45,27 @@ def test_kernels_gbs_uses_mean_time_and_skips_missing():
     assert set(g) == {"combine"}
     assert g["combine"] == pytest.approx(bench.side_kernel_bytes(wl)["combine"] / 0.02e-3 / 1e9,
                                          abs=0.05)
+
+
+def test_reference_arm_line_on_the_small_config():
+    """The oracle arm runs on the host alone and prints one line with the
+    contract's keys and the workload-defining config keys of the other arm."""
+    import json
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny",
+                        "--steps", "1", "--warmup", "1"], cwd=ROOT, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0
+    wl = WORKLOADS["tiny"]
+    want = _load_bench().workload_config(wl, line["config"]["active_experts"])
+    assert {k: line["config"][k] for k in want} == want
+    assert 1 <= line["config"]["active_experts"] <= wl.E
+    assert line["e2e"]["value"] == line["value"]
+    assert line["cpu_baseline"]["kind"] == "oracle"
