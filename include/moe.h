@@ -107,8 +107,10 @@ typedef struct moe_plan_s *moe_plan_t;
 
 /* Build a plan for T tokens, hidden size H, expert intermediate size I, E
  * experts and top-k.  Host only; enqueues nothing and allocates no device
- * memory.  Requirements: T >= 1; H % 128 == 0; I % 128 == 0; 1 <= k <= E <= 256;
- * T*k < 2^31.  Returns MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED otherwise.  */
+ * memory.  Requirements: T >= 1; H % 256 == 0 (FC2 output tiles are 256
+ * columns wide); I % 128 == 0; 1 <= k <= E <= 256; T*k < 2^31.  Returns
+ * MOE_ERR_INVALID_ARG (sizes, k > E, activation parameters) or
+ * MOE_ERR_UNSUPPORTED (H, I or E outside what the kernels handle) otherwise. */
 moe_status moe_plan(int T, int H, int I, int E, int k, moe_dtypes dtypes,
                     moe_act_params act, moe_plan_t *out);
 
