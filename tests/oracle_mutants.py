@@ -1,5 +1,6 @@
 """Mutation check of the oracle's pins (test infrastructure; run by hand:
-``python tests/oracle_mutants.py``, about four minutes on CPU).
+``python tests/oracle_mutants.py [--scratch DIR] [index ...]``, about four
+minutes on CPU; scratch copies go to DIR, else the system's temporary folder).
 
 Each entry plants one plausible mistake (a wrong exponent bias, a dropped term,
 a swapped gate/up, a transposed or reversed scale index, a wrong rounding rule,
@@ -115,12 +116,12 @@ MUTANTS = [
 ]
 
 
-def run(selected=None):
+def run(selected=None, scratch_root=None):
     survivors, missing = [], []
     for i, (rel, text, repl, note) in enumerate(MUTANTS):
         if selected and i not in selected:
             continue
-        scratch = tempfile.mkdtemp(prefix="oracle_mutant_")
+        scratch = tempfile.mkdtemp(prefix="oracle_mutant_", dir=scratch_root)
         try:
             for d in ("oracle", "tests", "moe_expert_ffn_permute_b200"):
                 shutil.copytree(os.path.join(ROOT, d), os.path.join(scratch, d),
@@ -150,4 +151,9 @@ def run(selected=None):
 
 
 if __name__ == "__main__":
-    sys.exit(0 if run([int(a) for a in sys.argv[1:]]) else 1)
+    import argparse
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--scratch", default=None, help="folder for the scratch copies")
+    ap.add_argument("index", nargs="*", type=int, help="run only these mutants")
+    a = ap.parse_args()
+    sys.exit(0 if run(a.index, a.scratch) else 1)
