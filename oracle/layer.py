@@ -163,6 +163,10 @@ def requant_1x128(a):
         for b in range(C // BLOCK):
             blk = a[r, b * BLOCK:(b + 1) * BLOCK]
             n = ue8m0_exponent_for(np.max(np.abs(blk)))
+            if n + 127 > 254:
+                # UE8M0 scales stop at 2^127 (byte 254; 255 is NaN).  Any binary32
+                # activation fits (n <= 120); larger float64 blocks have no encoding.
+                raise ValueError(f"block amax {np.max(np.abs(blk))!r} exceeds 448 * 2^127")
             sf[r, b] = n + 127
             codes[r, b * BLOCK:(b + 1) * BLOCK] = encode_e4m3_rne_satfinite(blk / 2.0 ** n)
     return codes, sf

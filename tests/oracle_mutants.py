@@ -20,7 +20,7 @@ ROOT = os.path.abspath(os.path.join(os.path.dirname(__file__), ".."))
 F, L = "oracle/formats.py", "oracle/layer.py"
 PIN_TESTS = ["tests/test_oracle_formats.py", "tests/test_oracle_layer.py",
              "tests/test_oracle_bf16.py", "tests/test_oracle_route_property.py",
-             "tests/test_golden_params.py"]
+             "tests/test_oracle_requant_property.py", "tests/test_golden_params.py"]
 
 _TAIL = ("                out[t] += w[t, j] * y[t * k + j]\n    if keep:\n        inter.update("
          "counts=counts, offsets=offsets, perm=perm, inv=inv, y=y)\n        return out, inter\n"
