@@ -110,15 +110,23 @@ typedef struct moe_plan_s *moe_plan_t;
  * memory.  Requirements: T >= 1; H % 256 == 0 (FC2 output tiles are 256
  * columns wide); I % 128 == 0; 1 <= k <= E <= 256; T*k < 2^31.  Returns
  * MOE_ERR_INVALID_ARG (sizes, k > E, activation parameters) or
- * MOE_ERR_UNSUPPORTED (H, I or E outside what the kernels handle) otherwise. */
+ * MOE_ERR_UNSUPPORTED (H, I or E outside what the kernels handle) otherwise.
+ * Source: the layer's sizes and variants as the Mega MoE pages name them
+ * (fw-ai/DeepGEMM PR #16, Overview; DeepGEMM PR #445, Summary, for the
+ * activation parameters).
+ */
 moe_status moe_plan(int T, int H, int I, int E, int k, moe_dtypes dtypes,
                     moe_act_params act, moe_plan_t *out);
 
-/* Release a plan (NULL is allowed). */
+/* Release a plan (NULL is allowed).
+ * No counterpart on the pages.
+ */
 void moe_plan_destroy(moe_plan_t plan);
 
 /* Size in bytes of the device workspace moe_forward and the step calls need
- * (256-byte aligned pointer required).  0 for a NULL plan.                   */
+ * (256-byte aligned pointer required).  0 for a NULL plan.
+ * No counterpart on the pages.
+ */
 size_t moe_workspace_bytes(moe_plan_t plan);
 
 /* The whole layer: route -> gather -> FC1 (+ activation + FP8 requant) -> FC2
@@ -130,7 +138,9 @@ size_t moe_workspace_bytes(moe_plan_t plan);
  *   w1, w1_scales, w2, w2_scales   weights in the plan's moe_wdtype layout
  *   out        bf16 [T,H]    written entirely
  *   workspace  moe_workspace_bytes(plan) bytes, device, 256-B aligned.
- * All pointers are device pointers.                                          */
+ * All pointers are device pointers.
+ * Sources: those of the steps below (moe_route ... moe_combine).
+ */
 moe_status moe_forward(moe_plan_t plan, const void *x, const uint8_t *x_scales,
                        const int32_t *topk_idx, const float *topk_w,
                        const void *w1, const uint8_t *w1_scales, const void *w2,
@@ -142,7 +152,10 @@ moe_status moe_forward(moe_plan_t plan, const void *x, const uint8_t *x_scales,
  * copies), the weights and the workspace are device pointers, and out_host is
  * a host bf16 [T,H] buffer.  The host-to-device copies, the layer and the
  * device-to-host copy of the output are enqueued on `stream`; the output is
- * valid after the stream has been synchronised.                             */
+ * valid after the stream has been synchronised.
+ * No counterpart on the pages (a host-buffer convenience around
+ * moe_forward).
+ */
 moe_status moe_forward_hostio(moe_plan_t plan, const void *x_host,
                               const uint8_t *x_scales_host,
                               const int32_t *topk_idx_host,
@@ -164,7 +177,10 @@ moe_status moe_route(moe_plan_t plan, const int32_t *topk_idx, void *workspace,
 
 /* Step 2, gather: copies the x rows (and their scale bytes) of every routed
  * slot into expert order inside the workspace, each expert's block starting
- * at a multiple of 128 rows.  Needs moe_route() first.                      */
+ * at a multiple of 128 rows.  Needs moe_route() first.
+ * Source: DeepGEMM PR #386 Description (tokens grouped per expert before the
+ * expert GEMMs).
+ */
 moe_status moe_gather(moe_plan_t plan, const void *x, const uint8_t *x_scales,
                       void *workspace, moe_stream_t stream);
 
@@ -173,19 +189,29 @@ moe_status moe_gather(moe_plan_t plan, const void *x, const uint8_t *x_scales,
  * Up to 4096 slots this is one launch in which each block repeats the
  * counting sort in shared memory and then copies its share of rows; above
  * that it enqueues the separate launches.  moe_forward() uses it.  Same
- * argument rules as the two calls.                                          */
+ * argument rules as the two calls.
+ * Sources: those of moe_route and moe_gather.
+ */
 moe_status moe_route_gather(moe_plan_t plan, const int32_t *topk_idx, const void *x,
                             const uint8_t *x_scales, void *workspace, moe_stream_t stream);
 
 /* Step 3, FC1: the FC1 grouped GEMM on the 5th-generation tensor cores with
  * the block scales applied in hardware, the fused (OAI-)SwiGLU, and the FP8
  * E4M3 + UE8M0 1x128 requantisation of the activation, all in one kernel.
- * Needs moe_gather() first.                                                 */
+ * Needs moe_gather() first.
+ * Sources: DeepGEMM PR #445 "Environment" (FP8 E4M3 weights) and Summary
+ * (the activation); DeepGEMM PR #386 title (native UE8M0 scales); TensorRT-
+ * LLM PR #16346 Description (FP8 + 1x128 UE8M0 requantisation in a GEMM
+ * epilogue).
+ */
 moe_status moe_fc1(moe_plan_t plan, const void *w1, const uint8_t *w1_scales,
                    void *workspace, moe_stream_t stream);
 
 /* Step 4, FC2: grouped GEMM of the requantised activation with W2; bf16 rows
- * written in slot order (y[s], s = t*k + j).  Needs moe_fc1() first.         */
+ * written in slot order (y[s], s = t*k + j).  Needs moe_fc1() first.
+ * Source: DeepGEMM PR #386 title ("direct combine": rows land where the
+ * combine reads them).
+ */
 moe_status moe_fc2(moe_plan_t plan, const void *w2, const uint8_t *w2_scales,
                    void *workspace, moe_stream_t stream);
 
@@ -194,7 +220,10 @@ moe_status moe_fc2(moe_plan_t plan, const void *w2, const uint8_t *w2_scales,
  * an FC2 tile of an m-tile starts once every FC1 tile of that m-tile has
  * published its activation rows.  Same results as moe_fc1() then moe_fc2().
  * Needs moe_gather() first (and moe_route() before it, which resets the
- * launch's counters).                                                      */
+ * launch's counters).
+ * Source: fw-ai/DeepGEMM PR #16 Overview (the persistent scheduler and its
+ * task-slot release ordering).
+ */
 moe_status moe_fc1_fc2(moe_plan_t plan, const void *w1, const uint8_t *w1_scales,
                        const void *w2, const uint8_t *w2_scales, void *workspace,
                        moe_stream_t stream);
@@ -268,7 +297,9 @@ moe_status moe_workspace_view(moe_plan_t plan, void *workspace,
  * b = column / 128 are stored inside the workspace in the layout the FC2
  * tensor cores read; this copies them out as a plain u8 [rows, I/128] array
  * (device pointer `dst`), enqueued on `stream`.  MOE_ERR_UNSUPPORTED for
- * MOE_W_BF16 plans (no scales).                                              */
+ * MOE_W_BF16 plans (no scales).
+ * No counterpart on the pages (inspection).
+ */
 moe_status moe_copy_act_scales(moe_plan_t plan, const void *workspace,
                                uint8_t *dst, moe_stream_t stream);
 
@@ -297,7 +328,10 @@ moe_status moe_plan_set_weight_layout(moe_plan_t plan, int layout);
  * (r % 32) * 16 + (r / 32) * 4 -- the layout the tensor core's scale copy
  * reads, so a pipeline stage needs two contiguous 512-byte copies instead of
  * 256 scattered 4-byte reads.  Done once per weight set, on `stream`.
- * MOE_ERR_UNSUPPORTED for other weight formats.                             */
+ * MOE_ERR_UNSUPPORTED for other weight formats.
+ * No counterpart on the pages (a storage layout for this library's tensor-
+ * core kernels).
+ */
 moe_status moe_prepack_weight_scales(moe_plan_t plan, const uint8_t *w1_scales,
                                      const uint8_t *w2_scales, uint8_t *w1_scales_chunked,
                                      uint8_t *w2_scales_chunked, moe_stream_t stream);
@@ -310,11 +344,15 @@ moe_status moe_prepack_weight_scales(moe_plan_t plan, const uint8_t *w1_scales,
  * weights; set the weight layout first).  Results are the same bytes either
  * way.  On pairs,
  * moe_fc1_fc2 enqueues two kernels: the weight scales (w1_scales, w2_scales)
- * are first expanded into a workspace region, then the GEMMs run.          */
+ * are first expanded into a workspace region, then the GEMMs run.
+ * No counterpart on the pages (the B200's 2-SM MMA).
+ */
 moe_status moe_plan_set_cta_pairs(moe_plan_t plan, int mode);
 
 /* 1 if moe_fc1_fc2 / moe_forward run the GEMMs on CTA pairs with the plan's
- * current settings, 0 if not (or plan is NULL).                             */
+ * current settings, 0 if not (or plan is NULL).
+ * No counterpart on the pages.
+ */
 int moe_plan_cta_pairs_active(moe_plan_t plan);
 
 /* Token-major ("swap AB") GEMM tiles, the swapAB variant of the Mega MoE
@@ -330,7 +368,9 @@ int moe_plan_cta_pairs_active(moe_plan_t plan);
 moe_status moe_plan_set_swap_ab(moe_plan_t plan, int mode);
 
 /* 0: the GEMMs use token-row tiles only; 1: token-major tiles throughout;
- * 2: chosen tile by tile (automatic mode).                                   */
+ * 2: chosen tile by tile (automatic mode).
+ * Source: as moe_plan_set_swap_ab.
+ */
 int moe_plan_swap_ab_active(moe_plan_t plan);
 
 /* Rearrange row-major FP8 or BF16 weights w1 [E,2I,H] and w2 [E,H,I] (device)
@@ -340,14 +380,19 @@ int moe_plan_swap_ab_active(moe_plan_t plan);
  * [E*2I, H] (or [E*H, I]) matrix, bytes 128kb..128kb+127 of each row -- is
  * 16384 bytes at offset (b * KB/128 + kb) * 16384, and byte c of tile row r
  * lies at r*128 + ((c/16) XOR (r%8))*16 + c%16.  Done once per weight set
- * (e.g. at model load), enqueued on `stream`.                               */
+ * (e.g. at model load), enqueued on `stream`.
+ * No counterpart on the pages (a storage layout for this library's tensor-
+ * core kernels).
+ */
 moe_status moe_prepack_weights(moe_plan_t plan, const void *w1, const void *w2,
                                void *w1_tiled, void *w2_tiled, moe_stream_t stream);
 
 /* Copy the FC1 activation codes out of the workspace as a row-major u8
  * [rows, I] array (MOE_W_BF16: bf16 [rows, I]; device pointer `dst`, 16-byte
  * aligned), enqueued on `stream`; inside the workspace they are kept in the
- * tiled layout.                                                             */
+ * tiled layout.
+ * No counterpart on the pages (inspection).
+ */
 moe_status moe_copy_act(moe_plan_t plan, const void *workspace, uint8_t *dst,
                         moe_stream_t stream);
 
@@ -357,22 +402,32 @@ moe_status moe_copy_act(moe_plan_t plan, const void *workspace, uint8_t *dst,
  * without CTA pairs) every FC2 tile waits for one FC1 completion more than its
  * m-tile can provide, so that bounded wait runs out (about 2 s): the launch
  * stops, the error word gets MOE_ERR_DEVICE_TIMEOUT, nothing traps or hangs,
- * and the output is undefined.  Other bits: MOE_ERR_INVALID_ARG.            */
+ * and the output is undefined.  Other bits: MOE_ERR_INVALID_ARG.
+ * No counterpart on the pages.
+ */
 moe_status moe_plan_set_debug(moe_plan_t plan, int flags);
 
-/* Zero the workspace's device error word (enqueued on `stream`). */
+/* Zero the workspace's device error word (enqueued on `stream`).
+ * No counterpart on the pages.
+ */
 moe_status moe_clear_device_error(moe_plan_t plan, void *workspace,
                                   moe_stream_t stream);
 
 /* Synchronises `stream`, reads the device error word and returns MOE_OK or
- * the most severe recorded status (timeout before bad routing).            */
+ * the most severe recorded status (timeout before bad routing).
+ * No counterpart on the pages.
+ */
 moe_status moe_check_device_error(moe_plan_t plan, const void *workspace,
                                   moe_stream_t stream);
 
-/* Human-readable name of a status code (static string). */
+/* Human-readable name of a status code (static string).
+ * No counterpart on the pages.
+ */
 const char *moe_status_str(moe_status status);
 
-/* Kernel launches one moe_forward enqueues for this plan. */
+/* Kernel launches one moe_forward enqueues for this plan.
+ * No counterpart on the pages.
+ */
 int moe_forward_launch_count(moe_plan_t plan);
 
 #ifdef __cplusplus
