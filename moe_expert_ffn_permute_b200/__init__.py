@@ -16,6 +16,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                 3: "MOE_ERR_ALIGNMENT", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_TIMEOUT",
                 6: "MOE_ERR_BAD_ROUTING"}
@@ -286,6 +287,48 @@ def moe_forward_launch_count(plan):
     return lib().moe_forward_launch_count(plan)
 
 
+def _expect(name, t, shape, dtype, device):
+    import torch
+    if t is None:
+        raise MoEError(MOE_ERR_INVALID_ARG, f"{name} is required")
+    if not isinstance(t, torch.Tensor):
+        return                      # a raw address: the caller vouches for it
+    if (tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous()
+            or t.device != device):
+        raise MoEError(MOE_ERR_INVALID_ARG,
+                       f"{name}: expected a contiguous {dtype} tensor of shape {tuple(shape)} on "
+                       f"{device}, got {t.dtype} {tuple(t.shape)} on {t.device}"
+                       f"{'' if t.is_contiguous() else ' (not contiguous)'}")
+
+
+def check_layer_args(T, H, I, E, k, w_dtype, device, x, x_scales, topk_idx, topk_w, w1,
+                     w1_scales, w2, w2_scales, out):
+    """Shapes, dtypes, contiguity and device of moe_forward's tensors for a plan
+    (T, H, I, E, k, w_dtype), as include/moe.h lays them out.  The C ABI sees
+    only pointers, so a wrong-sized tensor would be read past its end; this
+    check catches that before the call.  Tiled weights and chunked scales have
+    the shapes of the row-major ones.  Raises MoEError(MOE_ERR_INVALID_ARG)."""
+    import torch
+    u8, bf16 = torch.uint8, torch.bfloat16
+    if w_dtype == "bf16":
+        _expect("x", x, (T, H), bf16, device)
+        _expect("w1", w1, (E, 2 * I, H), bf16, device)
+        _expect("w2", w2, (E, H, I), bf16, device)
+    else:
+        _expect("x", x, (T, H), u8, device)
+        _expect("x_scales", x_scales, (T, H // 128), u8, device)
+        if w_dtype == "e4m3":
+            shapes = ((E, 2 * I, H), (E, 2 * I // 128, H // 128), (E, H, I), (E, H // 128, I // 128))
+        else:
+            shapes = ((E, 2 * I, H // 2), (E, 2 * I, H // 32), (E, H, I // 2), (E, H, I // 32))
+        for name, t, shape in zip(("w1", "w1_scales", "w2", "w2_scales"),
+                                  (w1, w1_scales, w2, w2_scales), shapes):
+            _expect(name, t, shape, u8, device)
+    _expect("topk_idx", topk_idx, (T, k), torch.int32, device)
+    _expect("topk_w", topk_w, (T, k), torch.float32, device)
+    _expect("out", out, (T, H), bf16, device)
+
+
 class MoELayer:
     """Convenience owner of a plan and its torch-allocated workspace."""
 
@@ -294,6 +337,7 @@ class MoELayer:
                  cta_pairs=None, swap_ab=None, chunked_scales=False):
         import torch
         self.T, self.H, self.I, self.E, self.k = T, H, I, E, k
+        self.w_dtype = w_dtype
         self.plan = moe_plan(T, H, I, E, k, w_dtype, act, alpha, up_bias, limit)
         if tiled_weights:
             moe_plan_set_weight_layout(self.plan, 1)
@@ -314,6 +358,9 @@ class MoELayer:
         import torch
         if out is None:
             out = torch.empty(self.T, self.H, dtype=torch.bfloat16, device=self.workspace.device)
+        check_layer_args(self.T, self.H, self.I, self.E, self.k, self.w_dtype,
+                         self.workspace.device, x, x_scales, topk_idx, topk_w, w1, w1_scales,
+                         w2, w2_scales, out)
         moe_forward(self.plan, x, x_scales, topk_idx, topk_w, w1, w1_scales, w2, w2_scales, out,
                     self.workspace, stream)
         return out

@@ -1,0 +1,65 @@
+"""The Python convenience layer's tensor checks (``check_layer_args``, called by
+``MoELayer.forward`` before the C ABI, which sees only pointers): every input
+the generators produce for each weight format passes, including prepacked
+weights and chunked scales (same shapes), and a wrong shape, dtype, device,
+layout or a missing tensor is refused with MOE_ERR_INVALID_ARG."""
+import pytest
+import torch
+
+import moe_expert_ffn_permute_b200 as moe
+from moe_expert_ffn_permute_b200.synth import Workload, make_inputs
+
+CPU = torch.device("cpu")
+CASES = [Workload("ragged", 300, 1024, 512, 8, 4, cfg_id=10),
+         Workload("ragged-fp4", 200, 1024, 512, 6, 3, w_dtype="e2m1", cfg_id=11),
+         Workload("ragged-bf16", 300, 1024, 512, 8, 4, w_dtype="bf16", cfg_id=30),
+         Workload("single", 1, 512, 128, 1, 1, cfg_id=12)]
+
+
+def _args(wl, d, **over):
+    out = torch.empty(wl.T, wl.H, dtype=torch.bfloat16)
+    a = dict(x=d["x"], x_scales=d["x_scales"], topk_idx=d["topk_idx"], topk_w=d["topk_w"],
+             w1=d["w1"], w1_scales=d["w1_scales"], w2=d["w2"], w2_scales=d["w2_scales"], out=out)
+    a.update(over)
+    return a
+
+
+def _check(wl, **a):
+    moe.check_layer_args(wl.T, wl.H, wl.I, wl.E, wl.k, wl.w_dtype, CPU, **a)
+
+
+@pytest.mark.parametrize("wl", CASES, ids=lambda w: w.name)
+def test_generated_inputs_pass(wl):
+    d = make_inputs(wl)
+    _check(wl, **_args(wl, d))
+    # Prepacked weights / chunked scales are buffers of the same shape.
+    _check(wl, **_args(wl, d, w1=torch.empty_like(d["w1"]), w2=torch.empty_like(d["w2"])))
+    # Raw addresses are passed through unchecked.
+    _check(wl, **_args(wl, d, w1=12345 * 256))
+
+
+@pytest.mark.parametrize("wl", CASES[:3], ids=lambda w: w.name)
+def test_bad_tensors_are_refused(wl):
+    d = make_inputs(wl)
+    bad = [dict(x=d["x"][:-1]),                                  # too few rows
+           dict(topk_idx=d["topk_idx"].long()),                  # int64 ids
+           dict(topk_w=d["topk_w"].double()),
+           dict(w2=d["w2"][:, :, :-16]),                         # short rows
+           dict(out=torch.empty(wl.T, wl.H, dtype=torch.float32)),
+           dict(x=d["x"].t().contiguous().t()),                  # not contiguous
+           dict(topk_idx=None)]
+    if wl.w_dtype != "bf16":
+        bad += [dict(x_scales=None), dict(w1_scales=d["w1_scales"][:-1])]
+    for over in bad:
+        with pytest.raises(moe.MoEError) as ei:
+            _check(wl, **_args(wl, d, **over))
+        assert ei.value.status == moe.MOE_ERR_INVALID_ARG, over
+    with pytest.raises(moe.MoEError):
+        moe.check_layer_args(wl.T, wl.H, wl.I, wl.E, wl.k, wl.w_dtype, torch.device("meta"),
+                             **_args(wl, d))
+
+
+def test_bf16_layers_ignore_scale_arguments():
+    wl = CASES[2]
+    d = make_inputs(wl)
+    _check(wl, **_args(wl, d, x_scales=torch.empty(1), w1_scales=None))
