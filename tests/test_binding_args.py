@@ -63,3 +63,23 @@ def test_bf16_layers_ignore_scale_arguments():
     wl = CASES[2]
     d = make_inputs(wl)
     _check(wl, **_args(wl, d, x_scales=torch.empty(1), w1_scales=None))
+
+
+@pytest.mark.parametrize("w_dtype", ["e4m3", "e2m1", "bf16"])
+def test_layer_forward_checks_before_the_call(monkeypatch, w_dtype):
+    """MoELayer.forward runs the checks and only then calls moe_forward (the
+    library calls that need a GPU are replaced by recorders here)."""
+    calls = []
+    monkeypatch.setattr(moe, "moe_clear_device_error", lambda *a, **k: None)
+    monkeypatch.setattr(moe, "moe_forward", lambda *a, **k: calls.append(a))
+    wl = Workload("t", 40, 512, 256, 4, 2, w_dtype=w_dtype, cfg_id=3)
+    d = make_inputs(wl)
+    lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype=w_dtype, device="cpu")
+    args = [d[n] for n in ("x", "x_scales", "topk_idx", "topk_w", "w1", "w1_scales", "w2",
+                           "w2_scales")]
+    out = lay.forward(*args)
+    assert out.shape == (wl.T, wl.H) and out.dtype == torch.bfloat16 and len(calls) == 1
+    args[0] = args[0][:-1]
+    with pytest.raises(moe.MoEError):
+        lay.forward(*args)
+    assert len(calls) == 1
