@@ -218,7 +218,7 @@ def run_b200(args, wl):
 
     import moe_expert_ffn_permute_b200 as moe
     from moe_expert_ffn_permute_b200.build import build
-    from moe_expert_ffn_permute_b200.synth import make_inputs
+    from workloads.synth import make_inputs
 
     rank, world, local = _dist()
     if world > 1:
@@ -475,7 +475,7 @@ def cpu_baseline(wl, d, args, ntok=None):
     """The float64 oracle, as it stands, on a bounded sample of the workload's
     tokens (the oracle's cost is dominated by dequantising the touched experts'
     weights, so a few tokens already take seconds)."""
-    from moe_expert_ffn_permute_b200.synth import to_numpy
+    from workloads.synth import to_numpy
     dn = to_numpy(d)
     ntok = ntok or args.cpu_tokens
     t0 = time.perf_counter()
@@ -491,7 +491,7 @@ def run_reference(args, wl):
     if rank != 0:
         return
     import torch
-    from moe_expert_ffn_permute_b200.synth import make_inputs, to_numpy
+    from workloads.synth import make_inputs, to_numpy
     d = make_inputs(wl, device="cuda" if torch.cuda.is_available() else "cpu")
     dn = to_numpy(d)
     ntok = args.cpu_tokens
@@ -537,7 +537,7 @@ def main():
                     help="weights as given (row-major, 2-D TMA; MXFP4 scales unchunked) "
                          "instead of prepacked")
     args = ap.parse_args()
-    from moe_expert_ffn_permute_b200.synth import WORKLOADS
+    from workloads.synth import WORKLOADS
     wl = WORKLOADS[args.workload]
     if args.tokens:
         wl = wl.with_tokens(args.tokens)

@@ -5,7 +5,7 @@ import torch
 
 import moe_expert_ffn_permute_b200 as moe
 from moe_expert_ffn_permute_b200.build import build
-from moe_expert_ffn_permute_b200.synth import Workload, make_inputs, to_numpy
+from workloads.synth import Workload, make_inputs, to_numpy
 from oracle import layer as L
 
 CALC_DIFF_MAX = 1e-4       # DeepGEMM-style calc_diff bound

@@ -6,7 +6,7 @@ import os
 
 import pytest
 
-from moe_expert_ffn_permute_b200.synth import WORKLOADS
+from workloads.synth import WORKLOADS
 
 ROOT = os.path.abspath(os.path.join(os.path.dirname(__file__), ".."))
 

@@ -7,7 +7,7 @@ import pytest
 import torch
 
 import moe_expert_ffn_permute_b200 as moe
-from moe_expert_ffn_permute_b200.synth import Workload, make_inputs
+from workloads.synth import Workload, make_inputs
 
 CPU = torch.device("cpu")
 CASES = [Workload("ragged", 300, 1024, 512, 8, 4, cfg_id=10),

@@ -6,7 +6,7 @@ import os
 import numpy as np
 
 from oracle import layer as L
-from moe_expert_ffn_permute_b200.synth import WORKLOADS
+from workloads.synth import WORKLOADS
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "activation_params.json")
 

@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import moe_expert_ffn_permute_b200 as moe
-from moe_expert_ffn_permute_b200.synth import WORKLOADS, Workload, to_numpy
+from workloads.synth import WORKLOADS, Workload, to_numpy
 from oracle import formats as F
 
 from gpu_helpers import assert_parity, ensure_built, inputs, oracle_layer, oracle_tokens

@@ -9,7 +9,7 @@ import pytest
 import torch
 
 import moe_expert_ffn_permute_b200 as moe
-from moe_expert_ffn_permute_b200.synth import Workload, to_numpy
+from workloads.synth import Workload, to_numpy
 from oracle import layer as L
 
 from gpu_helpers import assert_parity, ensure_built, inputs, oracle_args, oracle_kw

@@ -5,7 +5,7 @@ import pytest
 import torch
 
 import moe_expert_ffn_permute_b200 as moe
-from moe_expert_ffn_permute_b200.synth import WORKLOADS, Workload, to_numpy
+from workloads.synth import WORKLOADS, Workload, to_numpy
 from oracle import layer as L
 
 from gpu_helpers import (assert_parity, ensure_built, inputs, layer_for, oracle_args,

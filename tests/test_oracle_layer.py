@@ -14,7 +14,7 @@ import torch
 
 from oracle import layer as L
 from oracle.formats import decode_e4m3, encode_e4m3_rne_satfinite
-from moe_expert_ffn_permute_b200.synth import Workload, make_inputs, to_numpy
+from workloads.synth import Workload, make_inputs, to_numpy
 
 
 # ------------------------------------------------------------------ routing
