@@ -4,8 +4,12 @@ python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl {b
 
 One step = one whole layer (route, gather, FC1 + SwiGLU + FP8 requant, FC2,
 combine) over one batch of seeded synthetic inputs already resident in HBM.
-The default workload is the decode-size layer (T=128, H=7168, I=2048, E=32,
-top-8, skewed routing).  With N > 1 (launched by torch.distributed.run) every
+The headline workload is the largest configuration that fits one GPU: the
+FP8-activation x MXFP4-weight layer at T=32768 (H=7168, I=3072, E=48, top-6);
+`per_config` adds a shorter record (tokens/s, step time, fused-GEMM time and
+its roofline fraction) of every configuration: decode, prefill, OAI, the BF16
+variant and MXFP4 at 128, 1024, 8192 and 32768 tokens.  With N > 1 (launched
+by torch.distributed.run, or started by `--gpus N` itself) every
 rank runs its own replica of the layer on its own GPU: the path has no exchange
 step, so there is no collective on the data path (weak scaling); the elapsed
 device time is the maximum over ranks.
@@ -212,179 +216,30 @@ def replica_throughput(tokens_per_rank, world, total_ms, steps):
     return tokens_per_rank * world / (total_ms * 1e-3 / steps)
 
 
-def run_b200(args, wl):
-    import torch
-    import torch.distributed as dist
+# The line's headline workload: the largest configuration that fits one GPU
+# (the FP8-activation x MXFP4-weight layer at 32768 tokens); the per-config
+# record covers every configuration of the layer.
+HEADLINE = ("mxfp4", 32768)
+PER_CONFIG = (("decode", None), ("prefill", None), ("oai", None), ("bf16", None),
+              ("mxfp4", 128), ("mxfp4", 1024), ("mxfp4", 8192), ("mxfp4", 32768))
+PER_CONFIG_STEPS = 10
 
-    import moe_expert_ffn_permute_b200 as moe
-    from moe_expert_ffn_permute_b200.build import build
-    from workloads.synth import make_inputs
 
-    rank, world, local = _dist()
-    if world > 1:
-        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=300))
-    torch.cuda.set_device(local)
-    if rank == 0:
-        build()
-    if world > 1:
-        dist.barrier()
-    lib = moe.lib()
-    dev = torch.device("cuda", local)
-    d = make_inputs(wl, device=dev)
-    # FP8 weights are rearranged once into the tensor-core tile layout (as at
-    # model load); the timed steps read them in that layout.
-    tiled = wl.w_dtype in ("e4m3", "bf16") and not args.row_major_weights
-    chunked = wl.w_dtype == "e2m1" and not args.row_major_weights
-    lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype=wl.w_dtype, act=wl.act,
-                       alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit, device=dev,
-                       tiled_weights=tiled, cta_pairs=args.cta_pairs if tiled else None,
-                       swap_ab=args.swap_ab, chunked_scales=chunked)
-    pairs = moe.moe_plan_cta_pairs_active(lay.plan)
-    d_row_major = dict(d)          # the oracle reads the original layout
-    if tiled:
-        d["w1"], d["w2"] = lay.prepack(d["w1"], d["w2"])
-        torch.cuda.synchronize()
-    if chunked:
-        d["w1_scales"], d["w2_scales"] = lay.prepack_scales(d["w1_scales"], d["w2_scales"])
-        torch.cuda.synchronize()
-    out = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=dev)
-    stream = torch.cuda.current_stream()
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    args_dev = (d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], d["w1"], d["w1_scales"],
-                d["w2"], d["w2_scales"])
+def workload(name, tokens=None):
+    from workloads.synth import WORKLOADS
+    wl = WORKLOADS[name]
+    return wl.with_tokens(tokens) if tokens else wl
 
-    def fwd(st=None):
-        moe.moe_forward(lay.plan, *args_dev, out, lay.workspace,
-                        st if st is not None else torch.cuda.current_stream())
 
-    steps = [("route_gather", lambda: moe.moe_route_gather(lay.plan, d["topk_idx"], d["x"],
-                                                           d["x_scales"], lay.workspace,
-                                                           stream)),
-             ("fc1_fc2", lambda: moe.moe_fc1_fc2(lay.plan, d["w1"], d["w1_scales"], d["w2"],
-                                                 d["w2_scales"], lay.workspace, stream)),
-             ("combine", lambda: moe.moe_combine(lay.plan, d["topk_w"], out, lay.workspace,
-                                                 stream))]
-    # Routing and gather as separate launches, and the two GEMMs as separate
-    # launches (informational; moe_forward fuses each pair).
-    extra = [("route_alone", lambda: moe.moe_route(lay.plan, d["topk_idx"], lay.workspace,
-                                                   stream)),
-             ("gather_alone", lambda: moe.moe_gather(lay.plan, d["x"], d["x_scales"],
-                                                     lay.workspace, stream)),
-             ("fc1_alone", lambda: moe.moe_fc1(lay.plan, d["w1"], d["w1_scales"],
-                                               lay.workspace, stream)),
-             ("fc2_alone", lambda: moe.moe_fc2(lay.plan, d["w2"], d["w2_scales"],
-                                               lay.workspace, stream))]
-
-    for _ in range(args.warmup):
-        fwd()
-    torch.cuda.synchronize()
-    if lay.check() != 0:
-        raise RuntimeError("device error during warm-up")
-
-    # The timed step replays a CUDA graph of moe_forward (the same kernels with
-    # the same arguments; the routing kernel resets the GEMM scheduler's
-    # counters inside the graph, so every replay starts from a clean state).
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        fwd()
-    torch.cuda.synchronize()
-
-    def step():
-        graph.replay()
-
-    # ---- timed: whole layer, device-resident inputs.  The clock sampler needs
-    # ~100 ms per sample, longer than K steps of this layer take, so the timed
-    # steps sit inside a window of continuous (untimed) steps of the same layer
-    # that starts and ends 0.6 s around them; all samples are taken under load.
-    clocks = Clocks(local)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-
-    def soak(seconds):
-        t_end = time.perf_counter() + seconds
-        while time.perf_counter() < t_end:
-            for _ in range(20):
-                step()
-            torch.cuda.synchronize()
-
-    def timed(fn):
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
-        for i in range(args.steps):
-            flush.fill_(i & 0xFF)
-            ev[i][0].record(stream)
-            fn()
-            ev[i][1].record(stream)
-        torch.cuda.synchronize()
-        return [a.elapsed_time(b) for a, b in ev]
-
-    soak(0.6)
-    step_ms = timed(step)
-    # ---- per-kernel split (the launch sequence of moe_forward, one event per
-    # step boundary, on the launching stream), then the unfused launches.
-    split = {name: [] for name, _ in steps + extra}
-
-    def split_timing():
-        for seq in (steps, extra):
-            for i in range(args.steps):
-                flush.fill_(i & 0xFF)
-                evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(seq) + 1)]
-                evs[0].record(stream)
-                for j, (_, fn) in enumerate(seq):
-                    fn()
-                    evs[j + 1].record(stream)
-                torch.cuda.synchronize()
-                for j, (name, _) in enumerate(seq):
-                    split[name].append(evs[j].elapsed_time(evs[j + 1]))
-
-    # Everything on the line is measured in the same sustained state: the
-    # eager calls and the per-kernel split also sit between continuous steps.
-    soak(0.3)
-    eager_ms = timed(fwd)
-    soak(0.3)
-    split_timing()
-    soak(0.3)
-    clk = clocks.stop()
-    if world > 1:
-        dist.barrier()
-    total_ms = sum(step_ms)
-
-    # ---- e2e through the host-buffer entry point
-    host = {k: (None if d[k] is None else d[k].cpu().pin_memory())
-            for k in ("x", "x_scales", "topk_idx", "topk_w")}
-    out_h = torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory()
-    for _ in range(args.warmup):
-        moe.moe_forward_hostio(lay.plan, host["x"], host["x_scales"], host["topk_idx"],
-                               host["topk_w"], d["w1"], d["w1_scales"], d["w2"], d["w2_scales"],
-                               out_h, lay.workspace, stream)
-    torch.cuda.synchronize()
-    e2e_ms = []
-    for i in range(args.steps):
-        flush.fill_(i & 0xFF)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        moe.moe_forward_hostio(lay.plan, host["x"], host["x_scales"], host["topk_idx"],
-                               host["topk_w"], d["w1"], d["w1_scales"], d["w2"], d["w2_scales"],
-                               out_h, lay.workspace, stream)
-        b.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms.append(a.elapsed_time(b))
-    if lay.check() != 0:
-        raise RuntimeError("device error during timing")
-
-    # ---- max over ranks
-    total_ms, e2e_total = max_over_ranks([total_ms, sum(e2e_ms)], world, dev)
-
-    alg_bytes, w_bytes, active = algorithmic_bytes(wl, d)
-    hbm, bf16, bf16_sus, peak_src = _peaks()
+def roofline(wl, alg_bytes, w_bytes, active, gemm_ms, pairs=False):
+    """Roofline of the dominant kernel (the fused FC1+FC2 GEMM launch) from its
+    mean split time: HBM-bound workloads count the active experts' weight and
+    scale bytes per launch against the measured copy bandwidth, tensor-bound
+    ones count 6*S*H*I FLOP against the measured sustained bf16 GEMM rate (x2
+    for FP8 and FP8 x FP4 operands: the GEMM time comes from continuous steps,
+    the sustained power-capped state)."""
+    hbm, _, bf16_sus, peak_src = _peaks()
     flops = 6.0 * wl.S * wl.H * wl.I
-    gemm_ms = statistics.mean(split["fc1_fc2"])
-    # Tensor peak of the GEMM's own input type: the measured bf16 figure for
-    # BF16 weights, twice it for FP8 (and E4M3 x E2M1) operands.  The GEMM time
-    # comes from the split taken between continuous steps, so the sustained
-    # (power-capped) bf16 measurement is the matching denominator.
     tc_mult = 1.0 if wl.w_dtype == "bf16" else 2.0
     hbm_bound = alg_bytes / (hbm * 1e9) > flops / (tc_mult * bf16_sus * 1e12)
     if hbm_bound:
@@ -405,41 +260,308 @@ def run_b200(args, wl):
     roof["peak_source"] = f"{peak_src}" + (" copy bandwidth" if roof["unit"] == "GB/s" else
                                            " bf16 sustained" if tc_mult == 1.0 else
                                            " bf16 sustained x2 (FP8 = 2x bf16 nominal)")
+    return roof
 
-    ms_per_step = total_ms / args.steps
+
+class LayerBench:
+    """One workload on this rank's GPU: seeded inputs, weights in the layout the
+    library streams fastest (FP8/BF16 tiles, MXFP4 scale chunks; prepacked once,
+    as at model load), the layer, and a CUDA graph of moe_forward."""
+
+    def __init__(self, wl, args, dev, keep_row_major=False):
+        import torch
+
+        import moe_expert_ffn_permute_b200 as moe
+        from workloads.synth import make_inputs
+        self.moe, self.wl, self.args, self.dev = moe, wl, args, dev
+        d = make_inputs(wl, device=dev)
+        self.tiled = wl.w_dtype in ("e4m3", "bf16") and not args.row_major_weights
+        self.chunked = wl.w_dtype == "e2m1" and not args.row_major_weights
+        self.lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype=wl.w_dtype, act=wl.act,
+                                alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit, device=dev,
+                                tiled_weights=self.tiled,
+                                cta_pairs=args.cta_pairs if self.tiled else None,
+                                swap_ab=args.swap_ab, chunked_scales=self.chunked)
+        self.pairs = moe.moe_plan_cta_pairs_active(self.lay.plan)
+        self.alg_bytes, self.w_bytes, self.active = algorithmic_bytes(wl, d)
+        self.d_row_major = dict(d) if keep_row_major else None   # the oracle's layout
+        if self.tiled:
+            d["w1"], d["w2"] = self.lay.prepack(d["w1"], d["w2"])
+        if self.chunked:
+            d["w1_scales"], d["w2_scales"] = self.lay.prepack_scales(d["w1_scales"],
+                                                                     d["w2_scales"])
+        torch.cuda.synchronize()
+        self.d = d
+        self.out = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=dev)
+        self.stream = torch.cuda.current_stream()
+        self.graph = None
+
+    def fwd(self):
+        d = self.d
+        self.moe.moe_forward(self.lay.plan, d["x"], d["x_scales"], d["topk_idx"], d["topk_w"],
+                             d["w1"], d["w1_scales"], d["w2"], d["w2_scales"], self.out,
+                             self.lay.workspace, self.stream)
+
+    def steps(self, unfused=False):
+        """The launch sequence of moe_forward one call per step (route+gather,
+        FC1+FC2, combine), or with routing, gather and the two GEMMs as separate
+        launches (informational)."""
+        moe, d, lay, st = self.moe, self.d, self.lay, self.stream
+        if not unfused:
+            return [("route_gather", lambda: moe.moe_route_gather(lay.plan, d["topk_idx"], d["x"],
+                                                                  d["x_scales"], lay.workspace, st)),
+                    ("fc1_fc2", lambda: moe.moe_fc1_fc2(lay.plan, d["w1"], d["w1_scales"], d["w2"],
+                                                        d["w2_scales"], lay.workspace, st)),
+                    ("combine", lambda: moe.moe_combine(lay.plan, d["topk_w"], self.out,
+                                                        lay.workspace, st))]
+        return [("route_alone", lambda: moe.moe_route(lay.plan, d["topk_idx"], lay.workspace, st)),
+                ("gather_alone", lambda: moe.moe_gather(lay.plan, d["x"], d["x_scales"],
+                                                        lay.workspace, st)),
+                ("fc1_alone", lambda: moe.moe_fc1(lay.plan, d["w1"], d["w1_scales"],
+                                                  lay.workspace, st)),
+                ("fc2_alone", lambda: moe.moe_fc2(lay.plan, d["w2"], d["w2_scales"],
+                                                  lay.workspace, st))]
+
+    def prepare(self, warmup):
+        import torch
+        for _ in range(warmup):
+            self.fwd()
+        torch.cuda.synchronize()
+        if self.lay.check() != 0:
+            raise RuntimeError(f"device error during warm-up of {self.wl.name}")
+        # The timed step replays a CUDA graph of moe_forward (the same kernels
+        # with the same arguments; the routing kernel resets the GEMM
+        # scheduler's counters inside the graph, so every replay starts clean).
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.fwd()
+        torch.cuda.synchronize()
+
+    def soak(self, seconds):
+        import torch
+        t_end = time.perf_counter() + seconds
+        while time.perf_counter() < t_end:
+            for _ in range(20):
+                self.graph.replay()
+            torch.cuda.synchronize()
+
+    def timed(self, fn, steps, flush):
+        """Per-step device times (ms): CUDA events on the launching stream, L2
+        flushed before every step outside the events."""
+        import torch
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for i in range(steps):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(self.stream)
+            fn()
+            ev[i][1].record(self.stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in ev]
+
+    def split(self, steps, flush, unfused=False):
+        """Per-launch device times (ms) of the launch sequence, one event per
+        launch boundary on the launching stream."""
+        import torch
+        seqs = [self.steps()] + ([self.steps(unfused=True)] if unfused else [])
+        out = {name: [] for seq in seqs for name, _ in seq}
+        for seq in seqs:
+            for i in range(steps):
+                flush.fill_(i & 0xFF)
+                evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(seq) + 1)]
+                evs[0].record(self.stream)
+                for j, (_, fn) in enumerate(seq):
+                    fn()
+                    evs[j + 1].record(self.stream)
+                torch.cuda.synchronize()
+                for j, (name, _) in enumerate(seq):
+                    out[name].append(evs[j].elapsed_time(evs[j + 1]))
+        return out
+
+    def e2e(self, steps, warmup, flush):
+        """Device time (ms per step) through the host-buffer entry point: the
+        step's inputs copied in from pinned host memory and its output copied
+        back, every step, inside the events."""
+        import torch
+        moe, d, lay = self.moe, self.d, self.lay
+        host = {k: (None if d[k] is None else d[k].cpu().pin_memory())
+                for k in ("x", "x_scales", "topk_idx", "topk_w")}
+        out_h = torch.empty(self.wl.T, self.wl.H, dtype=torch.bfloat16).pin_memory()
+
+        def call():
+            moe.moe_forward_hostio(lay.plan, host["x"], host["x_scales"], host["topk_idx"],
+                                   host["topk_w"], d["w1"], d["w1_scales"], d["w2"],
+                                   d["w2_scales"], out_h, lay.workspace, self.stream)
+        for _ in range(warmup):
+            call()
+        torch.cuda.synchronize()
+        ms = self.timed(call, steps, flush)
+        h2d = int(sum(v.numel() * v.element_size() for v in host.values() if v is not None))
+        return ms, h2d, int(out_h.numel() * 2)
+
+    def release(self):
+        import torch
+        self.graph = None
+        self.lay = None
+        self.d = None
+        self.out = None
+        torch.cuda.empty_cache()
+
+
+def measure_rank(args, dev):
+    """This rank's measurements: the headline workload (timed steps, eager
+    steps, per-launch split, e2e, clocks) and a shorter record of every
+    configuration.  Returns plain numbers so that the line can be assembled
+    from any number of ranks (``assemble_line``)."""
+    import torch
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    rank, world, local = _dist()
+    wl = workload(args.workload, args.tokens)
+    lb = LayerBench(wl, args, dev, keep_row_major=(rank == 0 and not args.no_cpu_baseline))
+    lb.prepare(args.warmup)
+    clocks = Clocks(local)
+    clocks.start()
+    # The clock sampler needs ~100 ms per sample, longer than K steps take, so
+    # the timed steps sit between continuous (untimed) steps of the same layer.
+    lb.soak(0.6)
+    step_ms = lb.timed(lb.graph.replay, args.steps, flush)
+    lb.soak(0.3)
+    eager_ms = lb.timed(lb.fwd, args.steps, flush)
+    lb.soak(0.3)
+    split = lb.split(args.steps, flush, unfused=True)
+    lb.soak(0.3)
+    clk = clocks.stop()
+    e2e_ms, h2d, d2h = lb.e2e(args.steps, args.warmup, flush)
+    if lb.lay.check() != 0:
+        raise RuntimeError("device error during timing")
+    main = {"wl": wl, "step_ms": step_ms, "eager_ms": eager_ms, "split": split,
+            "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h, "clocks": clk, "active": lb.active,
+            "alg_bytes": lb.alg_bytes, "w_bytes": lb.w_bytes, "pairs": lb.pairs,
+            "tiled": lb.tiled, "chunked": lb.chunked,
+            "swap": lb.moe.moe_plan_swap_ab_active(lb.lay.plan),
+            "launches": lb.moe.moe_forward_launch_count(lb.lay.plan)}
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, lb.d_row_major, args)
+    lb.release()
+    per = []
+    if not args.no_per_config:
+        for name, tokens in PER_CONFIG:
+            w = workload(name, tokens)
+            b = LayerBench(w, args, dev)
+            b.prepare(min(args.warmup, 3))
+            c = Clocks(local)
+            c.start()
+            b.soak(0.3)
+            ms = b.timed(b.graph.replay, PER_CONFIG_STEPS, flush)
+            sp = b.split(PER_CONFIG_STEPS, flush)
+            b.soak(0.1)
+            cc = c.stop()
+            if b.lay.check() != 0:
+                raise RuntimeError(f"device error during timing of {w.name}")
+            per.append({"wl": w, "step_ms": ms, "split": sp, "active": b.active,
+                        "alg_bytes": b.alg_bytes, "w_bytes": b.w_bytes, "pairs": b.pairs,
+                        "clocks": cc})
+            b.release()
+    return main, per, cpu
+
+
+def assemble_line(args, world, device, main, per, cpu):
+    """The contract's JSON line from this rank's measurements: every time is
+    first replaced by its maximum over ranks (one all-reduce, the same on every
+    rank), so a replica job is as fast as its slowest rank and `value` counts
+    the tokens of all ranks (weak scaling)."""
+    wl = main["wl"]
+    steps = len(main["step_ms"])
+    # Every time on the line, as (key, local value); one all-reduce of them all.
+    keys = [("total", sum(main["step_ms"])), ("e2e", sum(main["e2e_ms"])),
+            ("eager", sum(main["eager_ms"]))]
+    keys += [(("split", k), statistics.mean(v)) for k, v in main["split"].items() if v]
+    for i, p in enumerate(per):
+        keys.append((("per", i, "total"), sum(p["step_ms"])))
+        keys += [(("per", i, k), statistics.mean(v)) for k, v in p["split"].items() if v]
+    red = dict(zip([k for k, _ in keys], max_over_ranks([v for _, v in keys], world, device)))
+    total_ms, e2e_total, eager_total = red["total"], red["e2e"], red["eager"]
+    split_ms = {k[1]: v for k, v in red.items() if isinstance(k, tuple) and k[0] == "split"}
+    gemm_ms = split_ms["fc1_fc2"]
+    ms_per_step = total_ms / steps
+    flops = 6.0 * wl.S * wl.H * wl.I
     res = {
-        "metric": METRIC, "value": round(replica_throughput(wl.T, world, total_ms, args.steps), 1),
-        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "metric": METRIC, "value": round(replica_throughput(wl.T, world, total_ms, steps), 1),
+        "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": {"e4m3": "fp8_e4m3", "e2m1": "fp8_e4m3xe2m1",
                                        "bf16": "bf16"}[wl.w_dtype],
         "data": "synthetic (seeded; random-init weights)",
-        "config": {**workload_config(wl, active), "l2": "flushed (256 MiB write) before each step",
-                   "weights": ("tiled (moe_prepack_weights, once)" if tiled else
+        "config": {**workload_config(wl, main["active"]),
+                   "l2": "flushed (256 MiB write) before each step",
+                   "weights": ("tiled (moe_prepack_weights, once)" if main["tiled"] else
                                "row-major codes, chunked scales (moe_prepack_weight_scales, once)"
-                               if chunked else "row-major"),
+                               if main["chunked"] else "row-major"),
                    "gemm_tiles": {0: "token rows", 1: "token-major (swap AB)",
                                   2: "token-major for tiles of <= 96 tokens, else token rows"}[
-                       moe.moe_plan_swap_ab_active(lay.plan)],
+                       main["swap"]],
                    "parallelism": f"replicas x{world}"},
         "achieved": {"tflops": round(flops / (ms_per_step * 1e-3) / 1e12, 2),
-                     "hbm_gbs": round(alg_bytes / (ms_per_step * 1e-3) / 1e9, 1),
-                     "alg_bytes": alg_bytes, "flops": flops},
-        "kernels_ms": {k: round(statistics.mean(v), 4) for k, v in split.items()},
-        "kernels_gbs": kernels_gbs(wl, split),
-        "eager_ms_per_step": round(sum(eager_ms) / args.steps, 4),
+                     "hbm_gbs": round(main["alg_bytes"] / (ms_per_step * 1e-3) / 1e9, 1),
+                     "alg_bytes": main["alg_bytes"], "flops": flops},
+        "kernels_ms": {k: round(v, 4) for k, v in split_ms.items()},
+        "kernels_gbs": kernels_gbs(wl, {k: [v] for k, v in split_ms.items()}),
+        "eager_ms_per_step": round(eager_total / steps, 4),
         "timing": "CUDA-graph replay of moe_forward, events on the launching stream",
-        "roofline": roof,
-        "e2e": {"value": round(replica_throughput(wl.T, world, e2e_total, args.steps), 1),
-                "unit": "tokens/s",
-                "h2d_bytes_per_step": int(sum(v.numel() * v.element_size() for v in host.values()
-                                              if v is not None)),
-                "d2h_bytes_per_step": int(out_h.numel() * 2)},
-        "gpu_launches": moe.moe_forward_launch_count(lay.plan) * args.steps,
-        "clocks": clk,
+        "roofline": roofline(wl, main["alg_bytes"], main["w_bytes"], main["active"], gemm_ms,
+                             main["pairs"]),
+        "e2e": {"value": round(replica_throughput(wl.T, world, e2e_total, steps), 1),
+                "unit": "tokens/s", "h2d_bytes_per_step": main["h2d"],
+                "d2h_bytes_per_step": main["d2h"]},
+        "gpu_launches": main["launches"] * steps,
+        "clocks": main["clocks"],
     }
-    if rank == 0 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(wl, d_row_major, args)
+    per_out = []
+    for i, p in enumerate(per):
+        w = p["wl"]
+        t_ms, g_ms = red[("per", i, "total")], red[("per", i, "fc1_fc2")]
+        n = len(p["step_ms"])
+        roof = roofline(w, p["alg_bytes"], p["w_bytes"], p["active"], g_ms, p["pairs"])
+        per_out.append({
+            "workload": w.name, "T": w.T, "w_dtype": w.w_dtype, "active_experts": p["active"],
+            "tokens_per_s": round(replica_throughput(w.T, world, t_ms, n), 1),
+            "ms_per_step": round(t_ms / n, 4), "fc1_fc2_ms": round(g_ms, 4),
+            "route_gather_ms": round(red[("per", i, "route_gather")], 4),
+            "combine_ms": round(red[("per", i, "combine")], 4),
+            "roofline": {k: roof[k] for k in ("bound", "achieved", "peak", "unit", "frac")},
+            "sm_mhz": p["clocks"].get("sm_mhz"), "reasons": p["clocks"].get("reasons"),
+            "steps": n})
+    if per_out:
+        res["per_config"] = per_out
+    if cpu is not None:
+        res["cpu_baseline"] = cpu
+    return res
+
+
+def run_b200(args):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from moe_expert_ffn_permute_b200.build import build
+
+    rank, world, local = _dist()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    if rank == 0:
+        build()
+    if world > 1:
+        dist.barrier()
+    import moe_expert_ffn_permute_b200 as moe
+    moe.lib()
+    dev = torch.device("cuda", local)
+    main, per, cpu = measure_rank(args, dev)
+    if world > 1:
+        dist.barrier()
+    res = assemble_line(args, world, dev, main, per, cpu)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -494,7 +616,7 @@ def run_reference(args, wl):
     from workloads.synth import make_inputs, to_numpy
     d = make_inputs(wl, device="cuda" if torch.cuda.is_available() else "cpu")
     dn = to_numpy(d)
-    ntok = args.cpu_tokens
+    ntok = args.ref_tokens
     for i in range(args.warmup):
         _oracle_sample(wl, dn, [i % wl.T])
     times = []
@@ -519,16 +641,36 @@ def run_reference(args, wl):
     print(json.dumps(res))
 
 
+def _respawn_under_torchrun(n):
+    """`--gpus N` without a launcher: start N ranks of this same command under
+    torch.distributed.run (one process per GPU) and return its exit code."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="decode")
-    ap.add_argument("--tokens", type=int, default=None, help="override T (mxfp4 sweep)")
+    ap.add_argument("--workload", default=HEADLINE[0])
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override T (the mxfp4 sweep); default: the headline's 32768 tokens "
+                         "for the mxfp4 workload")
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
-    ap.add_argument("--cpu-tokens", type=int, default=2)
+    ap.add_argument("--cpu-tokens", type=int, default=2,
+                    help="tokens of the oracle sample beside the GPU line (cpu_baseline)")
+    ap.add_argument("--ref-tokens", type=int, default=1,
+                    help="tokens per step of the oracle arm (--impl reference)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per-configuration record (headline workload only)")
     ap.add_argument("--cta-pairs", type=int, default=0, choices=[0, 1, 2],
                     help="GEMM on CTA pairs: 0 automatic, 1 never, 2 always (tiled FP8 only)")
     ap.add_argument("--swap-ab", type=int, default=0, choices=[0, 1, 2],
@@ -537,14 +679,19 @@ def main():
                     help="weights as given (row-major, 2-D TMA; MXFP4 scales unchunked) "
                          "instead of prepacked")
     args = ap.parse_args()
-    from workloads.synth import WORKLOADS
-    wl = WORKLOADS[args.workload]
-    if args.tokens:
-        wl = wl.with_tokens(args.tokens)
+    if args.tokens is None and args.workload == HEADLINE[0]:
+        args.tokens = HEADLINE[1]
+    world_env = os.environ.get("WORLD_SIZE")
+    if args.gpus > 1 and world_env is None:
+        sys.exit(_respawn_under_torchrun(args.gpus))
+    if world_env is not None and int(world_env) != args.gpus:
+        sys.exit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world_env}: launch one rank "
+                 f"per GPU (torch.distributed.run --nproc-per-node {args.gpus})")
+    wl = workload(args.workload, args.tokens)
     if args.impl == "reference":
         run_reference(args, wl)
     else:
-        run_b200(args, wl)
+        run_b200(args)
 
 
 if __name__ == "__main__":

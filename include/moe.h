@@ -248,8 +248,8 @@ moe_status moe_quantize_act(const void *x_bf16, int T, int H, uint8_t *x_codes,
 /* Allocation-free routing.  The pages have no counterpart of this entry point.
  *
  * Same result as moe_route() (counts i32[E], offsets i32[E+1], perm i32[S],
- * inv i32[S], all device pointers owned by the caller; out-of-range expert ids
- * give inv[s] = -1), but it needs no workspace and allocates nothing: its
+ * inv i32[S], all device pointers owned by the caller, 4-byte aligned), but
+ * it needs no workspace and allocates nothing: its
  * scratch (per-block histograms, tile offsets, an error word) is a ~515 KiB
  * array in the library's static device memory, which every GPU that loads the
  * library keeps until the process exits.  It is meant for callers that cannot
@@ -264,7 +264,16 @@ moe_status moe_quantize_act(const void *x_bf16, int T, int H, uint8_t *x_codes,
  *   - All calls share the one array and it keeps the last call's contents;
  *     the call clears what must start at zero.  Calls that overlap on the GPU
  *     (different streams, no ordering between them) race on the array and
- *     must not be issued.                                                   */
+ *     must not be issued.
+ *   - Expert ids outside [0, E) are handled as moe_route() handles them (the
+ *     slot is not routed: inv[s] = -1, -1 is a masked slot), but an id other
+ *     than -1 is NOT reported: this entry point has no workspace error word
+ *     for moe_check_device_error() to read, and reading its own would need a
+ *     device synchronisation.  Callers that must detect bad ids check
+ *     counts (sum < T*k) or inv themselves.
+ *   - Returns MOE_ERR_CUDA only for a failure of its own launches or copies;
+ *     an error left by an earlier, unrelated launch is neither reported nor
+ *     cleared.                                                              */
 #define MOE_ROUTE_STATIC_MAX_SLOTS (1 << 20)
 moe_status moe_route_static(const int32_t *topk_idx, int T, int k, int E,
                             int32_t *counts, int32_t *offsets, int32_t *perm,
@@ -397,7 +406,10 @@ moe_status moe_copy_act(moe_plan_t plan, const void *workspace, uint8_t *dst,
                         moe_stream_t stream);
 
 /* Debug flags (0 by default).  Bit 0: FC1 also writes the fp32 activation
- * before requantisation to act_f32 (costs bandwidth).  Bit 1: test hook for
+ * before requantisation to act_f32 (costs bandwidth); that buffer is placed at
+ * the end of the workspace, so setting or clearing bit 0 changes
+ * moe_workspace_bytes() (query it again and allocate at least that much
+ * before the next call) but moves no other buffer.  Bit 1: test hook for
  * the failure path -- in the fused FC1+FC2 launch (moe_fc1_fc2, moe_forward
  * without CTA pairs) every FC2 tile waits for one FC1 completion more than its
  * m-tile can provide, so that bounded wait runs out (about 2 s): the launch

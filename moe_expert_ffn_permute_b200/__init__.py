@@ -177,9 +177,40 @@ def moe_quantize_act(x_bf16, T, H, x_codes, x_scales, stream=None):
                                   _stream(stream)), "moe_quantize_act")
 
 
+def _expect_i32(name, t, numel):
+    """A tensor argument of moe_route_static: contiguous int32 on a CUDA device
+    with at least `numel` elements (the C ABI would otherwise write past its
+    end or read host memory).  Raw addresses are passed through unchecked."""
+    if t is None:
+        raise MoEError(MOE_ERR_INVALID_ARG, f"moe_route_static: {name} is required")
+    if isinstance(t, int):
+        return
+    import torch
+    if t.dtype != torch.int32:
+        raise MoEError(MOE_ERR_INVALID_ARG, f"moe_route_static: {name} must be int32, got {t.dtype}")
+    if not t.is_contiguous():
+        raise MoEError(MOE_ERR_INVALID_ARG, f"moe_route_static: {name} must be contiguous")
+    if t.numel() < numel:
+        raise MoEError(MOE_ERR_INVALID_ARG,
+                       f"moe_route_static: {name} holds {t.numel()} elements, needs {numel}")
+
+
 def moe_route_static(topk_idx, T, k, E, counts, offsets, perm, inv, stream=None):
     """Routing without a workspace: scratch lives in the library's static device
-    memory (at most MOE_ROUTE_STATIC_MAX_SLOTS slots; calls must not overlap)."""
+    memory (at most MOE_ROUTE_STATIC_MAX_SLOTS slots; calls must not overlap).
+    Expert ids outside [0, E) other than -1 are dropped without an error status."""
+    T, k, E = int(T), int(k), int(E)
+    if T >= 1 and k >= 1 and E >= 1 and T * k <= ROUTE_STATIC_MAX_SLOTS and E <= 256:
+        S = T * k
+        args = (("topk_idx", topk_idx, S), ("counts", counts, E), ("offsets", offsets, E + 1),
+                ("perm", perm, S), ("inv", inv, S))
+        for name, t, n in args:
+            _expect_i32(name, t, n)
+        for name, t, _ in args:
+            if not isinstance(t, int) and not t.is_cuda:
+                raise MoEError(MOE_ERR_INVALID_ARG,
+                               f"moe_route_static: {name} must be on a CUDA device")
+    # Sizes out of range are refused by the library itself (nothing enqueued).
     _check(lib().moe_route_static(_ptr(topk_idx), T, k, E, *map(_ptr, (counts, offsets, perm,
                                                                          inv)),
                                   _stream(stream)), "moe_route_static")

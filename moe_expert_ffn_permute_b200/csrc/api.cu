@@ -2,11 +2,46 @@
 // workspace layout, and the stream-ordered launch sequence of the layer.
 #include <cmath>
 #include <cstring>
+#include <mutex>
 #include <new>
+#include <utility>
+#include <vector>
 
 #include "internal.h"
 
 namespace moe {
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_device_mu;
+int g_sm_count[kMaxDevices] = {};
+std::vector<std::pair<const void*, int>> g_smem_set;   // (kernel, device) done
+}  // namespace
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  std::lock_guard<std::mutex> lock(g_device_mu);
+  if (g_sm_count[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    g_sm_count[dev] = n;
+  }
+  return g_sm_count[dev];
+}
+
+cudaError_t ensure_max_dynamic_smem(const void* kernel, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_device_mu);
+  for (const auto& kd : g_smem_set)
+    if (kd.first == kernel && kd.second == dev) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) g_smem_set.emplace_back(kernel, dev);
+  return e;
+}
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -39,7 +74,6 @@ void compute_layout(moe_plan_s* p) {
   L.xg_sf = take(bf16 ? 0 : rows / kTileM * (p->H / 128) * 512);
   L.act = take(rows * p->I * elem);
   L.act_sf = take(bf16 ? 0 : rows / kTileM * (p->I / 128) * 512);
-  L.act_f32 = take(p->debug_act_f32 ? rows * p->I * 4 : 0);
   L.y = take(S * p->H * 2);
   // One 1 KB record per (expert, n-tile, k-block) of each GEMM: the two 128-row
   // weight blocks of a 256-wide tile, each block's scale byte repeated 512 times.
@@ -51,6 +85,8 @@ void compute_layout(moe_plan_s* p) {
   L.in_idx = take(S * 4);
   L.in_w = take(S * 4);
   L.out_stage = take(static_cast<size_t>(p->T) * p->H * 2);
+  // Debug capture last: switching it on or off moves no other buffer.
+  L.act_f32 = take(p->debug_act_f32 ? rows * p->I * 4 : 0);
   L.total = off;
 }
 

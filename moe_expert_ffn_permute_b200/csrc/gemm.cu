@@ -907,17 +907,6 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
   return r == CUDA_SUCCESS;
 }
 
-int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
-
 template <int kW>
 cudaError_t launch_gemm(const moe_plan_s* pl, int phases, bool dynamic, const void* w1,
                         const uint8_t* w1s, const void* w2, const uint8_t* w2s, uint8_t* ws,
@@ -979,14 +968,10 @@ cudaError_t launch_gemm(const moe_plan_s* pl, int phases, bool dynamic, const vo
   p.err = reinterpret_cast<uint32_t*>(ws + L.err);
   const size_t smem = sizeof(Smem) + 1024;
   auto kern = moe_gemm_kernel<kW>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  const int grid = static_cast<int>(std::min<long long>(num_sms(), max_tiles));
+  cudaError_t e = ensure_max_dynamic_smem(reinterpret_cast<const void*>(kern),
+                                          static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int grid = static_cast<int>(std::min<long long>(sm_count(), max_tiles));
   return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, maps[0], maps[1], maps[2],
                     maps[3], p);
 }

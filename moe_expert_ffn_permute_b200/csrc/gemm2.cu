@@ -543,17 +543,6 @@ bool map_rows(CUtensorMap* m, const void* base, uint64_t bytes, uint32_t width,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int num_sms2() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
-
 }  // namespace
 
 size_t gemm_pair_smem_bytes() { return sizeof(Smem) + 1024; }
@@ -630,7 +619,7 @@ cudaError_t launch_fc12_pairs(const moe_plan_s* pl, const void* w1, const uint8_
     return cudaErrorInvalidValue;
 
   const uint64_t units = (sfb1_bytes + sfb2_bytes) / 16;
-  const int xblocks = static_cast<int>(std::min<uint64_t>((units + 255) / 256, 4ull * num_sms2()));
+  const int xblocks = static_cast<int>(std::min<uint64_t>((units + 255) / 256, 4ull * static_cast<uint64_t>(sm_count())));
   cudaError_t e = launch_pdl(expand_pair_scales_kernel, dim3(xblocks), dim3(256), 0, st, w1s, w2s,
                              reinterpret_cast<uint4*>(ws + L.pair_sf1),
                              reinterpret_cast<uint4*>(ws + L.pair_sf2), pl->E, pl->I, pl->H);
@@ -659,15 +648,11 @@ cudaError_t launch_fc12_pairs(const moe_plan_s* pl, const void* w1, const uint8_
   p.y = reinterpret_cast<uint16_t*>(ws + L.y);
   p.err = reinterpret_cast<uint32_t*>(ws + L.err);
   const size_t smem = sizeof(Smem) + 1024;
-  static bool attr_set = false;
-  if (!attr_set) {
-    e = cudaFuncSetAttribute(moe_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  e = ensure_max_dynamic_smem(reinterpret_cast<const void*>(moe_gemm_pair_kernel),
+                              static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
   const long long max_pairs = (pl->rows_cap / kTileM + 1) / 2 * (pl->H / 256 + pl->I / 128);
-  const int clusters = static_cast<int>(std::min<long long>(num_sms2() / 2, max_pairs));
+  const int clusters = static_cast<int>(std::min<long long>(sm_count() / 2, max_pairs));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters);
   cfg.blockDim = dim3(kThreads);

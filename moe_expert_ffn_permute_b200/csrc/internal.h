@@ -74,7 +74,30 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-// Kernel launchers (return cudaGetLastError()).
+// Launch without attributes.  Returns this launch's own status: unlike
+// cudaGetLastError() after a <<<>>> launch, it neither reports nor clears an
+// error left behind by some earlier, unrelated launch.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_plain(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                         cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = nullptr;
+  cfg.numAttrs = 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Streaming multiprocessors of the current device (looked up once per device;
+// thread-safe).
+int sm_count();
+// Raise a kernel's dynamic shared-memory limit to `bytes` on the current
+// device, once per (kernel, device); thread-safe.
+cudaError_t ensure_max_dynamic_smem(const void* kernel, int bytes);
+
+// Kernel launchers (each returns the status of its own launches).
 cudaError_t launch_route(const moe_plan_s* p, const int32_t* topk_idx, uint8_t* ws,
                          cudaStream_t st);
 // Routing and gather fused in one launch (slot counts up to kFusedMaxSlots).

@@ -74,25 +74,24 @@ int blocks_for(long long n) {
 cudaError_t launch_prepack(const uint8_t* src, long long rows, int K, uint8_t* dst,
                            cudaStream_t st) {
   const long long n = rows * (K / 16);
-  prepack_kernel<<<blocks_for(n), 256, 0, st>>>(reinterpret_cast<const uint4*>(src), rows, K, dst);
-  return cudaGetLastError();
+  return launch_plain(prepack_kernel, dim3(blocks_for(n)), dim3(256), 0, st,
+                      reinterpret_cast<const uint4*>(src), rows, K, dst);
 }
 
 cudaError_t launch_prepack_fp4_scales(const uint8_t* src, long long rows, int K, uint8_t* dst,
                                       cudaStream_t st) {
   const int kb_n = K / 128;
-  prepack_fp4_scales_kernel<<<blocks_for(rows * kb_n), 256, 0, st>>>(
-      reinterpret_cast<const uint32_t*>(src), rows, kb_n, dst);
-  return cudaGetLastError();
+  return launch_plain(prepack_fp4_scales_kernel, dim3(blocks_for(rows * kb_n)), dim3(256), 0, st,
+                      reinterpret_cast<const uint32_t*>(src), rows, kb_n, dst);
 }
 
 cudaError_t launch_unpack_act(const moe_plan_s* p, const uint8_t* ws, uint8_t* dst,
                               cudaStream_t st) {
   const int row_bytes = p->I * (p->w_dtype == MOE_W_BF16 ? 2 : 1);
   const long long n = p->rows_cap * (row_bytes / 16);
-  unpack_kernel<<<blocks_for(n), 256, 0, st>>>(ws + p->ws.act, p->rows_cap, row_bytes,
-                                               reinterpret_cast<uint4*>(dst));
-  return cudaGetLastError();
+  return launch_plain(unpack_kernel, dim3(blocks_for(n)), dim3(256), 0, st,
+                      static_cast<const uint8_t*>(ws + p->ws.act), p->rows_cap, row_bytes,
+                      reinterpret_cast<uint4*>(dst));
 }
 
 }  // namespace moe

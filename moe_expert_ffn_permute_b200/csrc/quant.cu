@@ -60,7 +60,8 @@ extern "C" moe_status moe_quantize_act(const void* x_bf16, int T, int H, uint8_t
   const long long blocks = static_cast<long long>(T) * (H / 128);
   const long long threads = blocks * 16;
   const int grid = static_cast<int>((threads + 255) / 256);
-  moe::quantize_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+  const cudaError_t e = moe::launch_plain(
+      moe::quantize_kernel, dim3(grid), dim3(256), 0, reinterpret_cast<cudaStream_t>(stream),
       static_cast<const uint4*>(x_bf16), blocks, reinterpret_cast<uint2*>(x_codes), x_scales);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -470,12 +470,7 @@ cudaError_t launch_route_gather(const moe_plan_s* p, const int32_t* topk_idx, co
   const auto& L = p->ws;
   const int S = static_cast<int>(p->S);
   // One warp per routed row (at most S), two blocks per SM at most.
-  int sms = 148;
-  {
-    int dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  }
+  const int sms = sm_count();
   const bool bf16 = p->w_dtype == MOE_W_BF16;   // 2-byte activations, no scales
   const int want = (S + kRouteThreads / 32 - 1) / (kRouteThreads / 32);
   const int blocks = std::max(1, std::min(want, 2 * sms));
@@ -495,9 +490,8 @@ cudaError_t launch_unpack_act_scales(const moe_plan_s* p, const uint8_t* ws, uin
                                      cudaStream_t st) {
   const long long n = p->rows_cap * (p->I / 128);
   const int blocks = static_cast<int>((n + 255) / 256);
-  unpack_act_scales_kernel<<<blocks, 256, 0, st>>>(ws + p->ws.act_sf, p->I / 128, p->rows_cap,
-                                                   dst);
-  return cudaGetLastError();
+  return launch_plain(unpack_act_scales_kernel, dim3(blocks), dim3(256), 0, st,
+                      static_cast<const uint8_t*>(ws + p->ws.act_sf), p->I / 128, p->rows_cap, dst);
 }
 
 }  // namespace moe
@@ -578,12 +572,17 @@ extern "C" moe_status moe_route_static(const int32_t* topk_idx, int T, int k, in
   if (cudaMemsetAsync(scratch + kStaticErrOff, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
   auto err = reinterpret_cast<uint32_t*>(scratch + kStaticErrOff);
   auto hist = reinterpret_cast<int32_t*>(scratch + kStaticHistOff);
-  if (nblk > 1)
-    route_hist_kernel<<<nblk, kRouteThreads, 0, st>>>(topk_idx, static_cast<int>(S), E, hist, err);
-  route_scatter_kernel<<<nblk, kRouteThreads, 0, st>>>(
-      topk_idx, static_cast<int>(S), E, nblk, hist, counts, offsets,
+  // Each launch's own status is checked (an earlier, unrelated launch error is
+  // neither reported here nor cleared).
+  if (nblk > 1 &&
+      launch_plain(route_hist_kernel, dim3(nblk), dim3(kRouteThreads), 0, st, topk_idx,
+                   static_cast<int>(S), E, hist, err) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const cudaError_t e = launch_plain(
+      route_scatter_kernel, dim3(nblk), dim3(kRouteThreads), 0, st, topk_idx,
+      static_cast<int>(S), E, nblk, static_cast<const int32_t*>(hist), counts, offsets,
       reinterpret_cast<int32_t*>(scratch + kStaticTileOff),
-      reinterpret_cast<int32_t*>(scratch + kStaticPadOff), nullptr, perm, inv, err, nullptr, 0,
-      nullptr, k);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+      reinterpret_cast<int32_t*>(scratch + kStaticPadOff), static_cast<int32_t*>(nullptr), perm,
+      inv, err, static_cast<uint32_t*>(nullptr), 0, static_cast<int32_t*>(nullptr), k);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -80,3 +80,27 @@ def oracle_tokens(wl, dn, tokens, keep=False):
 
 def inputs(wl, device="cuda", seed=None):
     return make_inputs(wl, device=device, seed=seed)
+
+
+def bench_layer(wl, d, swap=None):
+    """The layer in the launch configuration bench.py times: FP8 / BF16 weights
+    prepacked into tiles, MXFP4 scales prepacked into chunks, automatic tile
+    orientation (unless `swap` forces one).  Returns (layer, weights dict)."""
+    tiled = wl.w_dtype in ("e4m3", "bf16")
+    chunked = wl.w_dtype == "e2m1"
+    lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype=wl.w_dtype, act=wl.act,
+                       alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit,
+                       tiled_weights=tiled, chunked_scales=chunked, swap_ab=swap)
+    w = {k: d[k] for k in ("w1", "w1_scales", "w2", "w2_scales")}
+    if tiled:
+        w["w1"], w["w2"] = lay.prepack(d["w1"], d["w2"])
+    if chunked:
+        w["w1_scales"], w["w2_scales"] = lay.prepack_scales(d["w1_scales"], d["w2_scales"])
+    return lay, w
+
+
+def bench_forward(lay, w, d, out=None):
+    out = lay.forward(d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], w["w1"],
+                      w["w1_scales"], w["w2"], w["w2_scales"], out=out)
+    torch.cuda.synchronize()
+    return out

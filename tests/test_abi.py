@@ -221,3 +221,26 @@ def test_fp4_chunked_scale_layout_rules():
     assert ei.value.status == 3
     moe.moe_plan_destroy(p)
     moe.moe_plan_destroy(q)
+
+
+def test_debug_capture_moves_no_other_buffer():
+    """Switching the fp32 debug capture on grows the workspace at its end only:
+    every other buffer keeps its offset (a workspace sized before the switch is
+    still valid for all of them)."""
+    fake = 1 << 30                                     # any 256-B aligned address
+    for w_dtype in ("e4m3", "e2m1", "bf16"):
+        p = moe.moe_plan(300, 1024, 512, 8, 4, w_dtype=w_dtype)
+        before = moe.moe_workspace_bytes(p)
+        v0 = moe.moe_workspace_view(p, fake)
+        moe.moe_plan_set_debug(p, 1)
+        after = moe.moe_workspace_bytes(p)
+        v1 = moe.moe_workspace_view(p, fake)
+        names = ("counts", "offsets", "perm", "inv", "pad_offsets", "act", "y", "error_word")
+        for name in names:
+            assert getattr(v0, name) == getattr(v1, name), (w_dtype, name)
+        assert v0.act_f32 is None and v1.act_f32 is not None
+        assert v1.act_f32 - fake >= before - 256          # placed after everything else
+        assert after - before >= v1.rows * 512 * 4
+        moe.moe_plan_set_debug(p, 0)
+        assert moe.moe_workspace_bytes(p) == before
+        moe.moe_plan_destroy(p)

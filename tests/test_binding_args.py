@@ -83,3 +83,30 @@ def test_layer_forward_checks_before_the_call(monkeypatch, w_dtype):
     with pytest.raises(moe.MoEError):
         lay.forward(*args)
     assert len(calls) == 1
+
+
+def test_route_static_refuses_bad_tensors_before_the_call():
+    """moe_route_static's binding checks dtype, contiguity, size and device of
+    its five tensors before the C call (which would otherwise write past a
+    short buffer); every refusal happens on the host."""
+    import torch
+    T, k, E = 16, 2, 8
+    S = T * k
+    good = dict(topk_idx=torch.zeros(S, dtype=torch.int32), counts=torch.zeros(E, dtype=torch.int32),
+                offsets=torch.zeros(E + 1, dtype=torch.int32), perm=torch.zeros(S, dtype=torch.int32),
+                inv=torch.zeros(S, dtype=torch.int32))
+    order = ("topk_idx", "counts", "offsets", "perm", "inv")
+
+    def call(**kw):
+        a = dict(good, **kw)
+        with pytest.raises(moe.MoEError) as ei:
+            moe.moe_route_static(a["topk_idx"], T, k, E, *(a[n] for n in order[1:]))
+        assert ei.value.status == moe.MOE_ERR_INVALID_ARG
+        return str(ei.value)
+
+    assert "int32" in call(counts=torch.zeros(E, dtype=torch.int64))
+    assert "needs 9" in call(offsets=torch.zeros(E, dtype=torch.int32))
+    assert "needs 32" in call(perm=torch.zeros(S - 1, dtype=torch.int32))
+    assert "contiguous" in call(inv=torch.zeros(S, 2, dtype=torch.int32)[:, 0])
+    assert "required" in call(topk_idx=None)
+    assert "CUDA device" in call()                     # right shapes, but host tensors

@@ -7,7 +7,8 @@ import torch
 import moe_expert_ffn_permute_b200 as moe
 from oracle import layer as L
 
-from gpu_helpers import ensure_built
+from gpu_helpers import assert_parity, ensure_built
+from workloads.synth import Workload, make_inputs, to_numpy
 
 pytestmark = pytest.mark.gpu
 
@@ -39,14 +40,28 @@ def test_quantize_matches_oracle_bytes(T, H, scale):
 
 
 def test_quantize_feeds_the_layer():
-    """Quantising with the kernel and running the layer equals running the layer
-    on the same codes quantised by the oracle."""
+    """bf16 activations quantised by the kernel, then the whole layer on those
+    codes, against the oracle layer on the oracle quantiser's codes of the same
+    bf16 values (the two quantisations are byte-identical, checked first)."""
     ensure_built()
-    T, H = 64, 512
-    x = torch.randn(T, H, device="cuda").to(torch.bfloat16)
+    wl = Workload("quant-chain", 96, 512, 256, 8, 2, cfg_id=42)
+    d = make_inputs(wl, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(42)
+    x = (torch.randn(wl.T, wl.H, generator=g, device="cuda") * 2.0).to(torch.bfloat16)
     codes, scales = _quant_gpu(x)
     ref_codes, ref_scales = L.requant_1x128(x.float().cpu().numpy().astype(np.float64))
-    assert (codes == ref_codes).all() and (scales == ref_scales).all()
+    np.testing.assert_array_equal(codes, ref_codes)
+    np.testing.assert_array_equal(scales, ref_scales)
+    lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k)
+    out = lay.forward(torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda(),
+                      d["topk_idx"], d["topk_w"], d["w1"], d["w1_scales"], d["w2"],
+                      d["w2_scales"])
+    torch.cuda.synchronize()
+    assert lay.check() == 0
+    dn = to_numpy(d)
+    ref = L.layer(ref_codes, ref_scales, dn["topk_idx"], dn["topk_w"], dn["w1"],
+                  dn["w1_scales"], dn["w2"], dn["w2_scales"])
+    assert_parity(out.float().cpu().numpy(), ref, "quantised input chain")
 
 
 def test_quantize_rejects_bad_shapes():

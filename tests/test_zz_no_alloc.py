@@ -66,3 +66,17 @@ def test_static_route_rejects_sizes_beyond_its_scratch():
     with pytest.raises(moe.MoEError) as ei:
         moe.moe_route_static(idx, T, k, E, idx, idx, idx, idx)
     assert ei.value.status == 2          # MOE_ERR_UNSUPPORTED, nothing enqueued
+
+
+def test_static_route_drops_a_bad_id_without_a_status():
+    """An expert id outside [0, E) (other than -1) leaves its slot unrouted
+    (inv = -1, not counted) and, as documented, is not reported: the call
+    returns MOE_OK because this entry point has no error word to read back."""
+    ensure_built()
+    T, k, E = 64, 4, 16
+    idx = torch.randint(0, E, (T, k), dtype=torch.int32, device="cuda")
+    idx[3, 1] = E + 3
+    idx[9, 0] = -1
+    got = _static_route(idx, T, k, E)
+    assert int(got["inv"][3 * k + 1]) == -1 and int(got["inv"][9 * k]) == -1
+    assert int(got["counts"].sum()) == T * k - 2
