@@ -16,9 +16,11 @@ device time is the maximum over ranks.
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
 on the launching stream; L2 is flushed (a 256 MiB buffer is overwritten)
-before every timed step, outside the events.  `e2e` times the same layer
-through the C ABI's host-buffer entry point (pinned host inputs copied in,
-output copied back, all inside the events).
+before every timed step, outside the events.  `e2e` times K steps through the
+C ABI's host-buffer entry point (moe_forward_hostio_batches: every step's
+pinned host inputs copied in and its output copied back, overlapped with the
+neighbouring steps' layers, all inside the events; the weights are larger
+than L2).
 
 `--impl reference` times the float64 CPU oracle on the host cores instead (a
 bounded sample of the workload's tokens per step) and prints the same line.
@@ -238,7 +240,7 @@ def roofline(wl, alg_bytes, w_bytes, active, gemm_ms, pairs=False):
     ones count 6*S*H*I FLOP against the measured sustained bf16 GEMM rate (x2
     for FP8 and FP8 x FP4 operands: the GEMM time comes from continuous steps,
     the sustained power-capped state)."""
-    hbm, _, bf16_sus, peak_src = _peaks()
+    hbm, bf16_burst, bf16_sus, peak_src = _peaks()
     flops = 6.0 * wl.S * wl.H * wl.I
     tc_mult = 1.0 if wl.w_dtype == "bf16" else 2.0
     hbm_bound = alg_bytes / (hbm * 1e9) > flops / (tc_mult * bf16_sus * 1e12)
@@ -249,6 +251,10 @@ def roofline(wl, alg_bytes, w_bytes, active, gemm_ms, pairs=False):
         roof = {"bound": "tensor", "achieved": round(flops / (gemm_ms * 1e-3) / 1e12, 1),
                 "peak": round(tc_mult * bf16_sus, 1), "unit": "TFLOP/s"}
     roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
+    if not hbm_bound:
+        # For a kernel whose clock stayed near its maximum (no power capping
+        # in the samples) the burst figure is the closer denominator.
+        roof["frac_of_burst_peak"] = round(roof["achieved"] / (tc_mult * bf16_burst), 4)
     roof["traffic"] = measured_traffic(wl.name)
     roof["kernel"] = (("moe_gemm_pair_kernel (CTA pairs, 2-SM MMA; with its weight-scale "
                        "expansion launch)" if pairs else "moe_gemm_kernel") +
@@ -275,7 +281,7 @@ class LayerBench:
         from workloads.synth import make_inputs
         self.moe, self.wl, self.args, self.dev = moe, wl, args, dev
         d = make_inputs(wl, device=dev)
-        self.tiled = wl.w_dtype in ("e4m3", "bf16") and not args.row_major_weights
+        self.tiled = not args.row_major_weights      # FP8/BF16 tiles; MXFP4 code tiles
         self.chunked = wl.w_dtype == "e2m1" and not args.row_major_weights
         self.lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype=wl.w_dtype, act=wl.act,
                                 alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit, device=dev,
@@ -297,10 +303,13 @@ class LayerBench:
         self.graph = None
 
     def fwd(self):
+        """moe_forward on the current stream (inside graph capture: the capture
+        stream, so that the graph records the launches)."""
+        import torch
         d = self.d
         self.moe.moe_forward(self.lay.plan, d["x"], d["x_scales"], d["topk_idx"], d["topk_w"],
                              d["w1"], d["w1_scales"], d["w2"], d["w2_scales"], self.out,
-                             self.lay.workspace, self.stream)
+                             self.lay.workspace, torch.cuda.current_stream())
 
     def steps(self, unfused=False):
         """The launch sequence of moe_forward one call per step (route+gather,
@@ -336,6 +345,13 @@ class LayerBench:
         with torch.cuda.graph(self.graph):
             self.fwd()
         torch.cuda.synchronize()
+        # The replay must run the layer: a graph that captured nothing would
+        # time an empty replay.  One replay into a poisoned output proves it.
+        self.out.fill_(float("nan"))
+        self.graph.replay()
+        torch.cuda.synchronize()
+        if bool(torch.isnan(self.out).any()):
+            raise RuntimeError(f"graph replay of {self.wl.name} did not recompute the output")
 
     def soak(self, seconds):
         import torch
@@ -379,25 +395,33 @@ class LayerBench:
         return out
 
     def e2e(self, steps, warmup, flush):
-        """Device time (ms per step) through the host-buffer entry point: the
+        """Device time (ms per step) through the host-buffer entry point: every
         step's inputs copied in from pinned host memory and its output copied
-        back, every step, inside the events."""
+        back, all inside the events (moe_forward_hostio_batches: the copies of
+        one step overlap the layer of the neighbouring steps)."""
         import torch
         moe, d, lay = self.moe, self.d, self.lay
         host = {k: (None if d[k] is None else d[k].cpu().pin_memory())
                 for k in ("x", "x_scales", "topk_idx", "topk_w")}
         out_h = torch.empty(self.wl.T, self.wl.H, dtype=torch.bfloat16).pin_memory()
 
-        def call():
-            moe.moe_forward_hostio(lay.plan, host["x"], host["x_scales"], host["topk_idx"],
-                                   host["topk_w"], d["w1"], d["w1_scales"], d["w2"],
-                                   d["w2_scales"], out_h, lay.workspace, self.stream)
-        for _ in range(warmup):
-            call()
+        def call(n):
+            moe.moe_forward_hostio_batches(
+                lay.plan, [host["x"]] * n,
+                None if host["x_scales"] is None else [host["x_scales"]] * n,
+                [host["topk_idx"]] * n, [host["topk_w"]] * n, d["w1"], d["w1_scales"], d["w2"],
+                d["w2_scales"], [out_h] * n, lay.workspace, self.stream)
+        call(max(warmup, 1))
         torch.cuda.synchronize()
-        ms = self.timed(call, steps, flush)
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(self.stream)
+        call(steps)
+        b.record(self.stream)
+        torch.cuda.synchronize()
+        total = a.elapsed_time(b)
         h2d = int(sum(v.numel() * v.element_size() for v in host.values() if v is not None))
-        return ms, h2d, int(out_h.numel() * 2)
+        return [total / steps] * steps, h2d, int(out_h.numel() * 2)
 
     def release(self):
         import torch
@@ -495,9 +519,10 @@ def assemble_line(args, world, device, main, per, cpu):
         "data": "synthetic (seeded; random-init weights)",
         "config": {**workload_config(wl, main["active"]),
                    "l2": "flushed (256 MiB write) before each step",
-                   "weights": ("tiled (moe_prepack_weights, once)" if main["tiled"] else
-                               "row-major codes, chunked scales (moe_prepack_weight_scales, once)"
-                               if main["chunked"] else "row-major"),
+                   "weights": ("tiled codes and chunked scales (moe_prepack_weights and "
+                               "moe_prepack_weight_scales, once)" if main["chunked"] else
+                               "tiled (moe_prepack_weights, once)" if main["tiled"] else
+                               "row-major"),
                    "gemm_tiles": {0: "token rows", 1: "token-major (swap AB)",
                                   2: "token-major for tiles of <= 96 tokens, else token rows"}[
                        main["swap"]],

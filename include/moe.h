@@ -164,6 +164,35 @@ moe_status moe_forward_hostio(moe_plan_t plan, const void *x_host,
                               const uint8_t *w2_scales, void *out_host,
                               void *workspace, moe_stream_t stream);
 
+/* n_batches consecutive layers with their activations on the HOST, pipelined:
+ * batch i's inputs (x_host[i], x_scales_host[i], topk_idx_host[i],
+ * topk_w_host[i]; the layouts of moe_forward) are copied in while batch i-1
+ * computes, and batch i's output (out_host[i], bf16 [T,H]) is copied back while
+ * batch i+1 computes.  The copies run on two streams the plan creates on its
+ * first such call on a device (released by moe_plan_destroy); the layers run
+ * on `stream`, in order.  Work enqueued on `stream` before the call comes
+ * first, and `stream` completes only after every output has landed: the
+ * outputs are valid once `stream` has been synchronised.  Host buffers should
+ * be pinned (pageable memory works, without overlap); out_host entries may
+ * repeat (each batch's copy lands after the previous one).  The workspace
+ * holds two staging sets, so consecutive batches never wait for one another's
+ * copies.  Two calls with the same plan must be ordered on one stream.
+ * Results are byte-identical to moe_forward on the same inputs.
+ * Errors: MOE_ERR_INVALID_ARG for n_batches < 1 or a NULL array or entry
+ * (x_scales_host may be NULL for MOE_W_BF16), checked before anything is
+ * enqueued; MOE_ERR_CUDA if creating the copy streams or an enqueue fails.
+ * No counterpart on the pages (a host-buffer serving loop around
+ * moe_forward).
+ */
+moe_status moe_forward_hostio_batches(moe_plan_t plan, int n_batches,
+                                      const void *const *x_host,
+                                      const uint8_t *const *x_scales_host,
+                                      const int32_t *const *topk_idx_host,
+                                      const float *const *topk_w_host, const void *w1,
+                                      const uint8_t *w1_scales, const void *w2,
+                                      const uint8_t *w2_scales, void *const *out_host,
+                                      void *workspace, moe_stream_t stream);
+
 /* ---- The steps of moe_forward, callable one by one (same workspace). ---- */
 
 /* Step 1, routing: per-expert histogram, exclusive scan and stable scatter of
@@ -324,7 +353,11 @@ typedef enum {
   /* MXFP4 only: the E2M1 codes stay row-major (read by TMA, which widens them),
    * w1_scales / w2_scales are the output of moe_prepack_weight_scales(),
    * 16-byte aligned.                                                          */
-  MOE_WEIGHTS_SCALES_CHUNKED = 2
+  MOE_WEIGHTS_SCALES_CHUNKED = 2,
+  /* MXFP4 only: the E2M1 codes are the output of moe_prepack_weights() (8 KB
+   * tiles, one contiguous stream per k-block of 128 weight rows) and the
+   * scales that of moe_prepack_weight_scales().  The fastest MXFP4 layout.   */
+  MOE_WEIGHTS_TILED_SCALES_CHUNKED = 3
 } moe_weight_layout;
 moe_status moe_plan_set_weight_layout(moe_plan_t plan, int layout);
 
@@ -388,7 +421,11 @@ int moe_plan_swap_ab_active(moe_plan_t plan);
  * row (K for FP8, 2K for BF16), tile (b, kb) -- rows 128b..128b+127 of the
  * [E*2I, H] (or [E*H, I]) matrix, bytes 128kb..128kb+127 of each row -- is
  * 16384 bytes at offset (b * KB/128 + kb) * 16384, and byte c of tile row r
- * lies at r*128 + ((c/16) XOR (r%8))*16 + c%16.  Done once per weight set
+ * lies at r*128 + ((c/16) XOR (r%8))*16 + c%16.  MXFP4 plans: the packed E2M1
+ * codes w1 u8 [E,2I,H/2], w2 u8 [E,H,I/2] go to 8192-byte tiles of 128 rows x
+ * 64 bytes (128 codes): with KB = K/2, tile (b, kb) at (b * KB/64 + kb) * 8192
+ * holds byte c of row r (bytes 64kb..64kb+63 of the row) at r*64 + c, no
+ * swizzle (layout MOE_WEIGHTS_TILED_SCALES_CHUNKED).  Done once per weight set
  * (e.g. at model load), enqueued on `stream`.
  * No counterpart on the pages (a storage layout for this library's tensor-
  * core kernels).

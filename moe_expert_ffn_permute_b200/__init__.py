@@ -54,6 +54,7 @@ _SIGS = {
     "moe_workspace_bytes": (ctypes.c_size_t, [_P]),
     "moe_forward": (ctypes.c_int, [_P] * 12),
     "moe_forward_hostio": (ctypes.c_int, [_P] * 12),
+    "moe_forward_hostio_batches": (ctypes.c_int, [_P, ctypes.c_int] + [_P] * 11),
     "moe_route": (ctypes.c_int, [_P] * 4),
     "moe_route_gather": (ctypes.c_int, [_P] * 6),
     "moe_quantize_act": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int, _P, _P, _P]),
@@ -167,6 +168,38 @@ def moe_forward_hostio(plan, x_host, x_scales_host, topk_idx_host, topk_w_host, 
                                     _stream(stream)), "moe_forward_hostio")
 
 
+def _ptr_array(items):
+    """A C array of addresses (void *[]) for a list of tensors / addresses;
+    None if `items` is None."""
+    if items is None:
+        return None
+    arr = (ctypes.c_void_p * len(items))(*[_ptr(v) for v in items])
+    return ctypes.cast(arr, ctypes.c_void_p).value, arr
+
+
+def moe_forward_hostio_batches(plan, x_host, x_scales_host, topk_idx_host, topk_w_host, w1,
+                               w1_scales, w2, w2_scales, out_host, workspace, stream=None):
+    """len(x_host) consecutive layers on host buffers (lists of pinned tensors or
+    addresses, one entry per batch; x_scales_host None for BF16 plans), copies
+    overlapped with the layers; outputs valid after the stream is synchronised."""
+    n = len(x_host)
+    for name, lst in (("x_scales_host", x_scales_host), ("topk_idx_host", topk_idx_host),
+                      ("topk_w_host", topk_w_host), ("out_host", out_host)):
+        if lst is not None and len(lst) != n:
+            raise MoEError(MOE_ERR_INVALID_ARG,
+                           f"moe_forward_hostio_batches: {name} has {len(lst)} entries, "
+                           f"x_host has {n}")
+    arrays = [_ptr_array(v) for v in (x_host, x_scales_host, topk_idx_host, topk_w_host)]
+    outs = _ptr_array(out_host)
+    keep = [a for a in arrays + [outs] if a is not None]   # alive until the call returns
+    addr = [None if a is None else a[0] for a in arrays]
+    _check(lib().moe_forward_hostio_batches(plan, n, addr[0], addr[1], addr[2], addr[3],
+                                            *map(_ptr, (w1, w1_scales, w2, w2_scales)),
+                                            None if outs is None else outs[0], _ptr(workspace),
+                                            _stream(stream)), "moe_forward_hostio_batches")
+    del keep
+
+
 def moe_route(plan, topk_idx, workspace, stream=None):
     _check(lib().moe_route(plan, _ptr(topk_idx), _ptr(workspace), _stream(stream)), "moe_route")
 
@@ -262,7 +295,8 @@ def moe_copy_act_scales(plan, workspace, dst, stream=None):
 
 
 def moe_plan_set_weight_layout(plan, layout):
-    """0 / False: row-major, 1 / True: tiled (FP8, BF16), 2: MXFP4 scales chunked."""
+    """0 / False: row-major, 1 / True: tiled (FP8, BF16), 2: MXFP4 scales chunked,
+    3: MXFP4 codes tiled and scales chunked."""
     _check(lib().moe_plan_set_weight_layout(plan, int(layout)), "moe_plan_set_weight_layout")
 
 
@@ -370,9 +404,14 @@ class MoELayer:
         self.T, self.H, self.I, self.E, self.k = T, H, I, E, k
         self.w_dtype = w_dtype
         self.plan = moe_plan(T, H, I, E, k, w_dtype, act, alpha, up_bias, limit)
-        if tiled_weights:
+        if w_dtype == "e2m1" and tiled_weights:
+            # MXFP4: tiled codes come with chunked scales (one layout value).
+            if not chunked_scales:
+                raise MoEError(MOE_ERR_INVALID_ARG, "tiled MXFP4 codes need chunked_scales=True")
+            moe_plan_set_weight_layout(self.plan, 3)
+        elif tiled_weights:
             moe_plan_set_weight_layout(self.plan, 1)
-        if chunked_scales:
+        elif chunked_scales:
             moe_plan_set_weight_layout(self.plan, 2)
         if cta_pairs is not None:
             moe_plan_set_cta_pairs(self.plan, cta_pairs)
@@ -397,7 +436,8 @@ class MoELayer:
         return out
 
     def prepack(self, w1, w2):
-        """Tiled copies of row-major FP8 or BF16 weights for a plan with tiled_weights."""
+        """Tiled copies of row-major weights (FP8 / BF16: 16 KB pre-swizzled
+        tiles; MXFP4 codes: 8 KB tiles) for a plan with tiled_weights."""
         import torch
         w1t, w2t = torch.empty_like(w1), torch.empty_like(w2)
         moe_prepack_weights(self.plan, w1, w2, w1t, w2t)

@@ -80,11 +80,13 @@ void compute_layout(moe_plan_s* p) {
   const bool fp8 = p->w_dtype == MOE_W_E4M3_UE8M0_128x128;
   L.pair_sf1 = take(fp8 ? E * (p->I / 128) * (p->H / 128) * 1024 : 0);
   L.pair_sf2 = take(fp8 ? E * (p->H / 256) * (p->I / 128) * 1024 : 0);
-  L.in_x = take(static_cast<size_t>(p->T) * p->H * elem);
-  L.in_xs = take(bf16 ? 0 : static_cast<size_t>(p->T) * (p->H / 128));
-  L.in_idx = take(S * 4);
-  L.in_w = take(S * 4);
-  L.out_stage = take(static_cast<size_t>(p->T) * p->H * 2);
+  for (int b = 0; b < 2; ++b) {
+    L.in_x[b] = take(static_cast<size_t>(p->T) * p->H * elem);
+    L.in_xs[b] = take(bf16 ? 0 : static_cast<size_t>(p->T) * (p->H / 128));
+    L.in_idx[b] = take(S * 4);
+    L.in_w[b] = take(S * 4);
+    L.out_stage[b] = take(static_cast<size_t>(p->T) * p->H * 2);
+  }
   // Debug capture last: switching it on or off moves no other buffer.
   L.act_f32 = take(p->debug_act_f32 ? rows * p->I * 4 : 0);
   L.total = off;
@@ -182,6 +184,7 @@ moe_status moe_plan(int T, int H, int I, int E, int k, moe_dtypes dtypes, moe_ac
   p->w_sf_chunked = 0;
   p->pair_mode = 0;
   p->swap_mode = 0;
+  p->io_device = -1;
   p->S = static_cast<long long>(T) * k;
   // Sum over experts of ceil(n_e / 128) <= floor((S + 127 E) / 128).
   p->rows_cap = ((p->S + 127ll * E) / kTileM) * kTileM;
@@ -192,20 +195,29 @@ moe_status moe_plan(int T, int H, int I, int E, int k, moe_dtypes dtypes, moe_ac
   return MOE_OK;
 }
 
-void moe_plan_destroy(moe_plan_t plan) { delete plan; }
+static void release_io(moe_plan_s* p);
+
+void moe_plan_destroy(moe_plan_t plan) {
+  if (plan == nullptr) return;
+  release_io(plan);
+  delete plan;
+}
 
 size_t moe_workspace_bytes(moe_plan_t plan) { return plan ? plan->ws.total : 0; }
 
 moe_status moe_plan_set_weight_layout(moe_plan_t plan, int layout) {
   if (plan == nullptr) return MOE_ERR_INVALID_ARG;
   if (layout != MOE_WEIGHTS_ROW_MAJOR && layout != MOE_WEIGHTS_TILED &&
-      layout != MOE_WEIGHTS_SCALES_CHUNKED)
+      layout != MOE_WEIGHTS_SCALES_CHUNKED && layout != MOE_WEIGHTS_TILED_SCALES_CHUNKED)
     return MOE_ERR_INVALID_ARG;
   const bool fp4 = plan->w_dtype == MOE_W_E2M1_UE8M0_1x32;
   if (layout == MOE_WEIGHTS_TILED && fp4) return MOE_ERR_UNSUPPORTED;
-  if (layout == MOE_WEIGHTS_SCALES_CHUNKED && !fp4) return MOE_ERR_UNSUPPORTED;
-  plan->w_tiled = layout == MOE_WEIGHTS_TILED ? 1 : 0;
-  plan->w_sf_chunked = layout == MOE_WEIGHTS_SCALES_CHUNKED ? 1 : 0;
+  if ((layout == MOE_WEIGHTS_SCALES_CHUNKED || layout == MOE_WEIGHTS_TILED_SCALES_CHUNKED) &&
+      !fp4)
+    return MOE_ERR_UNSUPPORTED;
+  plan->w_tiled = (layout == MOE_WEIGHTS_TILED || layout == MOE_WEIGHTS_TILED_SCALES_CHUNKED);
+  plan->w_sf_chunked =
+      (layout == MOE_WEIGHTS_SCALES_CHUNKED || layout == MOE_WEIGHTS_TILED_SCALES_CHUNKED);
   return MOE_OK;
 }
 
@@ -241,11 +253,18 @@ moe_status moe_prepack_weights(moe_plan_t plan, const void* w1, const void* w2, 
   if (plan == nullptr || w1 == nullptr || w2 == nullptr || w1_tiled == nullptr ||
       w2_tiled == nullptr)
     return MOE_ERR_INVALID_ARG;
-  if (plan->w_dtype == MOE_W_E2M1_UE8M0_1x32) return MOE_ERR_UNSUPPORTED;
   if (!aligned(w1, 16) || !aligned(w2, 16) || !aligned(w1_tiled, 16) || !aligned(w2_tiled, 16))
     return MOE_ERR_ALIGNMENT;
   auto st = reinterpret_cast<cudaStream_t>(stream);
   const long long E = plan->E;
+  if (plan->w_dtype == MOE_W_E2M1_UE8M0_1x32) {
+    // E2M1 codes: 64-byte (128-element) k-blocks, 8 KB tiles of 128 rows.
+    if (moe::launch_prepack_fp4(static_cast<const uint8_t*>(w1), E * 2 * plan->I, plan->H / 2,
+                                static_cast<uint8_t*>(w1_tiled), st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return cuda_status(moe::launch_prepack_fp4(static_cast<const uint8_t*>(w2), E * plan->H,
+                                               plan->I / 2, static_cast<uint8_t*>(w2_tiled), st));
+  }
   const int elem = plan->w_dtype == MOE_W_BF16 ? 2 : 1;   // bytes per weight
   if (moe::launch_prepack(static_cast<const uint8_t*>(w1), E * 2 * plan->I, plan->H * elem,
                           static_cast<uint8_t*>(w1_tiled), st) != cudaSuccess)
@@ -413,23 +432,139 @@ moe_status moe_forward_hostio(moe_plan_t plan, const void* x_host, const uint8_t
   const auto& L = plan->ws;
   const size_t T = plan->T, H = plan->H, S = static_cast<size_t>(plan->S);
   const bool bf16 = plan->w_dtype == MOE_W_BF16;
-  if (cudaMemcpyAsync(ws + L.in_x, x_host, T * H * (bf16 ? 2 : 1), cudaMemcpyHostToDevice, st) !=
+  if (cudaMemcpyAsync(ws + L.in_x[0], x_host, T * H * (bf16 ? 2 : 1), cudaMemcpyHostToDevice, st) !=
           cudaSuccess ||
-      (!bf16 && cudaMemcpyAsync(ws + L.in_xs, x_scales_host, T * (H / 128),
+      (!bf16 && cudaMemcpyAsync(ws + L.in_xs[0], x_scales_host, T * (H / 128),
                                 cudaMemcpyHostToDevice, st) != cudaSuccess) ||
-      cudaMemcpyAsync(ws + L.in_idx, topk_idx_host, S * 4, cudaMemcpyHostToDevice, st) !=
+      cudaMemcpyAsync(ws + L.in_idx[0], topk_idx_host, S * 4, cudaMemcpyHostToDevice, st) !=
           cudaSuccess ||
-      cudaMemcpyAsync(ws + L.in_w, topk_w_host, S * 4, cudaMemcpyHostToDevice, st) !=
+      cudaMemcpyAsync(ws + L.in_w[0], topk_w_host, S * 4, cudaMemcpyHostToDevice, st) !=
           cudaSuccess)
     return MOE_ERR_CUDA;
-  uint8_t* out_dev = ws + L.out_stage;
-  s = moe_forward(plan, ws + L.in_x, bf16 ? nullptr : ws + L.in_xs,
-                  reinterpret_cast<const int32_t*>(ws + L.in_idx),
-                  reinterpret_cast<const float*>(ws + L.in_w), w1, w1_scales, w2, w2_scales,
+  uint8_t* out_dev = ws + L.out_stage[0];
+  s = moe_forward(plan, ws + L.in_x[0], bf16 ? nullptr : ws + L.in_xs[0],
+                  reinterpret_cast<const int32_t*>(ws + L.in_idx[0]),
+                  reinterpret_cast<const float*>(ws + L.in_w[0]), w1, w1_scales, w2, w2_scales,
                   out_dev, workspace, stream);
   if (s != MOE_OK) return s;
   if (cudaMemcpyAsync(out_host, out_dev, T * H * 2, cudaMemcpyDeviceToHost, st) != cudaSuccess)
     return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+// Copy streams and events of the batched host-buffer entry, created on the
+// first call on a device (a plan moved to another device gets new ones).
+static void release_io(moe_plan_s* p) {
+  if (p->io_device < 0) return;
+  int cur = 0;
+  const bool restore = cudaGetDevice(&cur) == cudaSuccess && cur != p->io_device;
+  if (restore) cudaSetDevice(p->io_device);
+  cudaStreamDestroy(p->io_h2d);
+  cudaStreamDestroy(p->io_d2h);
+  cudaEventDestroy(p->io_entry);
+  for (int b = 0; b < 2; ++b) {
+    cudaEventDestroy(p->io_in[b]);
+    cudaEventDestroy(p->io_done[b]);
+    cudaEventDestroy(p->io_out[b]);
+  }
+  if (restore) cudaSetDevice(cur);
+  p->io_device = -1;
+}
+
+static cudaError_t ensure_io(moe_plan_s* p) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (p->io_device == dev) return cudaSuccess;
+  release_io(p);
+  const unsigned ev_flags = cudaEventDisableTiming;
+  if ((e = cudaStreamCreateWithFlags(&p->io_h2d, cudaStreamNonBlocking)) != cudaSuccess) return e;
+  if ((e = cudaStreamCreateWithFlags(&p->io_d2h, cudaStreamNonBlocking)) != cudaSuccess) {
+    cudaStreamDestroy(p->io_h2d);
+    return e;
+  }
+  cudaEvent_t* evs[7] = {&p->io_entry, &p->io_in[0], &p->io_in[1], &p->io_done[0],
+                         &p->io_done[1], &p->io_out[0], &p->io_out[1]};
+  for (int i = 0; i < 7; ++i) {
+    if ((e = cudaEventCreateWithFlags(evs[i], ev_flags)) != cudaSuccess) {
+      for (int j = 0; j < i; ++j) cudaEventDestroy(*evs[j]);
+      cudaStreamDestroy(p->io_h2d);
+      cudaStreamDestroy(p->io_d2h);
+      return e;
+    }
+  }
+  p->io_device = dev;
+  return cudaSuccess;
+}
+
+moe_status moe_forward_hostio_batches(moe_plan_t plan, int n_batches,
+                                      const void* const* x_host,
+                                      const uint8_t* const* x_scales_host,
+                                      const int32_t* const* topk_idx_host,
+                                      const float* const* topk_w_host, const void* w1,
+                                      const uint8_t* w1_scales, const void* w2,
+                                      const uint8_t* w2_scales, void* const* out_host,
+                                      void* workspace, moe_stream_t stream) {
+  moe_status s = check_ws(plan, workspace);
+  if (s != MOE_OK) return s;
+  if (n_batches < 1 || x_host == nullptr || topk_idx_host == nullptr ||
+      topk_w_host == nullptr || out_host == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  const bool bf16 = plan->w_dtype == MOE_W_BF16;
+  if (!bf16 && x_scales_host == nullptr) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < n_batches; ++i)
+    if (x_host[i] == nullptr || (!bf16 && x_scales_host[i] == nullptr) ||
+        topk_idx_host[i] == nullptr || topk_w_host[i] == nullptr || out_host[i] == nullptr)
+      return MOE_ERR_INVALID_ARG;
+  if ((s = check_weights(plan, w1, w1_scales)) != MOE_OK) return s;
+  if ((s = check_weights(plan, w2, w2_scales)) != MOE_OK) return s;
+  if (ensure_io(plan) != cudaSuccess) return MOE_ERR_CUDA;
+  auto ws = static_cast<uint8_t*>(workspace);
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  const auto& L = plan->ws;
+  const size_t T = plan->T, H = plan->H, S = static_cast<size_t>(plan->S);
+  const size_t x_bytes = T * H * (bf16 ? 2 : 1), out_bytes = T * H * 2;
+  cudaStream_t h2d = plan->io_h2d, d2h = plan->io_d2h;
+  // Everything enqueued on `stream` before this call comes first.
+  if (cudaEventRecord(plan->io_entry, st) != cudaSuccess ||
+      cudaStreamWaitEvent(h2d, plan->io_entry, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(d2h, plan->io_entry, 0) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  for (int i = 0; i < n_batches; ++i) {
+    const int b = i & 1;
+    // Staging set b's inputs are free once the layer of batch i-2 is done.
+    if (i >= 2 && cudaStreamWaitEvent(h2d, plan->io_done[b], 0) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (cudaMemcpyAsync(ws + L.in_x[b], x_host[i], x_bytes, cudaMemcpyHostToDevice, h2d) !=
+            cudaSuccess ||
+        (!bf16 && cudaMemcpyAsync(ws + L.in_xs[b], x_scales_host[i], T * (H / 128),
+                                  cudaMemcpyHostToDevice, h2d) != cudaSuccess) ||
+        cudaMemcpyAsync(ws + L.in_idx[b], topk_idx_host[i], S * 4, cudaMemcpyHostToDevice,
+                        h2d) != cudaSuccess ||
+        cudaMemcpyAsync(ws + L.in_w[b], topk_w_host[i], S * 4, cudaMemcpyHostToDevice, h2d) !=
+            cudaSuccess ||
+        cudaEventRecord(plan->io_in[b], h2d) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    // The layer waits for its inputs and, for staging set b's output, for the
+    // output copy of batch i-2.
+    if (cudaStreamWaitEvent(st, plan->io_in[b], 0) != cudaSuccess ||
+        (i >= 2 && cudaStreamWaitEvent(st, plan->io_out[b], 0) != cudaSuccess))
+      return MOE_ERR_CUDA;
+    s = moe_forward(plan, ws + L.in_x[b], bf16 ? nullptr : ws + L.in_xs[b],
+                    reinterpret_cast<const int32_t*>(ws + L.in_idx[b]),
+                    reinterpret_cast<const float*>(ws + L.in_w[b]), w1, w1_scales, w2,
+                    w2_scales, ws + L.out_stage[b], workspace, stream);
+    if (s != MOE_OK) return s;
+    if (cudaEventRecord(plan->io_done[b], st) != cudaSuccess ||
+        cudaStreamWaitEvent(d2h, plan->io_done[b], 0) != cudaSuccess ||
+        cudaMemcpyAsync(out_host[i], ws + L.out_stage[b], out_bytes, cudaMemcpyDeviceToHost,
+                        d2h) != cudaSuccess ||
+        cudaEventRecord(plan->io_out[b], d2h) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  // `stream` completes only after every output copy has landed.
+  for (int b = 0; b < 2 && b < n_batches; ++b)
+    if (cudaStreamWaitEvent(st, plan->io_out[b], 0) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
 

@@ -116,6 +116,7 @@ struct Params {
                              // 0 never, 1 always, 2 for tiles of at most kSwapRows rows
   int dep_extra;             // test hook: FC2 waits for this many FC1 completions more
   int sf_chunked;            // MXFP4 weight scales prepacked into 512-byte chunks
+  int fp4_tiled;             // MXFP4 codes prepacked into 8 KB tiles (one TMA box each)
   Phase ph[2];
   const int32_t* tile_off;
   const int32_t* counts;
@@ -399,6 +400,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                   sm.b[stage] + 128 * BK,
                   ph.w_tiles + (static_cast<size_t>(brow1 / 128) * ph.k_blocks + kb) * kTileBytes,
                   kTileBytes, &sm.full[stage], pol_b);
+            } else if (kFp4 && p.fp4_tiled) {
+              // Tiled E2M1 codes: the k-block of a 128-row block is one
+              // contiguous 8 KB tile, row (block * k_blocks + kb) * 128 of the map.
+              tma_load_2d(sm.b[stage], tb, 0, (brow0 / 128 * ph.k_blocks + kb) * 128,
+                          &sm.full[stage], pol_b);
+              tma_load_2d(sm.b[stage] + 128 * BK, tb, 0, (brow1 / 128 * ph.k_blocks + kb) * 128,
+                          &sm.full[stage], pol_b);
             } else if (t.kind == 0) {
               tma_load_2d(sm.b[stage], tb, kb * BK, brow0, &sm.full[stage], pol_b);
               tma_load_2d(sm.b[stage] + 128 * BK, tb, kb * BK, brow1, &sm.full[stage], pol_b);
@@ -924,9 +932,13 @@ cudaError_t launch_gemm(const moe_plan_s* pl, int phases, bool dynamic, const vo
   p.dep_extra = pl->debug_fault ? 1 : 0;
   p.sf_chunked = pl->w_sf_chunked;
   long long max_tiles = 0;
-  const bool tiled = pl->w_tiled != 0;
   constexpr bool kFp4 = kW == kWFp4;
   constexpr bool kBf16 = kW == kWBf16;
+  // FP8 / BF16 tiles are pre-swizzled and bulk-copied; E2M1 tiles are read by a
+  // tensor map over the tile array (the copy widens the codes).
+  const bool tiled = pl->w_tiled != 0 && !kFp4;
+  const bool fp4_tiled = pl->w_tiled != 0 && kFp4;
+  p.fp4_tiled = fp4_tiled ? 1 : 0;
   // Bytes of one weight row of K elements, and the map's inner extent: FP4 maps
   // count 4-bit elements (the copy widens them), the others count bytes.
   auto row_bytes = [](int K) { return kFp4 ? K / 2 : (kBf16 ? 2 * K : K); };
@@ -935,8 +947,9 @@ cudaError_t launch_gemm(const moe_plan_s* pl, int phases, bool dynamic, const vo
   auto k_blocks = [](int K) { return kBf16 ? K / 64 : K / 128; };
   if (phases & 1) {
     const int K = pl->H;
-    if (!tiled && !make_map(&maps[1], w1, inner(K), static_cast<uint64_t>(pl->E) * 2 * pl->I,
-                            row_bytes(K), 128, kFp4))
+    const uint64_t rows = static_cast<uint64_t>(pl->E) * 2 * pl->I;
+    if (fp4_tiled ? !make_map(&maps[1], w1, 128, rows * (K / 128), 64, 128, true)
+                  : (!tiled && !make_map(&maps[1], w1, inner(K), rows, row_bytes(K), 128, kFp4)))
       return cudaErrorInvalidValue;
     p.ph[0] = Phase{pl->I / 128, k_blocks(K), 2 * pl->I, kBf16 ? nullptr : ws + L.xg_sf, w1s,
                     ws + L.xg, tiled ? static_cast<const uint8_t*>(w1) : nullptr};
@@ -944,8 +957,9 @@ cudaError_t launch_gemm(const moe_plan_s* pl, int phases, bool dynamic, const vo
   }
   if (phases & 2) {
     const int K = pl->I;
-    if (!tiled && !make_map(&maps[3], w2, inner(K), static_cast<uint64_t>(pl->E) * pl->H,
-                            row_bytes(K), 256, kFp4))
+    const uint64_t rows = static_cast<uint64_t>(pl->E) * pl->H;
+    if (fp4_tiled ? !make_map(&maps[3], w2, 128, rows * (K / 128), 64, 128, true)
+                  : (!tiled && !make_map(&maps[3], w2, inner(K), rows, row_bytes(K), 256, kFp4)))
       return cudaErrorInvalidValue;
     p.ph[1] = Phase{pl->H / 256, k_blocks(K), pl->H, kBf16 ? nullptr : ws + L.act_sf, w2s,
                     ws + L.act, tiled ? static_cast<const uint8_t*>(w2) : nullptr};

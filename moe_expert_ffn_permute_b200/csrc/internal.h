@@ -27,8 +27,10 @@ struct WorkspaceLayout {
   size_t act_f32;           // debug capture (0 bytes when off)
   size_t y;                 // FC2 output, bf16, slot order
   size_t pair_sf1, pair_sf2;   // weight scales expanded for the CTA-pair GEMM (FP8 plans)
-  size_t in_x, in_xs, in_idx, in_w;   // staging for moe_forward_hostio inputs
-  size_t out_stage;                   // and its bf16 output
+  // Two staging sets for the host-buffer entries (moe_forward_hostio uses set
+  // 0; moe_forward_hostio_batches alternates between them): inputs and output.
+  size_t in_x[2], in_xs[2], in_idx[2], in_w[2];
+  size_t out_stage[2];
   size_t total;
 };
 
@@ -40,10 +42,16 @@ struct moe_plan_s {
   moe_act_params act;
   int debug_act_f32;
   int debug_fault;       // test hook: the fused GEMM's FC2 dependency can never be met
-  int w_tiled;           // weights given as pre-swizzled tiles (moe_prepack_weights)
+  int w_tiled;           // weights given as tiles (moe_prepack_weights): FP8 / BF16
+                         // pre-swizzled 16 KB tiles, E2M1 plain 8 KB tiles
   int w_sf_chunked;      // MXFP4 scales given in 512-byte chunks (moe_prepack_weight_scales)
   int pair_mode;         // 2-SM GEMM: 0 automatic, 1 never, 2 always
   int swap_mode;         // token-major MMAs: 0 automatic, 1 never, 2 always
+  // Copy streams and events of moe_forward_hostio_batches, created on its
+  // first call on a device (io_device = that device, -1 before).
+  int io_device;
+  cudaStream_t io_h2d, io_d2h;
+  cudaEvent_t io_entry, io_in[2], io_done[2], io_out[2];
   long long S;           // T*k
   long long rows_cap;    // padded row capacity (multiple of 128)
   int route_blocks;
@@ -125,6 +133,9 @@ cudaError_t launch_unpack_act(const moe_plan_s* p, const uint8_t* ws, uint8_t* d
                               cudaStream_t st);
 cudaError_t launch_prepack(const uint8_t* src, long long rows, int K, uint8_t* dst,
                            cudaStream_t st);
+// Packed E2M1 weights [rows, row_bytes] -> 8 KB tiles of 128 rows x 64 bytes.
+cudaError_t launch_prepack_fp4(const uint8_t* src, long long rows, int row_bytes, uint8_t* dst,
+                               cudaStream_t st);
 cudaError_t launch_unpack_act_scales(const moe_plan_s* p, const uint8_t* ws, uint8_t* dst,
                                      cudaStream_t st);
 

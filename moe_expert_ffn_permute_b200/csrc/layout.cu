@@ -29,6 +29,29 @@ __global__ void __launch_bounds__(256) prepack_kernel(const uint4* __restrict__ 
   }
 }
 
+// Packed E2M1 weights [rows, row_bytes] -> tiles of 128 rows x 64 bytes (128
+// codes of one k-block per row), 8 KB each, tile (b, kb) at (b * row_bytes/64 +
+// kb) * 8192, row r of the tile at r * 64 -- contiguous in HBM, so that one
+// k-block of 128 weight rows is a single 8 KB stream; the tensor map that
+// reads it widens the codes into the tensor core's padded shared-memory
+// layout.  One thread per 16-byte chunk.
+__global__ void __launch_bounds__(256) prepack_fp4_kernel(const uint4* __restrict__ src,
+                                                          long long rows, int row_bytes,
+                                                          uint8_t* __restrict__ dst) {
+  const int vec = row_bytes / 16;
+  const int kb_n = row_bytes / 64;
+  const long long n = rows * vec;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long row = i / vec;
+    const int c = static_cast<int>(i - row * vec);
+    const long long rb = row / 128;
+    const int r = static_cast<int>(row - rb * 128);
+    uint8_t* d = dst + (rb * kb_n + (c >> 2)) * 8192ll + r * 64 + (c & 3) * 16;
+    *reinterpret_cast<uint4*>(d) = __ldg(&src[i]);
+  }
+}
+
 // Tiles -> row-major (inspection of the FC1 activation).
 __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__ src, long long rows,
                                                      int K, uint4* __restrict__ dst) {
@@ -76,6 +99,13 @@ cudaError_t launch_prepack(const uint8_t* src, long long rows, int K, uint8_t* d
   const long long n = rows * (K / 16);
   return launch_plain(prepack_kernel, dim3(blocks_for(n)), dim3(256), 0, st,
                       reinterpret_cast<const uint4*>(src), rows, K, dst);
+}
+
+cudaError_t launch_prepack_fp4(const uint8_t* src, long long rows, int row_bytes, uint8_t* dst,
+                               cudaStream_t st) {
+  const long long n = rows * (row_bytes / 16);
+  return launch_plain(prepack_fp4_kernel, dim3(blocks_for(n)), dim3(256), 0, st,
+                      reinterpret_cast<const uint4*>(src), rows, row_bytes, dst);
 }
 
 cudaError_t launch_prepack_fp4_scales(const uint8_t* src, long long rows, int K, uint8_t* dst,

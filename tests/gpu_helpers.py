@@ -84,9 +84,9 @@ def inputs(wl, device="cuda", seed=None):
 
 def bench_layer(wl, d, swap=None):
     """The layer in the launch configuration bench.py times: FP8 / BF16 weights
-    prepacked into tiles, MXFP4 scales prepacked into chunks, automatic tile
+    prepacked into tiles, MXFP4 codes into tiles and scales into chunks, automatic tile
     orientation (unless `swap` forces one).  Returns (layer, weights dict)."""
-    tiled = wl.w_dtype in ("e4m3", "bf16")
+    tiled = True                     # FP8 / BF16 tiles, MXFP4 code tiles
     chunked = wl.w_dtype == "e2m1"
     lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype=wl.w_dtype, act=wl.act,
                        alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit,

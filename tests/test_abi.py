@@ -244,3 +244,41 @@ def test_debug_capture_moves_no_other_buffer():
         moe.moe_plan_set_debug(p, 0)
         assert moe.moe_workspace_bytes(p) == before
         moe.moe_plan_destroy(p)
+
+
+def test_hostio_batches_validates_before_enqueuing(L):
+    """The batched host-buffer entry refuses a bad batch count or a missing
+    array / entry before it touches CUDA (it creates its copy streams only
+    after validation)."""
+    p = moe.moe_plan(64, 512, 256, 8, 2)
+    ws, w = 1 << 30, 1 << 20                               # aligned stand-ins, never read
+    arr = lambda n, v=1 << 12: (ctypes.c_void_p * n)(*([v] * n))
+    good = dict(x=arr(2), xs=arr(2), idx=arr(2), tw=arr(2), out=arr(2))
+
+    def call(n, **kw):
+        a = dict(good, **kw)
+        return L.moe_forward_hostio_batches(p, n, a["x"], a["xs"], a["idx"], a["tw"], w, w, w, w,
+                                            a["out"], ws, None)
+    assert call(0) == 1
+    assert call(-3) == 1
+    assert call(2, x=None) == 1
+    assert call(2, xs=None) == 1                            # FP8 plans need x scales
+    assert call(2, out=arr(2, 0)) == 1                      # a NULL entry
+    assert call(2, idx=(ctypes.c_void_p * 2)(1 << 12, None)) == 1
+    assert L.moe_forward_hostio_batches(p, 2, good["x"], good["xs"], good["idx"], good["tw"],
+                                        w + 1, w, w, w, good["out"], ws, None) == 3
+    moe.moe_plan_destroy(p)
+
+
+def test_weight_layout_values_per_format():
+    """Tiled MXFP4 codes (layout 3) need an MXFP4 plan; FP8 / BF16 take the
+    pre-swizzled tiles (1); chunked scales alone (2) are MXFP4 only."""
+    expect = {"e4m3": {0: 0, 1: 0, 2: 2, 3: 2}, "bf16": {0: 0, 1: 0, 2: 2, 3: 2},
+              "e2m1": {0: 0, 1: 2, 2: 0, 3: 0}}
+    for w_dtype, codes in expect.items():
+        p = moe.moe_plan(64, 512, 256, 8, 2, w_dtype=w_dtype)
+        for layout, status in codes.items():
+            got = moe.lib().moe_plan_set_weight_layout(p, layout)
+            assert got == status, (w_dtype, layout, got)
+        assert moe.lib().moe_plan_set_weight_layout(p, 4) == 1
+        moe.moe_plan_destroy(p)

@@ -5,7 +5,7 @@ import pytest
 import torch
 
 import moe_expert_ffn_permute_b200 as moe
-from workloads.synth import WORKLOADS, Workload, to_numpy
+from workloads.synth import WORKLOADS, Workload, make_activations, to_numpy
 from oracle import layer as L
 
 from gpu_helpers import (assert_parity, ensure_built, inputs, layer_for, oracle_args,
@@ -522,20 +522,41 @@ def test_fp4_scale_chunk_layout_matches_its_definition():
 
 
 @pytest.mark.parametrize("swap", [1, 2], ids=["token-rows", "swap-ab"])
-def test_fp4_chunked_scales_give_the_same_bytes(swap):
+def test_fp4_chunked_scales_and_tiled_codes_give_the_same_bytes(swap):
+    """MXFP4 weights row-major, with chunked scales, and with tiled codes and
+    chunked scales: the same output bytes in either tile orientation."""
     wl = RAGGED_FP4
     d = inputs(wl)
     outs = []
-    for chunked in (False, True):
+    for chunked, tiled in ((False, False), (True, False), (True, True)):
         lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype="e2m1", swap_ab=swap,
-                           chunked_scales=chunked)
+                           chunked_scales=chunked, tiled_weights=tiled)
         s1, s2 = (lay.prepack_scales(d["w1_scales"], d["w2_scales"]) if chunked
                   else (d["w1_scales"], d["w2_scales"]))
-        outs.append(lay.forward(d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], d["w1"], s1,
-                                d["w2"], s2))
+        w1, w2 = lay.prepack(d["w1"], d["w2"]) if tiled else (d["w1"], d["w2"])
+        outs.append(lay.forward(d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], w1, s1, w2,
+                                s2))
         torch.cuda.synchronize()
         assert lay.check() == 0
     assert torch.equal(outs[0], outs[1])
+    assert torch.equal(outs[0], outs[2])
+
+
+def test_fp4_code_tiles_match_their_definition():
+    """moe_prepack_weights on MXFP4 codes: tile (b, kb) at (b * KB/64 + kb) * 8192
+    holds bytes 64kb..64kb+63 of row 128b + r at r * 64 (KB = K/2 bytes a row)."""
+    wl = RAGGED_FP4
+    d = inputs(wl)
+    lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype="e2m1", chunked_scales=True,
+                       tiled_weights=True)
+    t1, t2 = lay.prepack(d["w1"], d["w2"])
+    torch.cuda.synchronize()
+    for src, got, K in ((d["w1"], t1, wl.H), (d["w2"], t2, wl.I)):
+        kbytes = K // 2
+        rows = src.numel() // kbytes
+        ref = (src.reshape(rows // 128, 128, kbytes // 64, 64)   # [b, r, kb, byte]
+               .permute(0, 2, 1, 3).contiguous().reshape(-1))
+        assert torch.equal(got.reshape(-1), ref)
 
 
 def test_fp4_chunked_scales_full_size_128_tokens():
@@ -569,3 +590,43 @@ def test_token_rows_are_independent_of_the_batch():
     torch.cuda.synchronize()
     assert full.check() == 0 and part.check() == 0
     assert torch.equal(out_part, out_full[tokens])
+
+
+@pytest.mark.parametrize("wl", [RAGGED, WORKLOADS["bf16"]], ids=lambda w: w.name)
+def test_hostio_batches_equal_device_forwards(wl):
+    """Three consecutive batches through the pipelined host-buffer entry (the
+    copies of one batch overlap the neighbours' layers, two staging sets):
+    every batch's output equals moe_forward on the same inputs, byte for byte,
+    also when the call is repeated and when all batches share one output
+    buffer (the last batch's output lands last)."""
+    base = inputs(wl)
+    batches = [make_activations(wl, device="cuda", seed=900 + i) for i in range(3)]
+    lay = layer_for(wl)
+    ref = []
+    for d in batches:
+        out = lay.forward(d["x"], d["x_scales"], d["topk_idx"], d["topk_w"], base["w1"],
+                          base["w1_scales"], base["w2"], base["w2_scales"])
+        torch.cuda.synchronize()
+        ref.append(out.cpu())
+    keys = ("x", "x_scales", "topk_idx", "topk_w")
+    host = [{k: (None if d[k] is None else d[k].cpu().pin_memory()) for k in keys}
+            for d in batches]
+    for repeat in range(2):
+        outs = [torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory() for _ in batches]
+        moe.moe_forward_hostio_batches(
+            lay.plan, [h["x"] for h in host],
+            None if host[0]["x_scales"] is None else [h["x_scales"] for h in host],
+            [h["topk_idx"] for h in host], [h["topk_w"] for h in host], base["w1"],
+            base["w1_scales"], base["w2"], base["w2_scales"], outs, lay.workspace)
+        torch.cuda.current_stream().synchronize()
+        for i in range(3):
+            assert torch.equal(outs[i], ref[i]), (repeat, i)
+    shared = torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory()
+    moe.moe_forward_hostio_batches(
+        lay.plan, [h["x"] for h in host],
+        None if host[0]["x_scales"] is None else [h["x_scales"] for h in host],
+        [h["topk_idx"] for h in host], [h["topk_w"] for h in host], base["w1"],
+        base["w1_scales"], base["w2"], base["w2_scales"], [shared] * 3, lay.workspace)
+    torch.cuda.current_stream().synchronize()
+    assert torch.equal(shared, ref[2])
+    assert lay.check() == 0

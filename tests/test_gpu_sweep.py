@@ -31,8 +31,7 @@ def _sampled_parity(wl, ntok, seed):
     assert lay.check() == 0
     rnd = np.random.default_rng(seed).choice(wl.T, size=min(ntok, wl.T), replace=False)
     tokens = np.array(sorted(set(rnd.tolist()) | {0, wl.T - 1}))
-    dn = {k: (None if v is None else v.cpu().numpy()) for k, v in d.items()}
-    ref = oracle_tokens(wl, dn, tokens)
+    ref = oracle_tokens(wl, to_numpy(d), tokens)
     assert_parity(out.float().cpu().numpy()[tokens], ref, wl.name)
 
 
