@@ -224,9 +224,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      // operand producer's expect-tx arrive + one arrive per scale-factor lane
-      // (BF16: the expect-tx arrive alone)
-      mbar_init(&sm.full[s], kBf16 ? 1 : 33);
+      // The operand producer's expect-tx arrive, plus the scale warp's: one
+      // arrive (lane 0, after the warp's shared-memory writes or bulk copies),
+      // or one per lane when its lanes' cp.async copies arrive themselves
+      // (unchunked MXFP4 scales); BF16 has no scales.
+      mbar_init(&sm.full[s], kBf16 ? 1 : (kFp4 && !p.sf_chunked ? 33 : 2));
       mbar_init(&sm.empty[s], 1);
     }
     mbar_init(&sm.tmem_full, 1);
@@ -434,9 +436,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               bulk_load(sm.sfb[stage] + 512,
                         ph.w_sf + (static_cast<size_t>(brow1 / 128) * ph.k_blocks + kb) * 512,
                         512, &sm.full[stage]);
+              mbar_arrive(&sm.full[stage]);
             }
             __syncwarp();
-            mbar_arrive(&sm.full[stage]);
           } else if (kFp4) {
             // One 32-bit word = the four 1x32 scales of this 128-wide k-block.
             const int kw = ph.k_blocks * 4;   // scale bytes per weight row
@@ -456,8 +458,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t u = __shfl_sync(0xffffffffu, sf1, kb & 31) * 0x01010101u;
             reinterpret_cast<uint4*>(sm.sfb[stage])[lane] = make_uint4(g, g, g, g);
             reinterpret_cast<uint4*>(sm.sfb[stage] + 512)[lane] = make_uint4(u, u, u, u);
+            // Every lane makes its writes visible to the tensor core (async
+            // proxy); the warp barrier orders them before lane 0's release.
             fence_proxy_async_smem();
-            mbar_arrive(&sm.full[stage]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.full[stage]);
           }
         }
         if (++stage == STAGES) {
@@ -474,6 +479,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int slot = 0, stage = 0;
       uint32_t sphase = 0, phase = 0, acc_phase = 0, sfset = 0;
+      // Shared-memory descriptors of stage 0, built once: a stage's descriptor
+      // is stage 0's plus its byte offset >> 4, and each 32-byte K step of a
+      // 128-byte k-block adds 2 (the 14-bit address field cannot carry: shared
+      // addresses stay below 2^18 bytes).  The issuing lane then spends a
+      // 64-bit add per operand instead of rebuilding every descriptor.
+      const uint64_t a_desc0 = umma_desc_sw128(smem_u32(sm.a[0]));
+      const uint64_t b_desc0 = umma_desc_sw128(smem_u32(sm.b[0]));
+      const uint64_t sfa_desc0 = sf_desc(smem_u32(sm.sfa[0]));
+      const uint64_t sfb_desc0 = sf_desc(smem_u32(sm.sfb[0]));
+      constexpr uint64_t kAStage = (BM * BK) >> 4, kBStage = (BN * BK) >> 4;
+      constexpr uint64_t kBHalf = (128 * BK) >> 4, kKStep = 32 >> 4;
+      constexpr uint64_t kSfaStage = 512 >> 4, kSfbStage = 1024 >> 4, kSfbHalf = 512 >> 4;
       Task t;
       bool aborted = false;
       while (!aborted && get_task_single(sm, slot, sphase, t, p.err)) {
@@ -481,65 +498,71 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&sm.tmem_empty, acc_phase ^ 1u, p.err, &sm.abort_flag)) break;
         tc_fence_after();
         const int k_blocks = p.ph[t.kind].k_blocks;
+        // Token-major tiles: N = the tile's tokens rounded up to 16.  The
+        // instruction descriptor of K step ks is this one with scale id ks.
+        const bool swap = swap_tile(p, t.rows);
+        const uint32_t n =
+            swap ? static_cast<uint32_t>(min(128, max(16, (t.rows + 15) & ~15))) : BN;
+        const uint32_t idesc0 =
+            kBf16 ? bf16_idesc(n)
+                  : (swap ? mxf8f6f4_idesc_ab(kFp4 ? 5u : 0u, 0u, n, 0)
+                          : mxf8f6f4_idesc(kFp4 ? 5u : 0u, BN, 0));
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (!mbar_wait(&sm.full[stage], phase, p.err, &sm.abort_flag)) {
             aborted = true;
             break;
           }
-          const uint32_t a_base = smem_u32(sm.a[stage]);
-          const uint32_t b_base = smem_u32(sm.b[stage]);
+          const uint64_t ad = a_desc0 + static_cast<uint64_t>(stage) * kAStage;
+          const uint64_t bd = b_desc0 + static_cast<uint64_t>(stage) * kBStage;
           if (kBf16) {
             // 128 bytes of K = 64 BF16 values: four MMAs of K = 16 (32 bytes each).
-            if (swap_tile(p, t.rows)) {
+            if (swap) {
               // Token-major, as for the block-scaled formats below.
-              const uint32_t n = static_cast<uint32_t>(min(128, max(16, (t.rows + 15) & ~15)));
 #pragma unroll
               for (int ks = 0; ks < 4; ++ks) {
                 const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
-                mma_bf16(tmem + kAccCol, umma_desc_sw128(b_base + ks * 32),
-                         umma_desc_sw128(a_base + ks * 32), bf16_idesc(n), acc);
-                mma_bf16(tmem + kAccCol + 128, umma_desc_sw128(b_base + 128 * BK + ks * 32),
-                         umma_desc_sw128(a_base + ks * 32), bf16_idesc(n), acc);
+                mma_bf16(tmem + kAccCol, bd + ks * kKStep, ad + ks * kKStep, idesc0, acc);
+                mma_bf16(tmem + kAccCol + 128, bd + kBHalf + ks * kKStep, ad + ks * kKStep,
+                         idesc0, acc);
               }
             } else {
 #pragma unroll
               for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tmem + kAccCol, umma_desc_sw128(a_base + ks * 32),
-                         umma_desc_sw128(b_base + ks * 32), bf16_idesc(BN),
+                mma_bf16(tmem + kAccCol, ad + ks * kKStep, bd + ks * kKStep, idesc0,
                          (kb > 0 || ks > 0) ? 1u : 0u);
             }
           } else {
-            // MXFP4 weight scales land by cp.async (generic proxy): order them
-            // before the tensor core's (async proxy) reads of shared memory.
-            if (kFp4) fence_proxy_async_smem();
+            // Unchunked MXFP4 weight scales land by cp.async (generic proxy):
+            // order them before the tensor core's (async proxy) reads.
+            if (kFp4 && !p.sf_chunked) fence_proxy_async_smem();
             const uint32_t sfa = tmem + kSfaCol + sfset * kSfSetStride;
             const uint32_t sfb = tmem + kSfbCol + sfset * kSfSetStride;
-            tmem_cp_32x128b_warpx4(sfa, sf_desc(smem_u32(sm.sfa[stage])));
-            tmem_cp_32x128b_warpx4(sfb, sf_desc(smem_u32(sm.sfb[stage])));
-            tmem_cp_32x128b_warpx4(sfb + 4, sf_desc(smem_u32(sm.sfb[stage] + 512)));
-            if (swap_tile(p, t.rows)) {
+            const uint64_t sfbd = sfb_desc0 + static_cast<uint64_t>(stage) * kSfbStage;
+            tmem_cp_32x128b_warpx4(sfa, sfa_desc0 + static_cast<uint64_t>(stage) * kSfaStage);
+            tmem_cp_32x128b_warpx4(sfb, sfbd);
+            tmem_cp_32x128b_warpx4(sfb + 4, sfbd + kSfbHalf);
+            if (swap) {
               // Token-major: each 128-row half of the weight tile is the A
               // operand (its scales: the weight chunk), the tile's tokens are B
               // with N = their count rounded up to 16 (scales: the token chunk).
               // D0 (columns 0..) holds the first half, D1 (columns 128..) the second.
-              const uint32_t n = static_cast<uint32_t>(min(128, max(16, (t.rows + 15) & ~15)));
 #pragma unroll
               for (int ks = 0; ks < 4; ++ks) {
-                const uint32_t idesc = mxf8f6f4_idesc_ab(kFp4 ? 5u : 0u, 0u, n, ks);
+                const uint32_t idesc = idesc0 | (static_cast<uint32_t>(ks) << 4) |
+                                       (static_cast<uint32_t>(ks) << 29);
                 const uint32_t ksh = static_cast<uint32_t>(ks) << 30;
                 const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
-                mma_mxf8f6f4(tmem + kAccCol, umma_desc_sw128(b_base + ks * 32),
-                             umma_desc_sw128(a_base + ks * 32), idesc, sfb | ksh, sfa | ksh, acc);
-                mma_mxf8f6f4(tmem + kAccCol + 128, umma_desc_sw128(b_base + 128 * BK + ks * 32),
-                             umma_desc_sw128(a_base + ks * 32), idesc, (sfb + 4) | ksh,
-                             sfa | ksh, acc);
+                mma_mxf8f6f4(tmem + kAccCol, bd + ks * kKStep, ad + ks * kKStep, idesc,
+                             sfb | ksh, sfa | ksh, acc);
+                mma_mxf8f6f4(tmem + kAccCol + 128, bd + kBHalf + ks * kKStep, ad + ks * kKStep,
+                             idesc, (sfb + 4) | ksh, sfa | ksh, acc);
               }
             } else {
 #pragma unroll
               for (int ks = 0; ks < 4; ++ks) {
-                const uint32_t idesc = mxf8f6f4_idesc(kFp4 ? 5u : 0u, BN, ks);
-                mma_mxf8f6f4(tmem + kAccCol, umma_desc_sw128(a_base + ks * 32),
-                             umma_desc_sw128(b_base + ks * 32), idesc,
+                const uint32_t idesc = idesc0 | (static_cast<uint32_t>(ks) << 4) |
+                                       (static_cast<uint32_t>(ks) << 29);
+                mma_mxf8f6f4(tmem + kAccCol, ad + ks * kKStep, bd + ks * kKStep, idesc,
                              sfa | (static_cast<uint32_t>(ks) << 30),
                              sfb | (static_cast<uint32_t>(ks) << 30), (kb > 0 || ks > 0) ? 1u : 0u);
               }
