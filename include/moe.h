@@ -415,6 +415,26 @@ moe_status moe_plan_set_swap_ab(moe_plan_t plan, int mode);
  */
 int moe_plan_swap_ab_active(moe_plan_t plan);
 
+/* Wide token-major tiles: the token-aware tiling of DeepGEMM PR #386
+ * ("Optimize sm100 version with token-aware BM240 tiling, native UE8M0, and
+ * direct combine", title).  The tokens of two consecutive 128-row tiles of
+ * one expert, up to 240 of them, become one token-major tile (the MMA's N),
+ * so an expert with 129..240 tokens streams its weights once instead of
+ * twice; two accumulators of 128 weight rows x 240 tokens fill TMEM columns
+ * 0..479.  The GEMM launch with wide tiles keeps three pipeline stages (its
+ * stages hold two token tiles).  mode 0: automatic (wide tiles when the layer
+ * has 96 < T*k/E <= 480 slots per expert), 1: never, 2: always.  Needs
+ * token-major tiles (not with moe_plan_set_swap_ab mode 1 or CTA pairs).
+ * Results agree with the other tilings within rounding (the MMA's N and the
+ * sum order inside it change) and are deterministic.                       */
+moe_status moe_plan_set_wide_tiles(moe_plan_t plan, int mode);
+
+/* 1 if moe_fc1_fc2 / moe_forward run the GEMM with wide token-major tiles with
+ * the plan's current settings, 0 if not (or plan is NULL).
+ * Source: as moe_plan_set_wide_tiles.
+ */
+int moe_plan_wide_tiles_active(moe_plan_t plan);
+
 /* Rearrange row-major FP8 or BF16 weights w1 [E,2I,H] and w2 [E,H,I] (device)
  * into the tiled layout (w1_tiled, w2_tiled: device buffers of the same sizes,
  * 16-byte aligned; must not overlap the inputs).  With KB = the bytes of one

@@ -73,6 +73,8 @@ _SIGS = {
     "moe_plan_set_swap_ab": (ctypes.c_int, [_P, ctypes.c_int]),
     "moe_prepack_weight_scales": (ctypes.c_int, [_P] * 6),
     "moe_plan_swap_ab_active": (ctypes.c_int, [_P]),
+    "moe_plan_set_wide_tiles": (ctypes.c_int, [_P, ctypes.c_int]),
+    "moe_plan_wide_tiles_active": (ctypes.c_int, [_P]),
     "moe_prepack_weights": (ctypes.c_int, [_P] * 6),
     "moe_copy_act": (ctypes.c_int, [_P] * 4),
     "moe_clear_device_error": (ctypes.c_int, [_P] * 3),
@@ -325,6 +327,16 @@ def moe_plan_swap_ab_active(plan):
     return int(lib().moe_plan_swap_ab_active(plan))
 
 
+def moe_plan_set_wide_tiles(plan, mode):
+    """0: automatic, 1: never, 2: always use wide token-major tiles (up to 240
+    tokens of two m-tiles of one expert per tile)."""
+    _check(lib().moe_plan_set_wide_tiles(plan, int(mode)), "moe_plan_set_wide_tiles")
+
+
+def moe_plan_wide_tiles_active(plan):
+    return bool(lib().moe_plan_wide_tiles_active(plan))
+
+
 def moe_prepack_weights(plan, w1, w2, w1_tiled, w2_tiled, stream=None):
     _check(lib().moe_prepack_weights(plan, *map(_ptr, (w1, w2, w1_tiled, w2_tiled)),
                                      _stream(stream)), "moe_prepack_weights")
@@ -399,7 +411,7 @@ class MoELayer:
 
     def __init__(self, T, H, I, E, k, w_dtype="e4m3", act="swiglu", alpha=1.0, up_bias=0.0,
                  limit=math.inf, device="cuda", debug=False, tiled_weights=False,
-                 cta_pairs=None, swap_ab=None, chunked_scales=False):
+                 cta_pairs=None, swap_ab=None, chunked_scales=False, wide_tiles=None):
         import torch
         self.T, self.H, self.I, self.E, self.k = T, H, I, E, k
         self.w_dtype = w_dtype
@@ -417,6 +429,8 @@ class MoELayer:
             moe_plan_set_cta_pairs(self.plan, cta_pairs)
         if swap_ab is not None:
             moe_plan_set_swap_ab(self.plan, swap_ab)
+        if wide_tiles is not None:
+            moe_plan_set_wide_tiles(self.plan, wide_tiles)
         if debug:
             moe_plan_set_debug(self.plan, True)
         nbytes = moe_workspace_bytes(self.plan)

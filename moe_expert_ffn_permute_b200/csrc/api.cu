@@ -121,6 +121,20 @@ int use_swap(const moe_plan_s* p) {
   if (use_pairs(p) || p->swap_mode == 1) return 0;
   return p->swap_mode == 2 ? 1 : 2;
 }
+
+// Wide token-major tiles (up to 240 tokens of two consecutive m-tiles of one
+// expert in one tile): they need token-major MMAs, and pay off when experts
+// hold about one to two m-tiles of tokens -- then each expert's weights stream
+// once instead of twice.  Automatic mode uses them for 96 < S/E <= 480 slots
+// per expert; decode-sized layers (few tokens per expert, where the wide
+// kernel's three pipeline stages would cost) and large ones (mostly full
+// 128-row tiles) keep the four-stage kernel.
+int use_wide(const moe_plan_s* p) {
+  if (use_swap(p) == 0 || p->wide_mode == 1) return 0;
+  if (p->wide_mode == 2) return 1;
+  const long long per_expert = p->S / p->E;
+  return per_expert > 96 && per_expert <= 480 ? 1 : 0;
+}
 }  // namespace moe
 
 static moe_status check_ws(moe_plan_t plan, const void* workspace) {
@@ -184,6 +198,7 @@ moe_status moe_plan(int T, int H, int I, int E, int k, moe_dtypes dtypes, moe_ac
   p->w_sf_chunked = 0;
   p->pair_mode = 0;
   p->swap_mode = 0;
+  p->wide_mode = 0;
   p->io_device = -1;
   p->S = static_cast<long long>(T) * k;
   // Sum over experts of ceil(n_e / 128) <= floor((S + 127 E) / 128).
@@ -300,6 +315,16 @@ moe_status moe_plan_set_swap_ab(moe_plan_t plan, int mode) {
 
 int moe_plan_swap_ab_active(moe_plan_t plan) {
   return plan == nullptr ? 0 : moe::use_swap(plan);
+}
+
+moe_status moe_plan_set_wide_tiles(moe_plan_t plan, int mode) {
+  if (plan == nullptr || mode < 0 || mode > 2) return MOE_ERR_INVALID_ARG;
+  plan->wide_mode = mode;
+  return MOE_OK;
+}
+
+int moe_plan_wide_tiles_active(moe_plan_t plan) {
+  return plan == nullptr ? 0 : moe::use_wide(plan);
 }
 
 int moe_plan_cta_pairs_active(moe_plan_t plan) {

@@ -57,13 +57,10 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 128, STAGES = 4, SCHED_DEPTH = 4;
+constexpr int BM = 128, BN = 256, BK = 128, SCHED_DEPTH = 4;
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
-// TMEM columns: accumulator 0-255; two sets of scale factors (A: 4 columns,
-// B: 8 columns), alternating per k-block so that loading the next k-block's
-// scales never waits for MMAs still reading the current ones.
-constexpr uint32_t kAccCol = 0, kSfaCol = 256, kSfbCol = 264, kSfSetStride = 16;
+constexpr uint32_t kAccCol = 0, kSfSetStride = 16;
 constexpr int kEpiWarps = 8;
 constexpr int kSchedConsumers = 3 + kEpiWarps;   // 2 producers, MMA, epilogue warps
 constexpr uint64_t kDepWaitLimitNs = 2000000000ull;
@@ -71,11 +68,36 @@ constexpr uint64_t kDepWaitLimitNs = 2000000000ull;
 // work token-major against 128 x 256 token-row, but its FC1 epilogue does more
 // (a cross-lane amax, a barrier, byte stores); token-major from this size down.
 constexpr int kSwapRows = 96;
+// Wide token-major tiles (token-aware tiling, DeepGEMM PR #386 "Optimize sm100
+// version with token-aware BM240 tiling, native UE8M0, and direct combine",
+// title): the tokens of two consecutive m-tiles of one expert, up to 240, are
+// the MMA's N, so an expert with 129..240 tokens streams its weights once.  Two
+// accumulators of 128 features x 240 tokens take TMEM columns 0..479; the scale
+// sets take the last 32.
+constexpr int kWideMaxRows = 240;
 
-struct __align__(1024) Smem {
-  uint8_t a[STAGES][BM * BK];
+// Per-kernel layout: the wide kernel's stages hold two token tiles (32 KB of
+// A), so it keeps three stages; its scale columns sit above both accumulators.
+template <bool kWide>
+struct Cfg {
+  static constexpr int kStages = kWide ? 3 : 4;
+  static constexpr int kARows = kWide ? 2 * BM : BM;        // token rows a stage holds
+  static constexpr uint32_t kD1Col = kWide ? 240u : 128u;    // token-major: second half's D
+  // TMEM scale sets (alternating per k-block, so that loading the next
+  // k-block's scales never waits for MMAs still reading the current ones):
+  // token scales (up to 8 columns: two 128-row chunks) and weight scales (8
+  // columns: two 128-row halves).
+  static constexpr uint32_t kSfaCol = kWide ? 480u : 256u;
+  static constexpr uint32_t kSfbCol = kWide ? 488u : 264u;
+  static constexpr int kSfaBytes = kWide ? 1024 : 512;       // token scale chunk(s) per stage
+};
+
+template <bool kWide>
+struct __align__(1024) SmemT {
+  static constexpr int STAGES = Cfg<kWide>::kStages;
+  uint8_t a[STAGES][Cfg<kWide>::kARows * BK];
   uint8_t b[STAGES][BN * BK];
-  uint8_t sfa[STAGES][512];
+  uint8_t sfa[STAGES][Cfg<kWide>::kSfaBytes];
   uint8_t sfb[STAGES][1024];
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
@@ -119,6 +141,7 @@ struct Params {
   int fp4_tiled;             // MXFP4 codes prepacked into 8 KB tiles (one TMA box each)
   Phase ph[2];
   const int32_t* tile_off;
+  const int32_t* pair_off;   // per expert: pairs of consecutive m-tiles (wide kernel)
   const int32_t* counts;
   const int32_t* offsets;
   const int32_t* perm;
@@ -143,6 +166,7 @@ struct Task {
 // Consumer side of the scheduler ring: copy the task info out of the slot,
 // order those reads before the release (acquire/release fence at CTA scope),
 // then arrive on the slot's empty barrier.
+template <class Smem>
 __device__ __forceinline__ bool get_task(Smem& sm, int& slot, uint32_t& phase, Task& t,
                                          uint32_t* err) {
   if (!mbar_wait(&sm.sched_full[slot], phase, err, &sm.abort_flag)) return false;
@@ -168,6 +192,7 @@ __device__ __forceinline__ bool get_task(Smem& sm, int& slot, uint32_t& phase, T
 // epilogue's transcendental pipe is shared by the E4M3 / bf16 conversions).
 // Single-thread variant of get_task for the MMA issuer, which runs its loop
 // on one lane only.
+template <class Smem>
 __device__ __forceinline__ bool get_task_single(Smem& sm, int& slot, uint32_t& phase, Task& t,
                                                 uint32_t* err) {
   if (!mbar_wait(&sm.sched_full[slot], phase, err, &sm.abort_flag)) return false;
@@ -188,8 +213,16 @@ __device__ __forceinline__ bool get_task_single(Smem& sm, int& slot, uint32_t& p
   return true;
 }
 
+// Token-major tile?  In the wide kernel a tile of more than 128 rows (two
+// m-tiles) is always token-major.
+template <bool kWide>
 __device__ __forceinline__ bool swap_tile(const Params& p, int rows) {
-  return p.swap == 1 || (p.swap == 2 && rows <= kSwapRows);
+  return (kWide && rows > BM) || p.swap == 1 || (p.swap == 2 && rows <= kSwapRows);
+}
+
+// Token-major N: the tile's rows rounded up to 16 (the MMA's N granularity).
+__device__ __forceinline__ uint32_t swap_n(int rows) {
+  return static_cast<uint32_t>(max(16, (rows + 15) & ~15));
 }
 
 __device__ __forceinline__ float sigmoidf_fast(float z) {
@@ -207,7 +240,7 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
 // kind::f16 MMA, no scales).
 enum : int { kWFp8 = 0, kWFp4 = 1, kWBf16 = 2 };
 
-template <int kW>
+template <int kW, bool kWide>
 __global__ void __launch_bounds__(kThreads, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a1,
                     const __grid_constant__ CUtensorMap tmap_b1,
@@ -215,6 +248,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tmap_b2, const Params p) {
   constexpr bool kFp4 = kW == kWFp4;
   constexpr bool kBf16 = kW == kWBf16;
+  using Smem = SmemT<kWide>;
+  using C = Cfg<kWide>;
+  constexpr int STAGES = Smem::STAGES;
   extern __shared__ uint8_t smem_raw[];
   griddep_launch_dependents();
   Smem& sm = *reinterpret_cast<Smem*>(
@@ -263,10 +299,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // out before any FC2 tile, so an FC2 tile only ever waits for FC1 tiles
     // that running CTAs already own (no deadlock, even if not all CTAs are
     // resident).
+    // Wide kernel: the index space runs over pairs of consecutive m-tiles of
+    // one expert, two indices per (pair, n-tile): a pair of at most 240 rows is
+    // one wide token-major task at the first index (the second is skipped); a
+    // pair of more rows is two tasks, one per m-tile; a lone m-tile is one.
     if (lane == 0) {
-      const int total_m = p.tile_off[p.E];
-      const int T1 = (p.phases & 1) ? total_m * p.ph[0].n_tiles : 0;
-      const int T2 = (p.phases & 2) ? total_m * p.ph[1].n_tiles : 0;
+      const int units = kWide ? 2 * p.pair_off[p.E] : p.tile_off[p.E];
+      const int T1 = (p.phases & 1) ? units * p.ph[0].n_tiles : 0;
+      const int T2 = (p.phases & 2) ? units * p.ph[1].n_tiles : 0;
       int slot = 0;
       uint32_t phase = 0;
       int e_cur[2] = {0, 0};
@@ -279,16 +319,39 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int local_tile = kind ? tile - T1 : tile;
           const int nt_n = p.ph[kind].n_tiles;
           t.kind = kind;
-          t.mt = local_tile / nt_n;
-          t.nt = local_tile - t.mt * nt_n;
           int& e = e_cur[kind];
-          if (p.tile_off[e] > t.mt) e = 0;   // round-robin order is monotone per phase
-          while (p.tile_off[e + 1] <= t.mt) ++e;
-          const int local = (t.mt - p.tile_off[e]) * BM;
-          t.e = e;
-          t.rows = min(BM, p.counts[e] - local);
-          t.pos = p.offsets[e] + local;
-          t.reuse = (p.tile_off[e + 1] - p.tile_off[e]) > 1;
+          if (kWide) {
+            const int unit = local_tile >> 1, sub = local_tile & 1;
+            const int pg = unit / nt_n;
+            t.nt = unit - pg * nt_n;
+            if (p.pair_off[e] > pg) e = 0;   // round-robin order is monotone per phase
+            while (p.pair_off[e + 1] <= pg) ++e;
+            const int mt0 = p.tile_off[e] + 2 * (pg - p.pair_off[e]);
+            const int local0 = (mt0 - p.tile_off[e]) * BM;
+            const int rows_all = min(2 * BM, p.counts[e] - local0);
+            if (rows_all <= kWideMaxRows) {
+              if (sub) continue;   // one task covers the pair (or the lone m-tile)
+              t.mt = mt0;
+              t.rows = rows_all;
+              t.pos = p.offsets[e] + local0;
+            } else {
+              t.mt = mt0 + sub;
+              t.rows = sub ? rows_all - BM : BM;
+              t.pos = p.offsets[e] + local0 + sub * BM;
+            }
+            t.e = e;
+            t.reuse = p.counts[e] > kWideMaxRows;
+          } else {
+            t.mt = local_tile / nt_n;
+            t.nt = local_tile - t.mt * nt_n;
+            if (p.tile_off[e] > t.mt) e = 0;   // round-robin order is monotone per phase
+            while (p.tile_off[e + 1] <= t.mt) ++e;
+            const int local = (t.mt - p.tile_off[e]) * BM;
+            t.e = e;
+            t.rows = min(BM, p.counts[e] - local);
+            t.pos = p.offsets[e] + local;
+            t.reuse = (p.tile_off[e + 1] - p.tile_off[e]) > 1;
+          }
         }
         if (!mbar_wait(&sm.sched_empty[slot], phase ^ 1u, p.err, &sm.abort_flag)) break;
         sm.task[slot] = make_int4(t.kind | (t.reuse << 1) | (t.e << 2), t.mt, t.nt, t.rows);
@@ -332,10 +395,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const CUtensorMap* tb = t.kind ? &tmap_b2 : &tmap_b1;
       // A token-major tile's MMAs read only its first N = round16(rows) token
       // rows, which are the first N * 128 bytes of the pre-swizzled tile (the
-      // swizzle permutes 16-byte chunks within a row): copy just those.
+      // swizzle permutes 16-byte chunks within a row): copy just those.  A wide
+      // tile's rows continue into the next m-tile's tile, copied right behind
+      // the first (row 128 + i keeps row i's swizzle phase).
+      const bool wide = kWide && t.rows > BM;
       const uint32_t a_bytes =
-          swap_tile(p, t.rows)
-              ? static_cast<uint32_t>(min(128, max(16, (t.rows + 15) & ~15))) * 128u
+          swap_tile<kWide>(p, t.rows)
+              ? (wide ? kTileBytes + swap_n(t.rows - BM) * 128u : swap_n(t.rows) * 128u)
               : kTileBytes;
       // Rows of B for this tile: two 128-row halves.
       int brow0, brow1;
@@ -352,17 +418,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         // scale chunks), then order those generic-proxy writes before this
         // thread's async-proxy (bulk copy) reads.
         if (lane == 0) {
-          const uint32_t* flag = p.fc1_done + t.mt;
-          if (ld_acquire_gpu(flag) < fc1_target) {
-            const uint64_t t0 = globaltimer();
-            while (ld_acquire_gpu(flag) < fc1_target) {
-              if (sm.abort_flag) break;
-              if (globaltimer() - t0 > kDepWaitLimitNs) {
-                atomicOr(p.err, kErrTimeoutBit);
-                sm.abort_flag = 1;
-                break;
+          // A wide tile reads the activation rows of two m-tiles.
+          for (int m = 0; m < (wide ? 2 : 1); ++m) {
+            const uint32_t* flag = p.fc1_done + t.mt + m;
+            if (ld_acquire_gpu(flag) < fc1_target) {
+              const uint64_t t0 = globaltimer();
+              while (ld_acquire_gpu(flag) < fc1_target) {
+                if (sm.abort_flag) break;
+                if (globaltimer() - t0 > kDepWaitLimitNs) {
+                  atomicOr(p.err, kErrTimeoutBit);
+                  sm.abort_flag = 1;
+                  break;
+                }
+                __nanosleep(128);
               }
-              __nanosleep(128);
             }
           }
           fence_proxy_async_global();
@@ -389,10 +458,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(&sm.full[stage], ab_bytes - kTileBytes + a_bytes);
             // Operand tiles are contiguous and pre-swizzled: one linear bulk
             // copy each (row-major weights fall back to 2-D TMA tiles).
-            bulk_load_hint(
-                sm.a[stage],
-                ph.a_tiles + (static_cast<size_t>(t.mt) * ph.k_blocks + kb) * kTileBytes,
-                a_bytes, &sm.full[stage], pol_a);
+            if (wide) {
+              bulk_load_hint(
+                  sm.a[stage],
+                  ph.a_tiles + (static_cast<size_t>(t.mt) * ph.k_blocks + kb) * kTileBytes,
+                  kTileBytes, &sm.full[stage], pol_a);
+              bulk_load_hint(
+                  sm.a[stage] + kTileBytes,
+                  ph.a_tiles + (static_cast<size_t>(t.mt + 1) * ph.k_blocks + kb) * kTileBytes,
+                  a_bytes - kTileBytes, &sm.full[stage], pol_a);
+            } else {
+              bulk_load_hint(
+                  sm.a[stage],
+                  ph.a_tiles + (static_cast<size_t>(t.mt) * ph.k_blocks + kb) * kTileBytes,
+                  a_bytes, &sm.full[stage], pol_a);
+            }
             if (ph.w_tiles != nullptr) {
               bulk_load_hint(
                   sm.b[stage],
@@ -419,10 +499,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
         } else {
           if (lane == 0) {
-            mbar_expect_tx(&sm.full[stage], 512);
+            // Token scale chunk of the tile's m-tile (and of the next one for
+            // a wide tile).
+            mbar_expect_tx(&sm.full[stage], wide ? 1024 : 512);
             bulk_load(sm.sfa[stage],
                       ph.sfa_chunks + (static_cast<size_t>(t.mt) * ph.k_blocks + kb) * 512, 512,
                       &sm.full[stage]);
+            if (wide)
+              bulk_load(sm.sfa[stage] + 512,
+                        ph.sfa_chunks + (static_cast<size_t>(t.mt + 1) * ph.k_blocks + kb) * 512,
+                        512, &sm.full[stage]);
           }
           if (kFp4 && p.sf_chunked) {
             // Prepacked scales: the stage's two 512-byte chunks (128 weight rows
@@ -488,9 +574,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t b_desc0 = umma_desc_sw128(smem_u32(sm.b[0]));
       const uint64_t sfa_desc0 = sf_desc(smem_u32(sm.sfa[0]));
       const uint64_t sfb_desc0 = sf_desc(smem_u32(sm.sfb[0]));
-      constexpr uint64_t kAStage = (BM * BK) >> 4, kBStage = (BN * BK) >> 4;
+      constexpr uint64_t kAStage = (C::kARows * BK) >> 4, kBStage = (BN * BK) >> 4;
       constexpr uint64_t kBHalf = (128 * BK) >> 4, kKStep = 32 >> 4;
-      constexpr uint64_t kSfaStage = 512 >> 4, kSfbStage = 1024 >> 4, kSfbHalf = 512 >> 4;
+      constexpr uint64_t kSfaStage = C::kSfaBytes >> 4, kSfbStage = 1024 >> 4;
+      constexpr uint64_t kSfHalf = 512 >> 4;   // the second 128-row chunk of a scale pair
       Task t;
       bool aborted = false;
       while (!aborted && get_task_single(sm, slot, sphase, t, p.err)) {
@@ -500,9 +587,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int k_blocks = p.ph[t.kind].k_blocks;
         // Token-major tiles: N = the tile's tokens rounded up to 16.  The
         // instruction descriptor of K step ks is this one with scale id ks.
-        const bool swap = swap_tile(p, t.rows);
-        const uint32_t n =
-            swap ? static_cast<uint32_t>(min(128, max(16, (t.rows + 15) & ~15))) : BN;
+        const bool swap = swap_tile<kWide>(p, t.rows);
+        const bool wide = kWide && t.rows > BM;   // tokens of two m-tiles, N up to 240
+        const uint32_t n = swap ? swap_n(t.rows) : BN;
         const uint32_t idesc0 =
             kBf16 ? bf16_idesc(n)
                   : (swap ? mxf8f6f4_idesc_ab(kFp4 ? 5u : 0u, 0u, n, 0)
@@ -522,8 +609,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int ks = 0; ks < 4; ++ks) {
                 const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
                 mma_bf16(tmem + kAccCol, bd + ks * kKStep, ad + ks * kKStep, idesc0, acc);
-                mma_bf16(tmem + kAccCol + 128, bd + kBHalf + ks * kKStep, ad + ks * kKStep,
-                         idesc0, acc);
+                mma_bf16(tmem + kAccCol + C::kD1Col, bd + kBHalf + ks * kKStep,
+                         ad + ks * kKStep, idesc0, acc);
               }
             } else {
 #pragma unroll
@@ -535,12 +622,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Unchunked MXFP4 weight scales land by cp.async (generic proxy):
             // order them before the tensor core's (async proxy) reads.
             if (kFp4 && !p.sf_chunked) fence_proxy_async_smem();
-            const uint32_t sfa = tmem + kSfaCol + sfset * kSfSetStride;
-            const uint32_t sfb = tmem + kSfbCol + sfset * kSfSetStride;
+            const uint32_t sfa = tmem + C::kSfaCol + sfset * kSfSetStride;
+            const uint32_t sfb = tmem + C::kSfbCol + sfset * kSfSetStride;
+            const uint64_t sfad = sfa_desc0 + static_cast<uint64_t>(stage) * kSfaStage;
             const uint64_t sfbd = sfb_desc0 + static_cast<uint64_t>(stage) * kSfbStage;
-            tmem_cp_32x128b_warpx4(sfa, sfa_desc0 + static_cast<uint64_t>(stage) * kSfaStage);
+            // Token scales: rows 0..127 in columns 0..3, a wide tile's rows
+            // 128.. in columns 4..7 (the layout N > 128 reads).
+            tmem_cp_32x128b_warpx4(sfa, sfad);
+            if (wide) tmem_cp_32x128b_warpx4(sfa + 4, sfad + kSfHalf);
             tmem_cp_32x128b_warpx4(sfb, sfbd);
-            tmem_cp_32x128b_warpx4(sfb + 4, sfbd + kSfbHalf);
+            tmem_cp_32x128b_warpx4(sfb + 4, sfbd + kSfHalf);
             if (swap) {
               // Token-major: each 128-row half of the weight tile is the A
               // operand (its scales: the weight chunk), the tile's tokens are B
@@ -554,8 +645,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
                 mma_mxf8f6f4(tmem + kAccCol, bd + ks * kKStep, ad + ks * kKStep, idesc,
                              sfb | ksh, sfa | ksh, acc);
-                mma_mxf8f6f4(tmem + kAccCol + 128, bd + kBHalf + ks * kKStep, ad + ks * kKStep,
-                             idesc, (sfb + 4) | ksh, sfa | ksh, acc);
+                mma_mxf8f6f4(tmem + kAccCol + C::kD1Col, bd + kBHalf + ks * kKStep,
+                             ad + ks * kKStep, idesc, (sfb + 4) | ksh, sfa | ksh, acc);
               }
             } else {
 #pragma unroll
@@ -608,26 +699,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (t.e < 0) break;
       if (!mbar_wait(&sm.tmem_full, acc_phase, p.err, &sm.abort_flag)) break;
       tc_fence_after();
-      if (swap_tile(p, t.rows)) {
+      if (swap_tile<kWide>(p, t.rows)) {
         // Token-major tile: TMEM lane = feature, column = token.  This warp
-        // owns feature f of the tile for the tokens of its half.
+        // owns feature f of the tile for the tokens of its half.  A wide tile
+        // (more than 128 rows, tokens of m-tiles mt and mt + 1) takes two
+        // rounds of 128 tokens; the accumulator is released after the last
+        // round's loads.
         const int f = q * 32 + lane;
+        const int rounds = (kWide && t.rows > BM) ? 2 : 1;
+        bool ok = true;
         if (t.kind == 0) {
-          const int tok0 = half * 64;
-          const int ntok = min(64, t.rows - tok0);   // uniform over the half's warps
+          for (int rho = 0; rho < rounds && ok; ++rho) {
+          const int mt = t.mt + rho;                  // m-tile of this round's tokens
+          const int tok0 = rho * BM + half * 64;      // first token (column) of this warp
+          const int ntok = min(64, t.rows - tok0);    // uniform over the half's warps
           // (Loaded unconditionally: TMEM columns are always addressable, and a
           // conditional load would move the arrays to local memory.)
           uint32_t g[64], u[64];
           tmem_ld_32x32b_x32(t_row + kAccCol + tok0, *reinterpret_cast<uint32_t(*)[32]>(g));
           tmem_ld_32x32b_x32(t_row + kAccCol + tok0 + 32,
                              *reinterpret_cast<uint32_t(*)[32]>(g + 32));
-          tmem_ld_32x32b_x32(t_row + kAccCol + 128 + tok0, *reinterpret_cast<uint32_t(*)[32]>(u));
-          tmem_ld_32x32b_x32(t_row + kAccCol + 128 + tok0 + 32,
+          tmem_ld_32x32b_x32(t_row + kAccCol + C::kD1Col + tok0,
+                             *reinterpret_cast<uint32_t(*)[32]>(u));
+          tmem_ld_32x32b_x32(t_row + kAccCol + C::kD1Col + tok0 + 32,
                              *reinterpret_cast<uint32_t(*)[32]>(u + 32));
           tmem_ld_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.tmem_empty);
+          if (rho == rounds - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.tmem_empty);
+          }
           if (ntok > 0) {
 #pragma unroll
             for (int j = 0; j < 64; ++j) {
@@ -648,17 +749,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             // BF16 activation, token-major: feature f of n-tile nt is column
             // 128 * nt + f, i.e. byte 2 * (f % 64) of a row of activation tile
             // (m-tile, 2 * nt + f / 64).
-            uint8_t* tile = p.act + (static_cast<size_t>(t.mt) * (p.I / 64) + 2 * t.nt + (f >> 6)) *
+            uint8_t* tile = p.act + (static_cast<size_t>(mt) * (p.I / 64) + 2 * t.nt + (f >> 6)) *
                                         kTileBytes;
 #pragma unroll
             for (int j = 0; j < 64; ++j) {
               if (j < ntok) {
                 const float av = __uint_as_float(g[j]);
-                const int rr = tok0 + j;
+                const int rr = half * 64 + j;   // row of the m-tile
                 *reinterpret_cast<uint16_t*>(tile + swz128(rr, (f & 63) >> 3) + (f & 7) * 2) =
                     static_cast<uint16_t>(pack_bf16x2(av, 0.0f) & 0xFFFFu);
                 if (p.act_f32 != nullptr)
-                  p.act_f32[(static_cast<size_t>(t.mt) * BM + rr) * p.I + t.nt * 128 + f] = av;
+                  p.act_f32[(static_cast<size_t>(mt) * BM + rr) * p.I + t.nt * 128 + f] = av;
               }
             }
           } else if (ntok > 0) {
@@ -687,7 +788,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 sm.swap_red[half][q][32 * r + lane] = m[0];
               }
             }
-            if (!half_sync()) break;
+            if (!half_sync()) {
+              ok = false;
+              break;
+            }
             const int nb = p.I / 128;
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
@@ -698,47 +802,59 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int n = ue8m0_exponent(m);
                 if (q == 0) sm.swap_inv[half][j] = __uint_as_float(static_cast<uint32_t>(127 - n) << 23);
                 if (q == 0) {
-                  const int rr = tok0 + j;   // row of the m-tile
+                  const int rr = half * 64 + j;   // row of the m-tile
                   *reinterpret_cast<uint32_t*>(
-                      p.act_sf_chunks + (static_cast<size_t>(t.mt) * nb + t.nt) * 512 +
+                      p.act_sf_chunks + (static_cast<size_t>(mt) * nb + t.nt) * 512 +
                       (rr & 31) * 16 + (rr >> 5) * 4) = (static_cast<uint32_t>(n + 127) & 0xFFu) * 0x01010101u;
                 }
               }
             }
-            if (!half_sync()) break;
-            uint8_t* tile = p.act + (static_cast<size_t>(t.mt) * nb + t.nt) * kTileBytes;
+            if (!half_sync()) {
+              ok = false;
+              break;
+            }
+            uint8_t* tile = p.act + (static_cast<size_t>(mt) * nb + t.nt) * kTileBytes;
 #pragma unroll
             for (int j = 0; j < 64; ++j) {
               if (j < ntok) {
                 const float av = __uint_as_float(g[j]);
-                const int rr = tok0 + j;
+                const int rr = half * 64 + j;
                 tile[swz128(rr, f >> 4) + (f & 15)] =
                     static_cast<uint8_t>(cvt_e4m3x2(av * sm.swap_inv[half][j], 0.0f) & 0xFFu);
                 if (p.act_f32 != nullptr)
-                  p.act_f32[(static_cast<size_t>(t.mt) * BM + rr) * p.I + t.nt * 128 + f] = av;
+                  p.act_f32[(static_cast<size_t>(mt) * BM + rr) * p.I + t.nt * 128 + f] = av;
               }
             }
           }
+          }   // rounds
+          if (!ok) break;
           if (p.phases & 2) {
+            // Publish this warp's rows of every m-tile the tile covers.
             __threadfence();
             __syncwarp();
-            if (lane == 0) atomicAdd(p.fc1_done + t.mt, 1u);
+            if (lane == 0)
+              for (int rho = 0; rho < rounds; ++rho) atomicAdd(p.fc1_done + t.mt + rho, 1u);
           }
         } else {
+          const uint32_t dcol = kAccCol + (half ? C::kD1Col : 0u);   // this half's features
+          const int h = t.nt * 256 + half * 128 + f;   // output column
+          for (int rho = 0; rho < rounds; ++rho) {
           uint32_t v[128];
 #pragma unroll
           for (int c = 0; c < 4; ++c)
-            tmem_ld_32x32b_x32(t_row + kAccCol + half * 128 + c * 32,
+            tmem_ld_32x32b_x32(t_row + dcol + rho * BM + c * 32,
                                *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c));
           tmem_ld_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.tmem_empty);
-          const int h = t.nt * 256 + half * 128 + f;   // output column
+          if (rho == rounds - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.tmem_empty);
+          }
+          const int base = rho * BM;   // first token of this round
           int pl[4];
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            const int j = lane + 32 * c;
+            const int j = base + lane + 32 * c;
             pl[c] = j < t.rows ? p.perm[t.pos + j] : 0;
           }
 #pragma unroll
@@ -746,11 +862,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj) {
               const int sl = __shfl_sync(0xffffffffu, pl[c], jj);
-              if (c * 32 + jj < t.rows)
+              if (base + c * 32 + jj < t.rows)
                 p.y[static_cast<size_t>(sl) * p.H + h] =
                     static_cast<uint16_t>(pack_bf16x2(__uint_as_float(v[c * 32 + jj]), 0.0f) & 0xFFFFu);
             }
           }
+          }   // rounds
         }
         acc_phase ^= 1u;
         continue;
@@ -938,7 +1055,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
   return r == CUDA_SUCCESS;
 }
 
-template <int kW>
+template <int kW, bool kWide>
 cudaError_t launch_gemm(const moe_plan_s* pl, int phases, bool dynamic, const void* w1,
                         const uint8_t* w1s, const void* w2, const uint8_t* w2s, uint8_t* ws,
                         cudaStream_t st) {
@@ -989,6 +1106,7 @@ cudaError_t launch_gemm(const moe_plan_s* pl, int phases, bool dynamic, const vo
     max_tiles += (pl->rows_cap / BM) * p.ph[1].n_tiles;
   }
   p.tile_off = reinterpret_cast<const int32_t*>(ws + L.tile_off);
+  p.pair_off = reinterpret_cast<const int32_t*>(ws + L.pair_off);
   p.counts = reinterpret_cast<const int32_t*>(ws + L.counts);
   p.offsets = reinterpret_cast<const int32_t*>(ws + L.offsets);
   p.perm = reinterpret_cast<const int32_t*>(ws + L.perm);
@@ -1003,8 +1121,8 @@ cudaError_t launch_gemm(const moe_plan_s* pl, int phases, bool dynamic, const vo
   p.limit = pl->act.limit;
   p.y = reinterpret_cast<uint16_t*>(ws + L.y);
   p.err = reinterpret_cast<uint32_t*>(ws + L.err);
-  const size_t smem = sizeof(Smem) + 1024;
-  auto kern = moe_gemm_kernel<kW>;
+  const size_t smem = sizeof(SmemT<kWide>) + 1024;
+  auto kern = moe_gemm_kernel<kW, kWide>;
   cudaError_t e = ensure_max_dynamic_smem(reinterpret_cast<const void*>(kern),
                                           static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -1015,20 +1133,24 @@ cudaError_t launch_gemm(const moe_plan_s* pl, int phases, bool dynamic, const vo
 
 }  // namespace
 
-size_t gemm_smem_bytes() { return sizeof(Smem) + 1024; }
+size_t gemm_smem_bytes() { return sizeof(SmemT<false>) + 1024; }
 
 // phases: 1 FC1 only, 2 FC2 only, 3 both in one launch (dynamic scheduling).
 static cudaError_t launch_phases(const moe_plan_s* p, int phases, const void* w1,
                                  const uint8_t* w1s, const void* w2, const uint8_t* w2s,
                                  uint8_t* ws, cudaStream_t st) {
   const bool dyn = phases == 3;
+  const bool wide = use_wide(p) != 0;
   switch (p->w_dtype) {
     case MOE_W_E2M1_UE8M0_1x32:
-      return launch_gemm<kWFp4>(p, phases, dyn, w1, w1s, w2, w2s, ws, st);
+      return wide ? launch_gemm<kWFp4, true>(p, phases, dyn, w1, w1s, w2, w2s, ws, st)
+                  : launch_gemm<kWFp4, false>(p, phases, dyn, w1, w1s, w2, w2s, ws, st);
     case MOE_W_BF16:
-      return launch_gemm<kWBf16>(p, phases, dyn, w1, w1s, w2, w2s, ws, st);
+      return wide ? launch_gemm<kWBf16, true>(p, phases, dyn, w1, w1s, w2, w2s, ws, st)
+                  : launch_gemm<kWBf16, false>(p, phases, dyn, w1, w1s, w2, w2s, ws, st);
     default:
-      return launch_gemm<kWFp8>(p, phases, dyn, w1, w1s, w2, w2s, ws, st);
+      return wide ? launch_gemm<kWFp8, true>(p, phases, dyn, w1, w1s, w2, w2s, ws, st)
+                  : launch_gemm<kWFp8, false>(p, phases, dyn, w1, w1s, w2, w2s, ws, st);
   }
 }
 

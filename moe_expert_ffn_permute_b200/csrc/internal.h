@@ -47,6 +47,7 @@ struct moe_plan_s {
   int w_sf_chunked;      // MXFP4 scales given in 512-byte chunks (moe_prepack_weight_scales)
   int pair_mode;         // 2-SM GEMM: 0 automatic, 1 never, 2 always
   int swap_mode;         // token-major MMAs: 0 automatic, 1 never, 2 always
+  int wide_mode;         // wide token-major tiles (two m-tiles): 0 automatic, 1 never, 2 always
   // Copy streams and events of moe_forward_hostio_batches, created on its
   // first call on a device (io_device = that device, -1 before).
   int io_device;
@@ -62,6 +63,7 @@ namespace moe {
 
 void compute_layout(moe_plan_s* p);
 int use_swap(const moe_plan_s* p);    // token-major (swap-AB) MMAs: 0 never, 1 all, 2 by tile
+int use_wide(const moe_plan_s* p);    // 1: the GEMM kernel with wide token-major tiles
 
 // Launch with programmatic stream serialization: the kernel may start while its
 // predecessor in the stream finishes; it must execute griddep_wait() before

@@ -282,3 +282,35 @@ def test_weight_layout_values_per_format():
             assert got == status, (w_dtype, layout, got)
         assert moe.lib().moe_plan_set_weight_layout(p, 4) == 1
         moe.moe_plan_destroy(p)
+
+
+def test_wide_tile_selection():
+    """Wide token-major tiles: automatic for 96 < T*k/E <= 480 slots per expert,
+    forced on or off by mode, and never without token-major tiles."""
+    def active(T, k, E, **modes):
+        p = moe.moe_plan(T, 1024, 512, E, k)
+        if "swap" in modes:
+            moe.moe_plan_set_swap_ab(p, modes["swap"])
+        if "wide" in modes:
+            moe.moe_plan_set_wide_tiles(p, modes["wide"])
+        a = moe.moe_plan_wide_tiles_active(p)
+        moe.moe_plan_destroy(p)
+        return a
+    assert active(1024, 6, 48)                 # 128 slots per expert
+    assert active(2048, 4, 64)                 # 128
+    assert not active(128, 8, 32)              # 32: decode size
+    assert not active(8192, 8, 32)             # 2048: prefill size
+    assert active(97, 4, 4)                    # 97 slots per expert
+    assert not active(96, 4, 4)                # 96
+    assert active(480, 4, 4)                   # 480
+    assert not active(481, 4, 4)               # 481
+    assert active(128, 8, 32, wide=2)
+    assert not active(1024, 6, 48, wide=1)
+    assert not active(1024, 6, 48, swap=1)     # needs token-major tiles
+    assert not active(1024, 6, 48, swap=1, wide=2)
+    with pytest.raises(moe.MoEError):
+        p = moe.moe_plan(64, 512, 256, 8, 2)
+        try:
+            moe.moe_plan_set_wide_tiles(p, 3)
+        finally:
+            moe.moe_plan_destroy(p)

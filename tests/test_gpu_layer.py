@@ -630,3 +630,121 @@ def test_hostio_batches_equal_device_forwards(wl):
     torch.cuda.current_stream().synchronize()
     assert torch.equal(shared, ref[2])
     assert lay.check() == 0
+
+
+WIDE_SPLIT = Workload("wide-split", 600, 1024, 512, 8, 4, cfg_id=25)   # ~300 rows per expert
+RAGGED_BF16 = Workload("ragged-bf16", 300, 1024, 512, 8, 4, w_dtype="bf16", cfg_id=26)
+
+
+def _layer_wide(wl, wide, debug=False, tiled=False, swap=None):
+    return moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype=wl.w_dtype, act=wl.act,
+                        alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit, debug=debug,
+                        tiled_weights=tiled, chunked_scales=tiled and wl.w_dtype == "e2m1",
+                        swap_ab=swap, wide_tiles=wide)
+
+
+def _forward(lay, d, w1=None, w2=None, s1=None, s2=None):
+    out = lay.forward(d["x"], d["x_scales"], d["topk_idx"], d["topk_w"],
+                      d["w1"] if w1 is None else w1, d["w1_scales"] if s1 is None else s1,
+                      d["w2"] if w2 is None else w2, d["w2_scales"] if s2 is None else s2)
+    torch.cuda.synchronize()
+    return out
+
+
+@pytest.mark.parametrize("wl", [RAGGED, RAGGED_FP4, RAGGED_OAI, RAGGED_BF16, WIDE_SPLIT,
+                                WORKLOADS["tiny"], SINGLE], ids=lambda w: w.name)
+def test_wide_tiles_match_oracle(wl):
+    """Wide token-major tiles forced on: pairs of m-tiles with 129..240 rows
+    become one tile of N up to 240 tokens, larger pairs two tiles, lone
+    m-tiles one; whole-layer parity with the oracle for every weight format."""
+    d = inputs(wl)
+    lay = _layer_wide(wl, 2)
+    assert moe.moe_plan_wide_tiles_active(lay.plan)
+    out = _forward(lay, d)
+    assert lay.check() == 0
+    dn = to_numpy(d)
+    if wl.w_dtype == "bf16":
+        ref = L.layer_bf16(dn["x"], dn["topk_idx"], dn["topk_w"], dn["w1"], dn["w2"],
+                           alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit)
+    else:
+        ref = L.layer(*oracle_args(dn), **oracle_kw(wl))
+    assert_parity(out.float().cpu().numpy(), ref, f"wide {wl.name}")
+
+
+@pytest.mark.parametrize("w_dtype", ["e4m3", "e2m1"])
+def test_wide_tile_boundaries_240_and_241_rows(w_dtype):
+    """An expert with exactly 240 tokens (the widest tile: accumulators fill
+    TMEM columns 0..479) and one with 241 (split into 128 + 113 rows)."""
+    wl = Workload("wide-edge", 481, 1024, 512, 2, 1, w_dtype=w_dtype, cfg_id=27)
+    d = inputs(wl)
+    d["topk_idx"][:241, 0] = 0
+    d["topk_idx"][241:, 0] = 1
+    d["topk_w"].fill_(1.0)
+    lay = _layer_wide(wl, 2)
+    out = _forward(lay, d)
+    assert lay.check() == 0
+    ref = L.layer(*oracle_args(to_numpy(d)), **oracle_kw(wl))
+    assert_parity(out.float().cpu().numpy(), ref, "wide 240/241")
+    # the same tokens with token-row tiles only agree within rounding
+    ref_rows = _forward(_layer_wide(wl, 1, swap=1), d)
+    assert_parity(out.float().cpu().numpy(), ref_rows.float().cpu().numpy(), "wide vs rows")
+
+
+@pytest.mark.parametrize("wl", [RAGGED, RAGGED_FP4, WIDE_SPLIT], ids=lambda w: w.name)
+def test_wide_requant_bytes_exact(wl):
+    """With wide tiles the FC1 epilogue's two rounds of tokens write FP8 codes
+    and scales equal to the oracle quantiser on the GPU's own fp32 activation."""
+    d = inputs(wl)
+    lay = _layer_wide(wl, 2, debug=True)
+    _forward(lay, d)
+    v = lay.view()
+    rows = v.rows
+    act_t = torch.empty(rows, wl.I, dtype=torch.uint8, device="cuda")
+    moe.moe_copy_act(lay.plan, lay.workspace, act_t)
+    a32 = _ws_bytes(lay, v.act_f32, rows * wl.I * 4).view(torch.float32).view(rows, wl.I)
+    sf = torch.empty(rows, wl.I // 128, dtype=torch.uint8, device="cuda")
+    moe.moe_copy_act_scales(lay.plan, lay.workspace, sf)
+    counts = _ws_bytes(lay, v.counts, 4 * wl.E).view(torch.int32).cpu().numpy()
+    pad = _ws_bytes(lay, v.pad_offsets, 4 * (wl.E + 1)).view(torch.int32).cpu().numpy()
+    act, a32, sf = act_t.cpu().numpy(), a32.cpu().numpy(), sf.cpu().numpy()
+    assert counts.max() > 128
+    for e in range(wl.E):
+        r = slice(pad[e], pad[e] + counts[e])
+        q_ref, s_ref = L.requant_1x128(a32[r].astype(np.float64))
+        np.testing.assert_array_equal(act[r], q_ref, err_msg=f"codes, expert {e}")
+        np.testing.assert_array_equal(sf[r], s_ref, err_msg=f"scales, expert {e}")
+
+
+@pytest.mark.parametrize("wl", [RAGGED, RAGGED_FP4, WIDE_SPLIT], ids=lambda w: w.name)
+def test_wide_fused_equals_separate_tiled_equals_row_major_and_repeatable(wl):
+    d = inputs(wl)
+    lay = _layer_wide(wl, 2)
+    full = _forward(lay, d)
+    again = _forward(lay, d)
+    assert torch.equal(full, again)
+    v = lay.view()
+    n = wl.T * wl.k * wl.H * 2
+    off = v.y - lay.workspace.data_ptr()
+    y_fused = lay.workspace[off:off + n].clone()
+    moe.moe_route(lay.plan, d["topk_idx"], lay.workspace)
+    moe.moe_gather(lay.plan, d["x"], d["x_scales"], lay.workspace)
+    moe.moe_fc1(lay.plan, d["w1"], d["w1_scales"], lay.workspace)
+    moe.moe_fc2(lay.plan, d["w2"], d["w2_scales"], lay.workspace)
+    torch.cuda.synchronize()
+    assert torch.equal(lay.workspace[off:off + n], y_fused)
+    tl = _layer_wide(wl, 2, tiled=True)
+    w1, w2 = tl.prepack(d["w1"], d["w2"])
+    s1, s2 = ((tl.prepack_scales(d["w1_scales"], d["w2_scales"])) if wl.w_dtype == "e2m1"
+              else (d["w1_scales"], d["w2_scales"]))
+    assert torch.equal(_forward(tl, d, w1, w2, s1, s2), full)
+
+
+def test_wide_tiles_auto_at_the_mid_size_workloads():
+    for wl in (WORKLOADS["mxfp4"].with_tokens(1024), WORKLOADS["oai"]):
+        lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype=wl.w_dtype, act=wl.act,
+                           alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit)
+        assert moe.moe_plan_wide_tiles_active(lay.plan), wl.name
+    for name in ("decode", "prefill"):
+        wl = WORKLOADS[name]
+        lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k)
+        assert not moe.moe_plan_wide_tiles_active(lay.plan), name
