@@ -422,8 +422,10 @@ int moe_plan_swap_ab_active(moe_plan_t plan);
  * so an expert with 129..240 tokens streams its weights once instead of
  * twice; two accumulators of 128 weight rows x 240 tokens fill TMEM columns
  * 0..479.  The GEMM launch with wide tiles keeps three pipeline stages (its
- * stages hold two token tiles).  mode 0: automatic (wide tiles when the layer
- * has 96 < T*k/E <= 480 slots per expert), 1: never, 2: always.  Needs
+ * stages hold two token tiles).  mode 0: automatic (wide tiles for MXFP4
+ * weights when the layer has 96 < T*k/E <= 224 slots per expert, where they
+ * measured faster; FP8 and BF16 weights measured slower with them), 1: never,
+ * 2: always.  Needs
  * token-major tiles (not with moe_plan_set_swap_ab mode 1 or CTA pairs).
  * Results agree with the other tilings within rounding (the MMA's N and the
  * sum order inside it change) and are deterministic.                       */

@@ -123,17 +123,19 @@ int use_swap(const moe_plan_s* p) {
 }
 
 // Wide token-major tiles (up to 240 tokens of two consecutive m-tiles of one
-// expert in one tile): they need token-major MMAs, and pay off when experts
-// hold about one to two m-tiles of tokens -- then each expert's weights stream
-// once instead of twice.  Automatic mode uses them for 96 < S/E <= 480 slots
-// per expert; decode-sized layers (few tokens per expert, where the wide
-// kernel's three pipeline stages would cost) and large ones (mostly full
-// 128-row tiles) keep the four-stage kernel.
+// expert in one tile): they need token-major MMAs and halve the weight stream
+// of experts with 129..240 tokens.  Measured (same box, wide on vs off):
+// MXFP4 weights gain 12% at 128 and 15% at 192 slots per expert and lose 7% at
+// 96; FP8 and BF16 weights lose 7-14% at 128-192 (their pre-swizzled weight
+// tiles are cheap bulk copies, so the wide kernel's three stages and longer
+// epilogue outweigh the halved stream).  Automatic mode: MXFP4 weights with
+// 96 < S/E <= 224 slots per expert.
 int use_wide(const moe_plan_s* p) {
   if (use_swap(p) == 0 || p->wide_mode == 1) return 0;
   if (p->wide_mode == 2) return 1;
+  if (p->w_dtype != MOE_W_E2M1_UE8M0_1x32) return 0;
   const long long per_expert = p->S / p->E;
-  return per_expert > 96 && per_expert <= 480 ? 1 : 0;
+  return per_expert > 96 && per_expert <= 224 ? 1 : 0;
 }
 }  // namespace moe
 

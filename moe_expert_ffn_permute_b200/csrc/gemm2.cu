@@ -329,6 +329,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (leader && lane == 0) {
       int slot = 0, stage = 0;
       uint32_t sphase = 0, phase = 0, acc_phase = 0, sfset = 0;
+      // Stage-0 descriptors built once; a stage adds its byte offset >> 4 and
+      // a 32-byte K step adds 2 (the 14-bit address field cannot carry).
+      const uint64_t a_desc0 = umma_desc_sw128(smem_u32(sm.a[0]));
+      const uint64_t b_desc0 = umma_desc_sw128(smem_u32(sm.b[0]));
+      const uint64_t sfa_desc0 = sf_desc(smem_u32(sm.sfa[0]));
+      const uint64_t sfb_desc0 = sf_desc(smem_u32(sm.sfb[0]));
+      constexpr uint64_t kAStage = (BM * BK) >> 4, kBStage = ((BN / 2) * BK) >> 4;
+      constexpr uint64_t kSfaStage = 512 >> 4, kSfbStage = 1024 >> 4, kKStep = 32 >> 4;
       Task t;
       bool aborted = false;
       while (!aborted) {
@@ -351,15 +359,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t sfa = tmem + kSfaCol + sfset * kSfSetStride;
           const uint32_t sfb = tmem + kSfbCol + sfset * kSfSetStride;
-          tmem_cp_pair_32x128b_warpx4(sfa, sf_desc(smem_u32(sm.sfa[stage])));
-          tmem_cp_pair_32x128b_warpx4(sfb, sf_desc(smem_u32(sm.sfb[stage])));
-          tmem_cp_pair_32x128b_warpx4(sfb + 4, sf_desc(smem_u32(sm.sfb[stage] + 512)));
-          const uint32_t a_base = smem_u32(sm.a[stage]);
-          const uint32_t b_base = smem_u32(sm.b[stage]);
+          const uint64_t sfbd = sfb_desc0 + static_cast<uint64_t>(stage) * kSfbStage;
+          tmem_cp_pair_32x128b_warpx4(sfa, sfa_desc0 + static_cast<uint64_t>(stage) * kSfaStage);
+          tmem_cp_pair_32x128b_warpx4(sfb, sfbd);
+          tmem_cp_pair_32x128b_warpx4(sfb + 4, sfbd + (512 >> 4));
+          const uint64_t ad = a_desc0 + static_cast<uint64_t>(stage) * kAStage;
+          const uint64_t bd = b_desc0 + static_cast<uint64_t>(stage) * kBStage;
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {
-            mma_mxf8f6f4_pair(tmem + kAccCol, umma_desc_sw128(a_base + ks * 32),
-                              umma_desc_sw128(b_base + ks * 32), mxf8f6f4_idesc_m256(BN, ks),
+            mma_mxf8f6f4_pair(tmem + kAccCol, ad + ks * kKStep, bd + ks * kKStep,
+                              mxf8f6f4_idesc_m256(BN, ks),
                               sfa | (static_cast<uint32_t>(ks) << 30),
                               sfb | (static_cast<uint32_t>(ks) << 30),
                               (kb > 0 || ks > 0) ? 1u : 0u);

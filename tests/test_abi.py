@@ -285,10 +285,11 @@ def test_weight_layout_values_per_format():
 
 
 def test_wide_tile_selection():
-    """Wide token-major tiles: automatic for 96 < T*k/E <= 480 slots per expert,
-    forced on or off by mode, and never without token-major tiles."""
-    def active(T, k, E, **modes):
-        p = moe.moe_plan(T, 1024, 512, E, k)
+    """Wide token-major tiles: automatic for MXFP4 weights with 96 < T*k/E <= 224
+    slots per expert, forced on or off by mode, never without token-major
+    tiles."""
+    def active(T, k, E, w_dtype="e2m1", **modes):
+        p = moe.moe_plan(T, 1024, 512, E, k, w_dtype=w_dtype)
         if "swap" in modes:
             moe.moe_plan_set_swap_ab(p, modes["swap"])
         if "wide" in modes:
@@ -297,14 +298,17 @@ def test_wide_tile_selection():
         moe.moe_plan_destroy(p)
         return a
     assert active(1024, 6, 48)                 # 128 slots per expert
-    assert active(2048, 4, 64)                 # 128
-    assert not active(128, 8, 32)              # 32: decode size
-    assert not active(8192, 8, 32)             # 2048: prefill size
+    assert active(1536, 6, 48)                 # 192
+    assert not active(1024, 6, 48, "e4m3")     # FP8 and BF16 weights: never automatically
+    assert not active(2048, 4, 64, "e4m3")
+    assert not active(512, 8, 32, "bf16")
+    assert not active(128, 6, 48)              # 16: decode size
+    assert not active(8192, 6, 48)             # 1024: prefill size
     assert active(97, 4, 4)                    # 97 slots per expert
     assert not active(96, 4, 4)                # 96
-    assert active(480, 4, 4)                   # 480
-    assert not active(481, 4, 4)               # 481
-    assert active(128, 8, 32, wide=2)
+    assert active(224, 4, 4)                   # 224
+    assert not active(225, 4, 4)               # 225
+    assert active(128, 8, 32, "e4m3", wide=2)
     assert not active(1024, 6, 48, wide=1)
     assert not active(1024, 6, 48, swap=1)     # needs token-major tiles
     assert not active(1024, 6, 48, swap=1, wide=2)

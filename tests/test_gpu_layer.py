@@ -740,11 +740,12 @@ def test_wide_fused_equals_separate_tiled_equals_row_major_and_repeatable(wl):
 
 
 def test_wide_tiles_auto_at_the_mid_size_workloads():
-    for wl in (WORKLOADS["mxfp4"].with_tokens(1024), WORKLOADS["oai"]):
+    for T in (1024, 1536):
+        wl = WORKLOADS["mxfp4"].with_tokens(T)
+        lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype=wl.w_dtype)
+        assert moe.moe_plan_wide_tiles_active(lay.plan), wl.name
+    for name in ("decode", "prefill", "oai"):
+        wl = WORKLOADS[name]
         lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k, w_dtype=wl.w_dtype, act=wl.act,
                            alpha=wl.alpha, up_bias=wl.up_bias, limit=wl.limit)
-        assert moe.moe_plan_wide_tiles_active(lay.plan), wl.name
-    for name in ("decode", "prefill"):
-        wl = WORKLOADS[name]
-        lay = moe.MoELayer(wl.T, wl.H, wl.I, wl.E, wl.k)
         assert not moe.moe_plan_wide_tiles_active(lay.plan), name
