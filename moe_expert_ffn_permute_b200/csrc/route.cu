@@ -190,43 +190,88 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
   }
 }
 
-// Gather: padded row P (m-tile P / 128, row r = P % 128) of expert e receives
-// x[perm[offsets[e] + local + r] / k]; one warp per row, 16-byte accesses,
-// written in the pre-swizzled tile layout the FC1 producer bulk-copies.
-// Its scale bytes go to the tensor-core scale-chunk layout: for k-block kb the
-// 512-byte chunk of the tile holds, at byte (r % 32) * 16 + (r / 32) * 4 + j
-// (j = 0..3), the row's UE8M0 byte, replicated over the four 32-wide K
-// sub-blocks.  Padding rows are left untouched (their results are never
-// stored).
+// Gather, token-major: one warp per token.  The token's x row is read once
+// (in chunks of 8 x 16 bytes per lane) and written to the padded row of each
+// of its routed slots: slot s = t*k + j at sorted position inv[s] of expert e
+// (the e with offsets[e] <= inv[s] < offsets[e+1]) goes to padded row
+// pad_off[e] + inv[s] - offsets[e] (m-tile P / 128, row P % 128), in the
+// pre-swizzled tile layout the FC1 producer bulk-copies.  Its scale bytes go
+// to the tensor-core scale-chunk layout: for k-block kb the 512-byte chunk of
+// the tile holds, at byte (r % 32) * 16 + (r / 32) * 4 + j (j = 0..3), the
+// row's UE8M0 byte, replicated over the four 32-wide K sub-blocks.  Padding
+// rows are left untouched (their results are never stored).  Reading x once
+// per token instead of once per slot matters when x does not fit in L2.
 constexpr int kGatherWarps = 8;
+constexpr int kGatherBatch = 8;   // 16-byte vectors per lane per chunk
 
 __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(
-    const uint8_t* __restrict__ x, const uint8_t* __restrict__ xs, int row_bytes, int E,
-    const int32_t* __restrict__ pad_off, const int32_t* __restrict__ row_token,
-    uint8_t* __restrict__ xg, uint8_t* __restrict__ xg_sf) {
+    const uint8_t* __restrict__ x, const uint8_t* __restrict__ xs, int row_bytes, int T, int k,
+    int E, const int32_t* __restrict__ offsets, const int32_t* __restrict__ pad_off,
+    const int32_t* __restrict__ inv, uint8_t* __restrict__ xg, uint8_t* __restrict__ xg_sf) {
+  __shared__ int32_t s_off[257];
+  __shared__ int32_t s_pad[257];
   griddep_launch_dependents();
   griddep_wait();
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+    s_off[e] = __ldg(&offsets[e]);
+    s_pad[e] = __ldg(&pad_off[e]);
+  }
+  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long P = static_cast<long long>(blockIdx.x) * kGatherWarps + warp;
-  if (P >= __ldg(&pad_off[E])) return;
-  const int t = __ldg(&row_token[P]);
-  if (t < 0) return;   // padding row
-  const int tile = static_cast<int>(P / kTileM);
-  const int r = static_cast<int>(P % kTileM);
+  const int t = blockIdx.x * kGatherWarps + warp;
+  if (t >= T) return;
   const int vec = row_bytes / 16;
   const int kb_n = row_bytes / 128;
-  const uint4* __restrict__ src =
-      reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * row_bytes);
-  // Destination: pre-swizzled 128 x 128-byte tiles [tile][k-block][16 KB].
-  uint8_t* __restrict__ dst = xg + static_cast<size_t>(tile) * kb_n * kTileBytes;
-  for (int c = lane; c < vec; c += 32)
-    *reinterpret_cast<uint4*>(dst + static_cast<size_t>(c >> 3) * kTileBytes + swz128(r, c & 7)) =
-        __ldg(&src[c]);
-  if (xs == nullptr) return;   // BF16 activations: no scales
-  uint8_t* chunk = xg_sf + static_cast<size_t>(tile) * kb_n * 512 + (r & 31) * 16 + (r >> 5) * 4;
-  for (int kb = lane; kb < kb_n; kb += 32) {
-    const uint32_t b = __ldg(&xs[static_cast<size_t>(t) * kb_n + kb]);
-    *reinterpret_cast<uint32_t*>(chunk + static_cast<size_t>(kb) * 512) = b * 0x01010101u;
+  const uint4* __restrict__ src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * row_bytes);
+  for (int j0 = 0; j0 < k; j0 += 32) {
+    // Lane l resolves slot j0 + l's padded row (-1: not routed).
+    int prow = -1;
+    if (j0 + lane < k) {
+      const int pos = __ldg(&inv[static_cast<size_t>(t) * k + j0 + lane]);
+      if (pos >= 0) {
+        int lo = 0, hi = E - 1;   // largest e with offsets[e] <= pos
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (s_off[mid] <= pos) lo = mid; else hi = mid - 1;
+        }
+        prow = s_pad[lo] + (pos - s_off[lo]);
+      }
+    }
+    const int nj = min(32, k - j0);
+    for (int c0 = 0; c0 < vec; c0 += 32 * kGatherBatch) {
+      uint4 v[kGatherBatch];
+#pragma unroll
+      for (int u = 0; u < kGatherBatch; ++u) {
+        const int c = c0 + lane + 32 * u;
+        if (c < vec) v[u] = __ldg(&src[c]);
+      }
+      for (int jj = 0; jj < nj; ++jj) {
+        const int P = __shfl_sync(0xffffffffu, prow, jj);
+        if (P < 0) continue;
+        uint8_t* __restrict__ dst =
+            xg + static_cast<size_t>(P / kTileM) * kb_n * kTileBytes;
+        const int r = P % kTileM;
+#pragma unroll
+        for (int u = 0; u < kGatherBatch; ++u) {
+          const int c = c0 + lane + 32 * u;
+          if (c < vec)
+            *reinterpret_cast<uint4*>(dst + static_cast<size_t>(c >> 3) * kTileBytes +
+                                      swz128(r, c & 7)) = v[u];
+        }
+      }
+    }
+    if (xs == nullptr) continue;   // BF16 activations: no scales
+    for (int jj = 0; jj < nj; ++jj) {
+      const int P = __shfl_sync(0xffffffffu, prow, jj);
+      if (P < 0) continue;
+      const int r = P % kTileM;
+      uint8_t* chunk = xg_sf + static_cast<size_t>(P / kTileM) * kb_n * 512 + (r & 31) * 16 +
+                       (r >> 5) * 4;
+      for (int kb = lane; kb < kb_n; kb += 32) {
+        const uint32_t b = __ldg(&xs[static_cast<size_t>(t) * kb_n + kb]);
+        *reinterpret_cast<uint32_t*>(chunk + static_cast<size_t>(kb) * 512) = b * 0x01010101u;
+      }
+    }
   }
 }
 
@@ -458,11 +503,13 @@ cudaError_t launch_route(const moe_plan_s* p, const int32_t* topk_idx, uint8_t* 
 cudaError_t launch_gather(const moe_plan_s* p, const uint8_t* x, const uint8_t* xs, uint8_t* ws,
                           cudaStream_t st) {
   const auto& L = p->ws;
-  const int blocks = static_cast<int>(p->rows_cap / kGatherWarps);
+  const int blocks = (p->T + kGatherWarps - 1) / kGatherWarps;   // one warp per token
   const bool bf16 = p->w_dtype == MOE_W_BF16;   // 2-byte activations, no scales
   return launch_pdl(gather_kernel, dim3(blocks), dim3(kGatherWarps * 32), 0, st, x,
-                    bf16 ? nullptr : xs, p->H * (bf16 ? 2 : 1), p->E, reinterpret_cast<const int32_t*>(ws + L.pad_off),
-                    reinterpret_cast<const int32_t*>(ws + L.row_token), ws + L.xg, ws + L.xg_sf);
+                    bf16 ? nullptr : xs, p->H * (bf16 ? 2 : 1), p->T, p->k, p->E,
+                    reinterpret_cast<const int32_t*>(ws + L.offsets),
+                    reinterpret_cast<const int32_t*>(ws + L.pad_off),
+                    reinterpret_cast<const int32_t*>(ws + L.inv), ws + L.xg, ws + L.xg_sf);
 }
 
 cudaError_t launch_route_gather(const moe_plan_s* p, const int32_t* topk_idx, const uint8_t* x,
