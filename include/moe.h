@@ -180,7 +180,9 @@ moe_status moe_forward_hostio(moe_plan_t plan, const void *x_host,
  * Results are byte-identical to moe_forward on the same inputs.
  * Errors: MOE_ERR_INVALID_ARG for n_batches < 1 or a NULL array or entry
  * (x_scales_host may be NULL for MOE_W_BF16), checked before anything is
- * enqueued; MOE_ERR_CUDA if creating the copy streams or an enqueue fails.
+ * enqueued; MOE_ERR_CUDA if creating the copy streams or an enqueue fails --
+ * then the batches enqueued before the failure stay enqueued (synchronise
+ * `stream` and the device before reusing the buffers).
  * No counterpart on the pages (a host-buffer serving loop around
  * moe_forward).
  */
