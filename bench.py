@@ -463,6 +463,7 @@ def measure_rank(args, dev):
             "alg_bytes": lb.alg_bytes, "w_bytes": lb.w_bytes, "pairs": lb.pairs,
             "tiled": lb.tiled, "chunked": lb.chunked,
             "swap": lb.moe.moe_plan_swap_ab_active(lb.lay.plan),
+            "wide": lb.moe.moe_plan_wide_tiles_active(lb.lay.plan),
             "launches": lb.moe.moe_forward_launch_count(lb.lay.plan)}
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
@@ -485,7 +486,7 @@ def measure_rank(args, dev):
                 raise RuntimeError(f"device error during timing of {w.name}")
             per.append({"wl": w, "step_ms": ms, "split": sp, "active": b.active,
                         "alg_bytes": b.alg_bytes, "w_bytes": b.w_bytes, "pairs": b.pairs,
-                        "clocks": cc})
+                        "clocks": cc, "wide": b.moe.moe_plan_wide_tiles_active(b.lay.plan)})
             b.release()
     return main, per, cpu
 
@@ -525,7 +526,8 @@ def assemble_line(args, world, device, main, per, cpu):
                                "row-major"),
                    "gemm_tiles": {0: "token rows", 1: "token-major (swap AB)",
                                   2: "token-major for tiles of <= 96 tokens, else token rows"}[
-                       main["swap"]],
+                       main["swap"]] + ("; wide token-major tiles over two m-tiles (up to 240 "
+                                        "tokens)" if main.get("wide") else ""),
                    "parallelism": f"replicas x{world}"},
         "achieved": {"tflops": round(flops / (ms_per_step * 1e-3) / 1e12, 2),
                      "hbm_gbs": round(main["alg_bytes"] / (ms_per_step * 1e-3) / 1e9, 1),
@@ -556,7 +558,7 @@ def assemble_line(args, world, device, main, per, cpu):
             "combine_ms": round(red[("per", i, "combine")], 4),
             "roofline": {k: roof[k] for k in ("bound", "achieved", "peak", "unit", "frac")},
             "sm_mhz": p["clocks"].get("sm_mhz"), "reasons": p["clocks"].get("reasons"),
-            "steps": n})
+            "wide_tiles": bool(p.get("wide")), "steps": n})
     if per_out:
         res["per_config"] = per_out
     if cpu is not None:

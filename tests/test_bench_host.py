@@ -69,3 +69,33 @@ def test_reference_arm_line_on_the_small_config():
     assert 1 <= line["config"]["active_experts"] <= wl.E
     assert line["e2e"]["value"] == line["value"]
     assert line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_gpus_without_a_launcher_respawns_under_torchrun(monkeypatch):
+    """`bench.py --gpus N` with no WORLD_SIZE in the environment starts N ranks
+    of the same command under torch.distributed.run (one process per GPU, the
+    rendezvous on 127.0.0.1) and exits with its status."""
+    import sys
+    bench = _load_bench()
+    calls = []
+    monkeypatch.setattr(bench.subprocess, "call", lambda cmd: calls.append(cmd) or 0)
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--gpus", "4", "--steps", "7"])
+    with pytest.raises(SystemExit) as ei:
+        bench.main()
+    assert ei.value.code == 0
+    (cmd,) = calls
+    assert cmd[1:4] == ["-m", "torch.distributed.run", "--nnodes=1"]
+    assert "--nproc-per-node=4" in cmd
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "7"]
+
+
+def test_gpus_disagreeing_with_world_size_is_refused(monkeypatch):
+    import sys
+    bench = _load_bench()
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--gpus", "4"])
+    with pytest.raises(SystemExit) as ei:
+        bench.main()
+    assert "WORLD_SIZE=2" in str(ei.value.code)
