@@ -20,7 +20,10 @@ ROOT = os.path.abspath(os.path.join(os.path.dirname(__file__), ".."))
 F, L = "oracle/formats.py", "oracle/layer.py"
 PIN_TESTS = ["tests/test_oracle_formats.py", "tests/test_oracle_layer.py",
              "tests/test_oracle_bf16.py", "tests/test_oracle_route_property.py",
-             "tests/test_oracle_requant_property.py", "tests/test_golden_params.py"]
+             "tests/test_oracle_requant_property.py", "tests/test_golden_params.py",
+             "tests/test_workload_recipe.py"]
+# What a scratch copy needs for the pin tests to import and run.
+COPIED = ("oracle", "tests", "workloads", "moe_expert_ffn_permute_b200")
 
 _TAIL = ("                out[t] += w[t, j] * y[t * k + j]\n    if keep:\n        inter.update("
          "counts=counts, offsets=offsets, perm=perm, inv=inv, y=y)\n        return out, inter\n"
@@ -116,16 +119,35 @@ MUTANTS = [
 ]
 
 
+def _scratch_copy(scratch_root):
+    scratch = tempfile.mkdtemp(prefix="oracle_mutant_", dir=scratch_root)
+    for d in COPIED:
+        shutil.copytree(os.path.join(ROOT, d), os.path.join(scratch, d),
+                        ignore=shutil.ignore_patterns("*.so", "_build", "__pycache__"))
+    return scratch
+
+
+def _pins(scratch):
+    return subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                           *PIN_TESTS], cwd=scratch, capture_output=True, text=True)
+
+
 def run(selected=None, scratch_root=None):
+    # The unmutated copy must pass, or every mutant would look caught.
+    scratch = _scratch_copy(scratch_root)
+    try:
+        base = _pins(scratch)
+    finally:
+        shutil.rmtree(scratch, ignore_errors=True)
+    if base.returncode != 0:
+        print("the pins fail on an unmutated copy; nothing to check:\n" + base.stdout[-2000:])
+        return False
     survivors, missing = [], []
     for i, (rel, text, repl, note) in enumerate(MUTANTS):
         if selected and i not in selected:
             continue
-        scratch = tempfile.mkdtemp(prefix="oracle_mutant_", dir=scratch_root)
+        scratch = _scratch_copy(scratch_root)
         try:
-            for d in ("oracle", "tests", "moe_expert_ffn_permute_b200"):
-                shutil.copytree(os.path.join(ROOT, d), os.path.join(scratch, d),
-                                ignore=shutil.ignore_patterns("*.so", "_build", "__pycache__"))
             path = os.path.join(scratch, rel)
             with open(path) as f:
                 src = f.read()
@@ -135,8 +157,7 @@ def run(selected=None, scratch_root=None):
                 continue
             with open(path, "w") as f:
                 f.write(src.replace(text, repl, 1))
-            r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
-                                *PIN_TESTS], cwd=scratch, capture_output=True, text=True)
+            r = _pins(scratch)
         finally:
             shutil.rmtree(scratch, ignore_errors=True)
         caught = r.returncode != 0
