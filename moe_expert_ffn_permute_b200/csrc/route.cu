@@ -39,16 +39,22 @@ __global__ void __launch_bounds__(kRouteThreads) route_hist_kernel(
   for (int e = tid; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
   const int base = blockIdx.x * kRouteChunk;
+  // All of this thread's ids are loaded before any is counted (one round trip).
+  constexpr int kPer = kRouteChunk / kRouteThreads;
+  int v[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int s = base + tid + u * kRouteThreads;
+    v[u] = s < S ? __ldg(&idx[s]) : kMaskedSlot;
+  }
   bool bad = false;
-  for (int i = tid; i < kRouteChunk; i += blockDim.x) {
-    const int s = base + i;
-    if (s < S) {
-      const int e = idx[s];
-      if (e >= 0 && e < E) {
-        atomicAdd(&hist[e], 1);
-      } else if (e != kMaskedSlot) {
-        bad = true;
-      }
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int e = v[u];
+    if (e >= 0 && e < E) {
+      atomicAdd(&hist[e], 1);
+    } else if (e != kMaskedSlot) {
+      bad = true;
     }
   }
   if (bad) atomicOr(err, kErrRoutingBit);
@@ -84,6 +90,16 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
   __shared__ int32_t tscan[257];   // padded m-tile offsets
   __shared__ int32_t wcount[kWarps][256];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int base = blockIdx.x * kRouteChunk;
+  // The block's ids, loaded once up front (their latency overlaps the scan
+  // below) instead of once per sub-chunk.
+  constexpr int kPer = kRouteChunk / kRouteThreads;
+  int v[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int s = base + tid + u * kRouteThreads;
+    v[u] = s < S ? __ldg(&idx[s]) : kMaskedSlot;
+  }
   if (nblk == 1) {
     // A single block holds every slot: count them here (no histogram launch).
     for (int e = tid; e < E; e += blockDim.x) {
@@ -92,8 +108,9 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
     }
     __syncthreads();
     bool bad = false;
-    for (int s = tid; s < S; s += blockDim.x) {
-      const int e = idx[s];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {   // S <= kRouteChunk: every id is in v
+      const int e = v[u];
       if (e >= 0 && e < E) atomicAdd(&total[e], 1); else if (e != kMaskedSlot) bad = true;
     }
     if (bad) atomicOr(err, kErrRoutingBit);
@@ -147,16 +164,17 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
   }
   // Positions past the routed slots (left by out-of-range ids) read -1.
   const int routed = scan[E];
-  const int base = blockIdx.x * kRouteChunk;
   for (int p = base + tid; p < base + kRouteChunk && p < S; p += blockDim.x)
     if (p >= routed) perm[p] = -1;
-  for (int sub = 0; sub < kRouteChunk; sub += kRouteThreads) {
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int sub = u * kRouteThreads;
     for (int i = tid; i < kWarps * 256; i += blockDim.x) (&wcount[0][0])[i] = 0;
     __syncthreads();
     const int s = base + sub + tid;
     int e = -1;
     if (s < S) {
-      e = idx[s];
+      e = v[u];
       if (e < 0 || e >= E) e = -1;
     }
     const unsigned peers = __match_any_sync(0xffffffffu, e);
@@ -276,16 +294,24 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(
 }
 
 // Routing and gather in one launch, for small slot counts (S <= kFusedMaxSlots):
-// every block loads the slot ids into shared memory and repeats the counting
-// sort there (histogram, exclusive scan, stable scatter by __match_any_sync
-// ranks, as route_scatter_kernel), so no block waits for another; block 0
-// also publishes what the separate routing launch writes (counts, offsets,
-// tile / pad / pair offsets, perm, inv, the row -> token map, the zeroed
-// GEMM counters, the error bit).  Then each warp copies routed rows: sorted
-// position pos of expert e goes to padded row 128 * tile_off[e] + pos -
+// every block repeats the counting sort for all S slots, so no block waits for
+// another; block 0 also publishes what the separate routing launch writes
+// (counts, offsets, tile / pad / pair offsets, perm, inv, the row -> token map,
+// the zeroed GEMM counters, the error bit).  Then each warp copies routed rows:
+// sorted position pos of expert e goes to padded row 128 * tile_off[e] + pos -
 // offsets[e], from token perm[pos] / k, in the same tiled layout and scale
 // chunks as gather_kernel.  The bytes written equal those of the two separate
 // launches.
+//
+// The sort is warp-local until one block-wide scan: warp w owns the contiguous
+// slots [w * C, (w + 1) * C) and walks them 32 at a time, ranking each slot
+// among the group's equal experts with __match_any_sync and keeping a running
+// count per expert in its own row of shared memory (warp-synchronous, no block
+// barrier per group).  A slot's sorted position is then the expert's offset,
+// plus the slots of that expert in lower warps, plus its rank inside the warp:
+// ascending slot order within each expert, as the stable scatter requires.
+// Thread e computes expert e's totals, and the exclusive scans over experts
+// (slots, padded m-tiles, m-tile pairs) are block scans over those threads.
 __global__ void __launch_bounds__(kRouteThreads) route_gather_kernel(
     const int32_t* __restrict__ idx, int S, int E, int k, const uint8_t* __restrict__ x,
     const uint8_t* __restrict__ xs, int row_bytes, int32_t* __restrict__ counts,
@@ -294,113 +320,127 @@ __global__ void __launch_bounds__(kRouteThreads) route_gather_kernel(
     uint32_t* err, uint32_t* __restrict__ sched, int sched_words,
     int32_t* __restrict__ row_token, uint8_t* __restrict__ xg, uint8_t* __restrict__ xg_sf) {
   constexpr int kWarps = kRouteThreads / 32;
-  extern __shared__ int32_t dyn[];
-  int32_t* ids = dyn;          // [S] expert id per slot (-1: not routed)
-  int32_t* sorted = dyn + S;   // [S] slot at each sorted position
-  __shared__ int32_t running[256];
-  __shared__ int32_t total[256];
+  constexpr int kPer = kFusedMaxSlots / kRouteThreads;   // 32-slot groups per warp, at most
+  constexpr int kNone = -1;                              // packed value of an unrouted slot
+  extern __shared__ int32_t sorted[];   // [S] slot at each sorted position
+  __shared__ int32_t wpre[kWarps][256];  // per warp and expert: count, then lower warps' count
+  __shared__ int32_t total[257];
   __shared__ int32_t scan[257];
-  __shared__ int32_t tscan[257];
-  __shared__ int32_t wcount[kWarps][256];
+  __shared__ int32_t tscan[257];        // padded m-tile offsets
+  __shared__ int32_t part[3][kWarps];   // per-warp sums for the block scans
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool lead = blockIdx.x == 0;
+  const int chunk = (S + 32 * kWarps - 1) / (32 * kWarps) * 32;   // slots per warp
   griddep_launch_dependents();
   griddep_wait();
   if (lead && sched != nullptr)
     for (int i = tid; i < sched_words; i += blockDim.x) sched[i] = 0u;
-  for (int e = tid; e < E; e += blockDim.x) total[e] = 0;
-  __syncthreads();
-  bool bad = false;
-  // All of this thread's ids are loaded before any is used (one round trip).
-  constexpr int kPer = kFusedMaxSlots / kRouteThreads;
+  for (int e = lane; e < E; e += 32) wpre[warp][e] = 0;
+  // This warp's ids, all loaded before any is used (one round trip).
   int v[kPer];
 #pragma unroll
   for (int u = 0; u < kPer; ++u) {
-    const int i = tid + u * kRouteThreads;
-    v[u] = i < S ? __ldg(&idx[i]) : kMaskedSlot;
+    const int s = warp * chunk + u * 32 + lane;
+    v[u] = u * 32 < chunk && s < S ? __ldg(&idx[s]) : kMaskedSlot;
   }
+  __syncwarp();
+  bool bad = false;
+  const unsigned lower = (1u << lane) - 1u;
 #pragma unroll
   for (int u = 0; u < kPer; ++u) {
-    const int i = tid + u * kRouteThreads;
-    if (i >= S) break;
+    if (u * 32 >= chunk) break;   // warp-uniform
     int e = v[u];
-    if (e >= 0 && e < E) {
-      atomicAdd(&total[e], 1);
-    } else {
+    if (!(e >= 0 && e < E)) {
       if (e != kMaskedSlot) bad = true;
       e = -1;
     }
-    ids[i] = e;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int before = e >= 0 ? wpre[warp][e] : 0;
+    __syncwarp();   // every lane has read its count before the group's leader updates it
+    if (e >= 0 && (peers & lower) == 0) wpre[warp][e] = before + __popc(peers);
+    __syncwarp();
+    v[u] = e >= 0 ? ((before + __popc(peers & lower)) << 9) | e : kNone;
   }
   if (lead && bad) atomicOr(err, kErrRoutingBit);
   __syncthreads();
-  if (tid == 0) {
-    int acc = 0, tacc = 0, pacc = 0;
-    for (int e = 0; e < E; ++e) {
-      scan[e] = acc;
-      tscan[e] = tacc;
-      running[e] = acc;
-      const int tiles = (total[e] + kTileM - 1) / kTileM;
-      if (lead) {
-        offsets[e] = acc;
-        counts[e] = total[e];
-        tile_off[e] = tacc;
-        pad_off[e] = tacc * kTileM;
-        pair_off[e] = pacc;
-      }
-      acc += total[e];
-      tacc += tiles;
-      pacc += (tiles + 1) / 2;
+  // Thread e: expert e's total, and its per-warp counts turned into the count
+  // of expert e in lower warps.
+  int tot = 0;
+  if (tid < E) {
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const int c = wpre[w][tid];
+      wpre[w][tid] = tot;
+      tot += c;
     }
-    scan[E] = acc;
-    tscan[E] = tacc;
+    total[tid] = tot;
+  }
+  const int tiles = (tot + kTileM - 1) / kTileM;
+  const int pairs = (tiles + 1) / 2;
+  // Inclusive scans over threads (experts) of tot, tiles and pairs.
+  int a = tot, b = tiles, c = pairs;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int a2 = __shfl_up_sync(0xffffffffu, a, off);
+    const int b2 = __shfl_up_sync(0xffffffffu, b, off);
+    const int c2 = __shfl_up_sync(0xffffffffu, c, off);
+    if (lane >= off) { a += a2; b += b2; c += c2; }
+  }
+  if (lane == 31) { part[0][warp] = a; part[1][warp] = b; part[2][warp] = c; }
+  __syncthreads();
+  for (int w = 0; w < warp; ++w) { a += part[0][w]; b += part[1][w]; c += part[2][w]; }
+  if (tid < E) {
+    const int ex = a - tot, tex = b - tiles, pex = c - pairs;
+    scan[tid] = ex;
+    tscan[tid] = tex;
     if (lead) {
-      offsets[E] = acc;
-      tile_off[E] = tacc;
-      pad_off[E] = tacc * kTileM;
-      pair_off[E] = pacc;
+      offsets[tid] = ex;
+      counts[tid] = tot;
+      tile_off[tid] = tex;
+      pad_off[tid] = tex * kTileM;
+      pair_off[tid] = pex;
+    }
+    if (tid == E - 1) {
+      scan[E] = a;
+      tscan[E] = b;
+      if (lead) {
+        offsets[E] = a;
+        tile_off[E] = b;
+        pad_off[E] = b * kTileM;
+        pair_off[E] = c;
+      }
     }
   }
   __syncthreads();
   const int routed = scan[E];
   if (lead) {
-    for (int e = 0; e < E; ++e) {
+    // Padding rows of the row -> token map read -1; so do positions past the
+    // routed slots (left by masked or out-of-range ids).
+    for (int e = warp; e < E; e += kWarps) {
       const int lo = tscan[e] * kTileM + total[e], hi = tscan[e + 1] * kTileM;
-      for (int r = lo + tid; r < hi; r += blockDim.x) row_token[r] = -1;
+      for (int r = lo + lane; r < hi; r += 32) row_token[r] = -1;
     }
     for (int q = routed + tid; q < S; q += blockDim.x) perm[q] = -1;
   }
-  for (int sub = 0; sub < S; sub += kRouteThreads) {
-    for (int i = tid; i < kWarps * 256; i += blockDim.x) (&wcount[0][0])[i] = 0;
-    __syncthreads();
-    const int sl = sub + tid;
-    const int e = sl < S ? ids[sl] : -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    if (e >= 0 && rank == 0) wcount[warp][e] = __popc(peers);
-    __syncthreads();
-    if (sl < S) {
-      if (e >= 0) {
-        int q = running[e] + rank;
-        for (int w = 0; w < warp; ++w) q += wcount[w][e];
-        sorted[q] = sl;   // q < routed <= S: the counts above bound it
-        if (lead) {
-          perm[q] = sl;
-          inv[sl] = q;
-          row_token[tscan[e] * kTileM + (q - scan[e])] = sl / k;
-        }
-      } else if (lead) {
-        inv[sl] = -1;
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    if (u * 32 >= chunk) break;
+    const int s = warp * chunk + u * 32 + lane;
+    if (s >= S) continue;
+    if (v[u] != kNone) {
+      const int e = v[u] & 511;
+      const int q = scan[e] + wpre[warp][e] + (v[u] >> 9);
+      sorted[q] = s;   // q < routed <= S: the counts above bound it
+      if (lead) {
+        perm[q] = s;
+        inv[s] = q;
+        row_token[tscan[e] * kTileM + (q - scan[e])] = s / k;
       }
+    } else if (lead) {
+      inv[s] = -1;
     }
-    __syncthreads();
-    for (int ee = tid; ee < E; ee += blockDim.x) {
-      int add = 0;
-      for (int w = 0; w < kWarps; ++w) add += wcount[w][ee];
-      running[ee] += add;
-    }
-    __syncthreads();
   }
+  __syncthreads();
   // Gather: one warp per routed row; all loads of a row are issued before its
   // stores.
   const int kb_n = row_bytes / 128;   // 128-byte k-blocks per row (scale blocks when FP8)
@@ -521,8 +561,15 @@ cudaError_t launch_route_gather(const moe_plan_s* p, const int32_t* topk_idx, co
   const bool bf16 = p->w_dtype == MOE_W_BF16;   // 2-byte activations, no scales
   const int want = (S + kRouteThreads / 32 - 1) / (kRouteThreads / 32);
   const int blocks = std::max(1, std::min(want, 2 * sms));
+  const int dyn = S * static_cast<int>(sizeof(int32_t));   // the sorted slot list
+  if (dyn > 48 * 1024) {
+    const cudaError_t a = ensure_max_dynamic_smem(
+        reinterpret_cast<const void*>(route_gather_kernel),
+        kFusedMaxSlots * static_cast<int>(sizeof(int32_t)));
+    if (a != cudaSuccess) return a;
+  }
   return launch_pdl(
-      route_gather_kernel, dim3(blocks), dim3(kRouteThreads), 2 * S * sizeof(int32_t), st,
+      route_gather_kernel, dim3(blocks), dim3(kRouteThreads), dyn, st,
       topk_idx, S, p->E, p->k, x, bf16 ? nullptr : xs, p->H * (bf16 ? 2 : 1),
       reinterpret_cast<int32_t*>(ws + L.counts),
       reinterpret_cast<int32_t*>(ws + L.offsets), reinterpret_cast<int32_t*>(ws + L.tile_off),
