@@ -62,14 +62,83 @@ __global__ void __launch_bounds__(kRouteThreads) route_hist_kernel(
   for (int e = tid; e < E; e += blockDim.x) block_hist[blockIdx.x * E + e] = hist[e];
 }
 
+// Block-wide exclusive scans over the experts: thread e holds expert e's
+// routed-slot count (0 for e >= E) and gets the expert's slot offset, padded
+// m-tile offset and m-tile-pair offset, plus the inclusive values (the totals,
+// at thread E - 1).  `part` is shared scratch; contains one block barrier.
+struct ExpertOffsets {
+  int slot, tile, pair;            // exclusive
+  int slot_end, tile_end, pair_end;   // inclusive
+};
+__device__ __forceinline__ ExpertOffsets expert_offsets(int count,
+                                                        int32_t (*part)[kRouteThreads / 32]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int tiles = (count + kTileM - 1) / kTileM;
+  const int pairs = (tiles + 1) / 2;
+  int a = count, b = tiles, c = pairs;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int a2 = __shfl_up_sync(0xffffffffu, a, off);
+    const int b2 = __shfl_up_sync(0xffffffffu, b, off);
+    const int c2 = __shfl_up_sync(0xffffffffu, c, off);
+    if (lane >= off) {
+      a += a2;
+      b += b2;
+      c += c2;
+    }
+  }
+  if (lane == 31) {
+    part[0][warp] = a;
+    part[1][warp] = b;
+    part[2][warp] = c;
+  }
+  __syncthreads();
+  for (int w = 0; w < warp; ++w) {
+    a += part[0][w];
+    b += part[1][w];
+    c += part[2][w];
+  }
+  return {a - count, b - tiles, c - pairs, a, b, c};
+}
+
+// Rank a warp's slots among equal experts.  The warp owns `groups` groups of
+// 32 consecutive slots (ids in v, one per lane and group; -1 for a masked or
+// absent slot, any other id outside [0, E) is reported through `bad`) and
+// keeps its running count per expert in `count[e]` (its own row of shared
+// memory, zeroed by the caller).  On return v[u] holds (rank << 9) | e for a
+// routed slot -- its rank among the warp's slots of expert e, in slot order --
+// and kUnrouted otherwise.
+constexpr int kUnrouted = -1;
+template <int kPer>
+__device__ __forceinline__ void rank_in_warp(int (&v)[kPer], int groups, int E,
+                                             int32_t* count, bool& bad) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lower = (1u << lane) - 1u;
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    if (u >= groups) break;   // warp-uniform
+    int e = v[u];
+    if (!(e >= 0 && e < E)) {
+      if (e != kMaskedSlot) bad = true;
+      e = -1;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int before = e >= 0 ? count[e] : 0;
+    __syncwarp();   // every lane has read its count before the group's leader updates it
+    if (e >= 0 && (peers & lower) == 0) count[e] = before + __popc(peers);
+    __syncwarp();
+    v[u] = e >= 0 ? ((before + __popc(peers & lower)) << 9) | e : kUnrouted;
+  }
+}
+
 // Kernel 2: scan + stable scatter.  Every block re-derives, from the block
-// histograms, the per-expert totals, the exclusive scan over experts and its
+// histograms, the per-expert totals, the exclusive scans over experts and its
 // own starting position per expert (the histograms are small, so this costs
 // less than a separate scan launch); block 0 publishes counts / offsets and
-// the padded tile offsets.  Then the block walks its chunk in sub-chunks of
-// 256 slots: inside a warp the rank of a slot among equal experts comes from
-// __match_any_sync, across warps from per-warp counts, across sub-chunks from
-// a running count per expert.
+// the padded tile offsets.  Inside the block, warp w owns 256 consecutive
+// slots and ranks them with rank_in_warp; a slot's sorted position is the
+// block's start for its expert + the expert's slots in lower warps + its rank
+// in the warp, i.e. ascending slot order within every expert.
 __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
     const int32_t* __restrict__ idx, int S, int E, int nblk,
     const int32_t* __restrict__ block_hist, int32_t* __restrict__ counts,
@@ -78,88 +147,86 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
     int32_t* __restrict__ perm, int32_t* __restrict__ inv, uint32_t* err,
     uint32_t* __restrict__ sched, int sched_words, int32_t* __restrict__ row_token, int k) {
   constexpr int kWarps = kRouteThreads / 32;
+  constexpr int kPer = kRouteChunk / kRouteThreads;   // 32-slot groups per warp
   griddep_launch_dependents();
   griddep_wait();
   // Block 0 also zeroes the fused GEMM's tile counter and per-m-tile
   // completion counts (sched may be null when no GEMM follows).
   if (blockIdx.x == 0 && sched != nullptr)
     for (int i = threadIdx.x; i < sched_words; i += blockDim.x) sched[i] = 0u;
-  __shared__ int32_t running[256];
-  __shared__ int32_t total[256];
+  __shared__ int32_t wpre[kWarps][256];   // per warp and expert: count, then lower warps' count
+  __shared__ int32_t start[256];          // this block's first position per expert
+  __shared__ int32_t total[257];
   __shared__ int32_t scan[257];
-  __shared__ int32_t tscan[257];   // padded m-tile offsets
-  __shared__ int32_t wcount[kWarps][256];
+  __shared__ int32_t tscan[257];          // padded m-tile offsets
+  __shared__ int32_t part[3][kWarps];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int base = blockIdx.x * kRouteChunk;
-  // The block's ids, loaded once up front (their latency overlaps the scan
-  // below) instead of once per sub-chunk.
-  constexpr int kPer = kRouteChunk / kRouteThreads;
+  const int wbase = base + warp * (kRouteChunk / kWarps);
+  // The warp's ids, loaded once up front (their latency overlaps the
+  // histogram sums below).
   int v[kPer];
 #pragma unroll
   for (int u = 0; u < kPer; ++u) {
-    const int s = base + tid + u * kRouteThreads;
+    const int s = wbase + u * 32 + lane;
     v[u] = s < S ? __ldg(&idx[s]) : kMaskedSlot;
   }
-  if (nblk == 1) {
-    // A single block holds every slot: count them here (no histogram launch).
-    for (int e = tid; e < E; e += blockDim.x) {
-      running[e] = 0;
-      total[e] = 0;
+  for (int e = lane; e < E; e += 32) wpre[warp][e] = 0;
+  // Thread e: expert e's slots in earlier blocks and in all blocks.
+  int before = 0, all = 0;
+  if (nblk > 1 && tid < E) {
+    for (int b = 0; b < nblk; ++b) {
+      const int c = block_hist[b * E + tid];
+      if (b < static_cast<int>(blockIdx.x)) before += c;
+      all += c;
     }
-    __syncthreads();
-    bool bad = false;
+  }
+  __syncwarp();
+  bool bad = false;
+  rank_in_warp<kPer>(v, kPer, E, wpre[warp], bad);
+  // With a single block nothing else has looked at the ids.
+  if (nblk == 1 && bad) atomicOr(err, kErrRoutingBit);
+  __syncthreads();
+  int mine = 0;   // this block's slots of expert tid
+  if (tid < E) {
 #pragma unroll
-    for (int u = 0; u < kPer; ++u) {   // S <= kRouteChunk: every id is in v
-      const int e = v[u];
-      if (e >= 0 && e < E) atomicAdd(&total[e], 1); else if (e != kMaskedSlot) bad = true;
-    }
-    if (bad) atomicOr(err, kErrRoutingBit);
-  } else {
-    for (int e = tid; e < E; e += blockDim.x) {
-      int before = 0, all = 0;
-      for (int b = 0; b < nblk; ++b) {
-        const int c = block_hist[b * E + e];
-        if (b < static_cast<int>(blockIdx.x)) before += c;
-        all += c;
-      }
-      running[e] = before;
-      total[e] = all;
+    for (int w = 0; w < kWarps; ++w) {
+      const int c = wpre[w][tid];
+      wpre[w][tid] = mine;
+      mine += c;
     }
   }
-  __syncthreads();
-  if (tid == 0) {
-    int acc = 0, tacc = 0, pacc = 0;
-    for (int e = 0; e < E; ++e) {
-      scan[e] = acc;
-      tscan[e] = tacc;
-      const int tiles = (total[e] + kTileM - 1) / kTileM;
-      if (blockIdx.x == 0) {
-        offsets[e] = acc;
-        counts[e] = total[e];
-        tile_off[e] = tacc;
-        pad_off[e] = tacc * kTileM;
-        if (pair_off != nullptr) pair_off[e] = pacc;   // pairs of m-tiles of one expert
-      }
-      acc += total[e];
-      tacc += tiles;
-      pacc += (tiles + 1) / 2;
-    }
-    scan[E] = acc;
-    tscan[E] = tacc;
+  if (nblk == 1) all = mine;
+  const ExpertOffsets o = expert_offsets(tid < E ? all : 0, part);
+  if (tid < E) {
+    total[tid] = all;
+    scan[tid] = o.slot;
+    tscan[tid] = o.tile;
+    start[tid] = o.slot + before;
     if (blockIdx.x == 0) {
-      offsets[E] = acc;
-      tile_off[E] = tacc;
-      pad_off[E] = tacc * kTileM;
-      if (pair_off != nullptr) pair_off[E] = pacc;
+      offsets[tid] = o.slot;
+      counts[tid] = all;
+      tile_off[tid] = o.tile;
+      pad_off[tid] = o.tile * kTileM;
+      if (pair_off != nullptr) pair_off[tid] = o.pair;   // pairs of m-tiles of one expert
+    }
+    if (tid == E - 1) {
+      scan[E] = o.slot_end;
+      tscan[E] = o.tile_end;
+      if (blockIdx.x == 0) {
+        offsets[E] = o.slot_end;
+        tile_off[E] = o.tile_end;
+        pad_off[E] = o.tile_end * kTileM;
+        if (pair_off != nullptr) pair_off[E] = o.pair_end;
+      }
     }
   }
   __syncthreads();
-  for (int e = tid; e < E; e += blockDim.x) running[e] += scan[e];
   // Padding rows of the row -> token map read -1 (experts split over blocks).
   if (row_token != nullptr) {
-    for (int e = blockIdx.x; e < E; e += gridDim.x) {
+    for (int e = blockIdx.x + warp * gridDim.x; e < E; e += kWarps * gridDim.x) {
       const int lo = tscan[e] * kTileM + total[e], hi = tscan[e + 1] * kTileM;
-      for (int r = lo + tid; r < hi; r += blockDim.x) row_token[r] = -1;
+      for (int r = lo + lane; r < hi; r += 32) row_token[r] = -1;
     }
   }
   // Positions past the routed slots (left by out-of-range ids) read -1.
@@ -168,43 +235,22 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
     if (p >= routed) perm[p] = -1;
 #pragma unroll
   for (int u = 0; u < kPer; ++u) {
-    const int sub = u * kRouteThreads;
-    for (int i = tid; i < kWarps * 256; i += blockDim.x) (&wcount[0][0])[i] = 0;
-    __syncthreads();
-    const int s = base + sub + tid;
-    int e = -1;
-    if (s < S) {
-      e = v[u];
-      if (e < 0 || e >= E) e = -1;
-    }
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    if (e >= 0 && rank == 0) wcount[warp][e] = __popc(peers);
-    __syncthreads();
-    if (s < S) {
-      if (e >= 0) {
-        int pos = running[e] + rank;
-        for (int w = 0; w < warp; ++w) pos += wcount[w][e];
-        if (pos >= 0 && pos < S) {   // always true; guards the store
-          perm[pos] = s;
-          inv[s] = pos;
-          if (row_token != nullptr) row_token[tscan[e] * kTileM + (pos - scan[e])] = s / k;
-        } else {
-          atomicOr(err, kErrRoutingBit);
-          inv[s] = -1;
-        }
+    const int s = wbase + u * 32 + lane;
+    if (s >= S) continue;
+    if (v[u] != kUnrouted) {
+      const int e = v[u] & 511;
+      const int pos = start[e] + wpre[warp][e] + (v[u] >> 9);
+      if (pos >= 0 && pos < S) {   // always true; guards the store
+        perm[pos] = s;
+        inv[s] = pos;
+        if (row_token != nullptr) row_token[tscan[e] * kTileM + (pos - scan[e])] = s / k;
       } else {
+        atomicOr(err, kErrRoutingBit);
         inv[s] = -1;
       }
+    } else {
+      inv[s] = -1;
     }
-    __syncthreads();
-    for (int ee = tid; ee < E; ee += blockDim.x) {
-      int add = 0;
-      for (int w = 0; w < kWarps; ++w) add += wcount[w][ee];
-      running[ee] += add;
-    }
-    __syncthreads();
-    if (base + sub + kRouteThreads >= S) break;
   }
 }
 
@@ -321,7 +367,6 @@ __global__ void __launch_bounds__(kRouteThreads) route_gather_kernel(
     int32_t* __restrict__ row_token, uint8_t* __restrict__ xg, uint8_t* __restrict__ xg_sf) {
   constexpr int kWarps = kRouteThreads / 32;
   constexpr int kPer = kFusedMaxSlots / kRouteThreads;   // 32-slot groups per warp, at most
-  constexpr int kNone = -1;                              // packed value of an unrouted slot
   extern __shared__ int32_t sorted[];   // [S] slot at each sorted position
   __shared__ int32_t wpre[kWarps][256];  // per warp and expert: count, then lower warps' count
   __shared__ int32_t total[257];
@@ -345,22 +390,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_gather_kernel(
   }
   __syncwarp();
   bool bad = false;
-  const unsigned lower = (1u << lane) - 1u;
-#pragma unroll
-  for (int u = 0; u < kPer; ++u) {
-    if (u * 32 >= chunk) break;   // warp-uniform
-    int e = v[u];
-    if (!(e >= 0 && e < E)) {
-      if (e != kMaskedSlot) bad = true;
-      e = -1;
-    }
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int before = e >= 0 ? wpre[warp][e] : 0;
-    __syncwarp();   // every lane has read its count before the group's leader updates it
-    if (e >= 0 && (peers & lower) == 0) wpre[warp][e] = before + __popc(peers);
-    __syncwarp();
-    v[u] = e >= 0 ? ((before + __popc(peers & lower)) << 9) | e : kNone;
-  }
+  rank_in_warp<kPer>(v, chunk / 32, E, wpre[warp], bad);
   if (lead && bad) atomicOr(err, kErrRoutingBit);
   __syncthreads();
   // Thread e: expert e's total, and its per-warp counts turned into the count
@@ -375,39 +405,25 @@ __global__ void __launch_bounds__(kRouteThreads) route_gather_kernel(
     }
     total[tid] = tot;
   }
-  const int tiles = (tot + kTileM - 1) / kTileM;
-  const int pairs = (tiles + 1) / 2;
-  // Inclusive scans over threads (experts) of tot, tiles and pairs.
-  int a = tot, b = tiles, c = pairs;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int a2 = __shfl_up_sync(0xffffffffu, a, off);
-    const int b2 = __shfl_up_sync(0xffffffffu, b, off);
-    const int c2 = __shfl_up_sync(0xffffffffu, c, off);
-    if (lane >= off) { a += a2; b += b2; c += c2; }
-  }
-  if (lane == 31) { part[0][warp] = a; part[1][warp] = b; part[2][warp] = c; }
-  __syncthreads();
-  for (int w = 0; w < warp; ++w) { a += part[0][w]; b += part[1][w]; c += part[2][w]; }
+  const ExpertOffsets o = expert_offsets(tot, part);
   if (tid < E) {
-    const int ex = a - tot, tex = b - tiles, pex = c - pairs;
-    scan[tid] = ex;
-    tscan[tid] = tex;
+    scan[tid] = o.slot;
+    tscan[tid] = o.tile;
     if (lead) {
-      offsets[tid] = ex;
+      offsets[tid] = o.slot;
       counts[tid] = tot;
-      tile_off[tid] = tex;
-      pad_off[tid] = tex * kTileM;
-      pair_off[tid] = pex;
+      tile_off[tid] = o.tile;
+      pad_off[tid] = o.tile * kTileM;
+      pair_off[tid] = o.pair;
     }
     if (tid == E - 1) {
-      scan[E] = a;
-      tscan[E] = b;
+      scan[E] = o.slot_end;
+      tscan[E] = o.tile_end;
       if (lead) {
-        offsets[E] = a;
-        tile_off[E] = b;
-        pad_off[E] = b * kTileM;
-        pair_off[E] = c;
+        offsets[E] = o.slot_end;
+        tile_off[E] = o.tile_end;
+        pad_off[E] = o.tile_end * kTileM;
+        pair_off[E] = o.pair_end;
       }
     }
   }
@@ -427,7 +443,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_gather_kernel(
     if (u * 32 >= chunk) break;
     const int s = warp * chunk + u * 32 + lane;
     if (s >= S) continue;
-    if (v[u] != kNone) {
+    if (v[u] != kUnrouted) {
       const int e = v[u] & 511;
       const int q = scan[e] + wpre[warp][e] + (v[u] >> 9);
       sorted[q] = s;   // q < routed <= S: the counts above bound it
