@@ -71,9 +71,9 @@ void compute_layout(moe_plan_s* p) {
   const bool bf16 = p->w_dtype == MOE_W_BF16;
   const size_t elem = bf16 ? 2 : 1;
   L.xg = take(rows * p->H * elem);
-  L.xg_sf = take(bf16 ? 0 : rows / kTileM * (p->H / 128) * 512);
+  L.xg_sf = take(bf16 ? 0 : rows / kTileM * sf_groups(p->H / 128) * 512);
   L.act = take(rows * p->I * elem);
-  L.act_sf = take(bf16 ? 0 : rows / kTileM * (p->I / 128) * 512);
+  L.act_sf = take(bf16 ? 0 : rows / kTileM * sf_groups(p->I / 128) * 512);
   L.y = take(S * p->H * 2);
   // One 1 KB record per (expert, n-tile, k-block) of each GEMM: the two 128-row
   // weight blocks of a 256-wide tile, each block's scale byte repeated 512 times.

@@ -123,7 +123,7 @@ struct Phase {
   int n_tiles;               // per m-tile: I/128 (FC1) or H/256 (FC2)
   int k_blocks;              // K / 128
   int b_rows_per_expert;     // 2I (FC1) or H (FC2)
-  const uint8_t* sfa_chunks; // [m-tiles][k_blocks][512]
+  const uint8_t* sfa_chunks; // token scales [m-tiles][sf_groups(k_blocks)][512]
   const uint8_t* w_sf;       // weight scales
   const uint8_t* a_tiles;    // A operand, pre-swizzled tiles [m-tiles][k_blocks][16 KB]
   const uint8_t* w_tiles;    // weights as pre-swizzled tiles [E * n-blocks][k_blocks][16 KB],
@@ -498,17 +498,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           __syncwarp();
         } else {
-          if (lane == 0) {
-            // Token scale chunk of the tile's m-tile (and of the next one for
-            // a wide tile).
+          // A group's first k-block brings the token scales of the group's four
+          // k-blocks (one chunk per m-tile; a wide tile's second m-tile too) and,
+          // for FP8 weights, writes the group's weight scales: the MMA issuer
+          // copies both into TMEM once per group.
+          const bool group_start = kb % kSfGroup == 0;
+          if (lane == 0 && group_start) {
+            const int groups = sf_groups(ph.k_blocks), g = kb / kSfGroup;
             mbar_expect_tx(&sm.full[stage], wide ? 1024 : 512);
             bulk_load(sm.sfa[stage],
-                      ph.sfa_chunks + (static_cast<size_t>(t.mt) * ph.k_blocks + kb) * 512, 512,
+                      ph.sfa_chunks + (static_cast<size_t>(t.mt) * groups + g) * 512, 512,
                       &sm.full[stage]);
             if (wide)
               bulk_load(sm.sfa[stage] + 512,
-                        ph.sfa_chunks + (static_cast<size_t>(t.mt + 1) * ph.k_blocks + kb) * 512,
-                        512, &sm.full[stage]);
+                        ph.sfa_chunks + (static_cast<size_t>(t.mt + 1) * groups + g) * 512, 512,
+                        &sm.full[stage]);
           }
           if (kFp4 && p.sf_chunked) {
             // Prepacked scales: the stage's two 512-byte chunks (128 weight rows
@@ -540,13 +544,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             cp_async_mbar_arrive_noinc(&sm.full[stage]);
           } else {
-            const uint32_t g = __shfl_sync(0xffffffffu, sf0, kb & 31) * 0x01010101u;
-            const uint32_t u = __shfl_sync(0xffffffffu, sf1, kb & 31) * 0x01010101u;
-            reinterpret_cast<uint4*>(sm.sfb[stage])[lane] = make_uint4(g, g, g, g);
-            reinterpret_cast<uint4*>(sm.sfb[stage] + 512)[lane] = make_uint4(u, u, u, u);
-            // Every lane makes its writes visible to the tensor core (async
-            // proxy); the warp barrier orders them before lane 0's release.
-            fence_proxy_async_smem();
+            if (group_start) {
+              // One scale per 128 x 128 weight block: byte c of every row's word
+              // is the block's scale for k-block kb + c (kb + c stays inside the
+              // 32 k-blocks held in sf0 / sf1).
+              uint32_t g = 0, u = 0;
+#pragma unroll
+              for (int c = 0; c < kSfGroup; ++c) {
+                const uint32_t gc = __shfl_sync(0xffffffffu, sf0, (kb + c) & 31);
+                const uint32_t uc = __shfl_sync(0xffffffffu, sf1, (kb + c) & 31);
+                if (kb + c < ph.k_blocks) {
+                  g |= (gc & 0xFFu) << (8 * c);
+                  u |= (uc & 0xFFu) << (8 * c);
+                }
+              }
+              reinterpret_cast<uint4*>(sm.sfb[stage])[lane] = make_uint4(g, g, g, g);
+              reinterpret_cast<uint4*>(sm.sfb[stage] + 512)[lane] = make_uint4(u, u, u, u);
+              // Every lane makes its writes visible to the tensor core (async
+              // proxy); the warp barrier orders them before lane 0's release.
+              fence_proxy_async_smem();
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.full[stage]);
           }
@@ -564,7 +581,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // k-block leaves the tensor pipe idle between k-blocks.
     if (lane == 0) {
       int slot = 0, stage = 0;
-      uint32_t sphase = 0, phase = 0, acc_phase = 0, sfset = 0;
+      uint32_t sphase = 0, phase = 0, acc_phase = 0;
+      // TMEM scale sets (two of each, alternating so that a copy never lands in
+      // the set the MMAs just issued may still read): token scales switch per
+      // group of four k-blocks, weight scales per k-block (MXFP4) or per group
+      // (FP8).  The first copy goes to set 0.
+      uint32_t tset = 1, wset = 1;
       // Shared-memory descriptors of stage 0, built once: a stage's descriptor
       // is stage 0's plus its byte offset >> 4, and each 32-byte K step of a
       // 128-byte k-block adds 2 (the 14-bit address field cannot carry: shared
@@ -622,45 +644,56 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Unchunked MXFP4 weight scales land by cp.async (generic proxy):
             // order them before the tensor core's (async proxy) reads.
             if (kFp4 && !p.sf_chunked) fence_proxy_async_smem();
-            const uint32_t sfa = tmem + C::kSfaCol + sfset * kSfSetStride;
-            const uint32_t sfb = tmem + C::kSfbCol + sfset * kSfSetStride;
-            const uint64_t sfad = sfa_desc0 + static_cast<uint64_t>(stage) * kSfaStage;
-            const uint64_t sfbd = sfb_desc0 + static_cast<uint64_t>(stage) * kSfbStage;
-            // Token scales: rows 0..127 in columns 0..3, a wide tile's rows
-            // 128.. in columns 4..7 (the layout N > 128 reads).
-            tmem_cp_32x128b_warpx4(sfa, sfad);
-            if (wide) tmem_cp_32x128b_warpx4(sfa + 4, sfad + kSfHalf);
-            tmem_cp_32x128b_warpx4(sfb, sfbd);
-            tmem_cp_32x128b_warpx4(sfb + 4, sfbd + kSfHalf);
+            // Scale-factor ids: the token operand reads byte kc of its words (its
+            // 1x128 scale for k-block kb); MXFP4 weights read byte ks (their four
+            // 1x32 scales), FP8 weights byte kc (one scale per 128 x 128 block).
+            const uint32_t kc = static_cast<uint32_t>(kb % kSfGroup);
+            const bool group_start = kc == 0;
+            const bool w_copy = kFp4 || group_start;
+            if (group_start) tset ^= 1u;
+            if (w_copy) wset ^= 1u;
+            const uint32_t sft = tmem + C::kSfaCol + tset * kSfSetStride;   // token scales
+            const uint32_t sfw = tmem + C::kSfbCol + wset * kSfSetStride;   // weight scales
+            if (group_start) {
+              // Token scales: rows 0..127 in columns 0..3, a wide tile's rows
+              // 128.. in columns 4..7 (the layout N > 128 reads).
+              const uint64_t sfad = sfa_desc0 + static_cast<uint64_t>(stage) * kSfaStage;
+              tmem_cp_32x128b_warpx4(sft, sfad);
+              if (wide) tmem_cp_32x128b_warpx4(sft + 4, sfad + kSfHalf);
+            }
+            if (w_copy) {
+              const uint64_t sfbd = sfb_desc0 + static_cast<uint64_t>(stage) * kSfbStage;
+              tmem_cp_32x128b_warpx4(sfw, sfbd);
+              tmem_cp_32x128b_warpx4(sfw + 4, sfbd + kSfHalf);
+            }
+            const uint32_t tok_sf = sft | (kc << 30);
             if (swap) {
               // Token-major: each 128-row half of the weight tile is the A
-              // operand (its scales: the weight chunk), the tile's tokens are B
-              // with N = their count rounded up to 16 (scales: the token chunk).
-              // D0 (columns 0..) holds the first half, D1 (columns 128..) the second.
+              // operand (A scale id: the weights'), the tile's tokens are B with
+              // N = their count rounded up to 16 (B scale id: kc).  D0 (columns
+              // 0..) holds the first half, D1 (columns 128..) the second.
 #pragma unroll
               for (int ks = 0; ks < 4; ++ks) {
-                const uint32_t idesc = idesc0 | (static_cast<uint32_t>(ks) << 4) |
-                                       (static_cast<uint32_t>(ks) << 29);
-                const uint32_t ksh = static_cast<uint32_t>(ks) << 30;
+                const uint32_t wid = kFp4 ? static_cast<uint32_t>(ks) : kc;
+                const uint32_t idesc = idesc0 | (kc << 4) | (wid << 29);
                 const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
                 mma_mxf8f6f4(tmem + kAccCol, bd + ks * kKStep, ad + ks * kKStep, idesc,
-                             sfb | ksh, sfa | ksh, acc);
+                             sfw | (wid << 30), tok_sf, acc);
                 mma_mxf8f6f4(tmem + kAccCol + C::kD1Col, bd + kBHalf + ks * kKStep,
-                             ad + ks * kKStep, idesc, (sfb + 4) | ksh, sfa | ksh, acc);
+                             ad + ks * kKStep, idesc, (sfw + 4) | (wid << 30), tok_sf, acc);
               }
             } else {
+              // Token rows are A (A scale id kc), the weights B.
 #pragma unroll
               for (int ks = 0; ks < 4; ++ks) {
-                const uint32_t idesc = idesc0 | (static_cast<uint32_t>(ks) << 4) |
-                                       (static_cast<uint32_t>(ks) << 29);
-                mma_mxf8f6f4(tmem + kAccCol, ad + ks * kKStep, bd + ks * kKStep, idesc,
-                             sfa | (static_cast<uint32_t>(ks) << 30),
-                             sfb | (static_cast<uint32_t>(ks) << 30), (kb > 0 || ks > 0) ? 1u : 0u);
+                const uint32_t wid = kFp4 ? static_cast<uint32_t>(ks) : kc;
+                const uint32_t idesc = idesc0 | (wid << 4) | (kc << 29);
+                mma_mxf8f6f4(tmem + kAccCol, ad + ks * kKStep, bd + ks * kKStep, idesc, tok_sf,
+                             sfw | (wid << 30), (kb > 0 || ks > 0) ? 1u : 0u);
               }
             }
           }
           tc_commit(&sm.empty[stage]);
-          sfset ^= 1u;
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -792,7 +825,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               ok = false;
               break;
             }
-            const int nb = p.I / 128;
+            const int nb = p.I / 128, groups = sf_groups(nb);
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
               const int j = lane + 32 * c;
@@ -803,9 +836,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (q == 0) sm.swap_inv[half][j] = __uint_as_float(static_cast<uint32_t>(127 - n) << 23);
                 if (q == 0) {
                   const int rr = half * 64 + j;   // row of the m-tile
-                  *reinterpret_cast<uint32_t*>(
-                      p.act_sf_chunks + (static_cast<size_t>(mt) * nb + t.nt) * 512 +
-                      (rr & 31) * 16 + (rr >> 5) * 4) = (static_cast<uint32_t>(n + 127) & 0xFFu) * 0x01010101u;
+                  p.act_sf_chunks[static_cast<size_t>(mt) * groups * 512 + sf_byte(rr, t.nt)] =
+                      static_cast<uint8_t>(n + 127);
                 }
               }
             }
@@ -959,14 +991,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(tile + swz128(row, half * 4 + v)) =
               make_uint4(w[0], w[1], w[2], w[3]);
         }
-        if (half == 0) {
-          const uint32_t sbyte = static_cast<uint32_t>(n + 127) & 0xFFu;
-          const int nb = p.I / 128;
-          uint32_t* sfd = reinterpret_cast<uint32_t*>(
-              p.act_sf_chunks + (static_cast<size_t>(t.mt) * nb + t.nt) * 512 +
-              (row & 31) * 16 + (row >> 5) * 4);
-          *sfd = sbyte * 0x01010101u;
-        }
+        if (half == 0)
+          p.act_sf_chunks[static_cast<size_t>(t.mt) * sf_groups(p.I / 128) * 512 +
+                          sf_byte(row, t.nt)] = static_cast<uint8_t>(n + 127);
         if (p.act_f32 != nullptr) {
           float4* fd = reinterpret_cast<float4*>(p.act_f32 + prow * p.I + t.nt * 128 + half * 64);
 #pragma unroll

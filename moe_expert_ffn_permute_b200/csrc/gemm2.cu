@@ -312,7 +312,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d_pair(sm.a[stage], &tm.a[g], 0, a_tile * 128, lead_full[stage], pol_a);
             tma_load_2d_pair(sm.b[stage], &tm.b[g], 0, b_tile * 128, lead_full[stage], pol_b);
           } else {
-            tma_load_2d_pair(sm.sfa[stage], &tm.sfa[g], 0, a_tile * 2, lead_full[stage], pol_a);
+            // Token scales: the chunk of the k-block's group (two 256-byte rows).
+            const int a_chunk = t.mt * sf_groups(ph.k_blocks) + kb / kSfGroup;
+            tma_load_2d_pair(sm.sfa[stage], &tm.sfa[g], 0, a_chunk * 2, lead_full[stage], pol_a);
             tma_load_2d_pair(sm.sfb[stage], &tm.sfb[g], 0, (rec0 + kb) * 4, lead_full[stage],
                              pol_b_reused);
           }
@@ -365,12 +367,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_cp_pair_32x128b_warpx4(sfb + 4, sfbd + (512 >> 4));
           const uint64_t ad = a_desc0 + static_cast<uint64_t>(stage) * kAStage;
           const uint64_t bd = b_desc0 + static_cast<uint64_t>(stage) * kBStage;
+          // Token rows (A) read byte kb % 4 of their scale words (the k-block's
+          // 1x128 scale); the weight records repeat one byte per block, read at
+          // K step ks.
+          const uint32_t kc = static_cast<uint32_t>(kb % kSfGroup);
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {
             mma_mxf8f6f4_pair(tmem + kAccCol, ad + ks * kKStep, bd + ks * kKStep,
-                              mxf8f6f4_idesc_m256(BN, ks),
-                              sfa | (static_cast<uint32_t>(ks) << 30),
-                              sfb | (static_cast<uint32_t>(ks) << 30),
+                              mxf8f6f4_idesc_m256(BN, 0) | (static_cast<uint32_t>(ks) << 4) |
+                                  (kc << 29),
+                              sfa | (kc << 30), sfb | (static_cast<uint32_t>(ks) << 30),
                               (kb > 0 || ks > 0) ? 1u : 0u);
           }
           tc_commit_pair_multicast(&sm.empty[stage], 0x3);
@@ -459,14 +465,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint4*>(tile + swz128(row, half * 4 + v)) =
                 make_uint4(w[0], w[1], w[2], w[3]);
           }
-          if (half == 0) {
-            const uint32_t sbyte = static_cast<uint32_t>(n + 127) & 0xFFu;
-            const int nb = p.I / 128;
-            uint32_t* sfd = reinterpret_cast<uint32_t*>(
-                p.act_sf_chunks + (static_cast<size_t>(t.mt) * nb + t.nt) * 512 +
-                (row & 31) * 16 + (row >> 5) * 4);
-            *sfd = sbyte * 0x01010101u;
-          }
+          if (half == 0)
+            p.act_sf_chunks[static_cast<size_t>(t.mt) * sf_groups(p.I / 128) * 512 +
+                            sf_byte(row, t.nt)] = static_cast<uint8_t>(n + 127);
           if (p.act_f32 != nullptr) {
             float4* fd =
                 reinterpret_cast<float4*>(p.act_f32 + prow * p.I + t.nt * 128 + half * 64);
@@ -611,8 +612,8 @@ cudaError_t launch_fc12_pairs(const moe_plan_s* pl, const void* w1, const uint8_
   const uint64_t E = pl->E;
   const uint64_t xg_bytes = rows * pl->H, act_bytes = rows * pl->I;
   const uint64_t w1_bytes = E * 2 * pl->I * pl->H, w2_bytes = E * pl->H * pl->I;
-  const uint64_t sfa1_bytes = rows / kTileM * (pl->H / 128) * 512;
-  const uint64_t sfa2_bytes = rows / kTileM * (pl->I / 128) * 512;
+  const uint64_t sfa1_bytes = rows / kTileM * sf_groups(pl->H / 128) * 512;
+  const uint64_t sfa2_bytes = rows / kTileM * sf_groups(pl->I / 128) * 512;
   const uint64_t sfb1_bytes = E * (pl->I / 128) * (pl->H / 128) * 1024;
   const uint64_t sfb2_bytes = E * (pl->H / 256) * (pl->I / 128) * 1024;
   Maps m;

@@ -15,6 +15,21 @@ constexpr int kRouteChunk = 2048;   // slots per routing block
 constexpr int kRouteThreads = 256;
 constexpr int kTileM = 128;          // rows per m-tile (expert blocks are padded to it)
 
+// Token scale chunks (the gathered x's and the FC1 activation's 1x128 UE8M0
+// scales, laid out for tcgen05.cp ...32x128b.warpx4): one 512-byte chunk per
+// 128-row tile and group of kSfGroup consecutive 128-wide k-blocks.  Row r's
+// scale for k-block kb is the byte at chunk kb / kSfGroup, offset
+// (r % 32) * 16 + (r / 32) * 4 + kb % kSfGroup.  A 1x128 scale is the same for
+// the four 32-wide K steps of its k-block, so the MMAs of k-block kb all read
+// byte kb % 4 (the scale-factor id) and one TMEM copy serves four k-blocks.
+constexpr int kSfGroup = 4;
+__host__ __device__ constexpr int sf_groups(int k_blocks) {
+  return (k_blocks + kSfGroup - 1) / kSfGroup;
+}
+__host__ __device__ constexpr int sf_byte(int r, int kb) {
+  return (kb / kSfGroup) * 512 + (r & 31) * 16 + (r >> 5) * 4 + kb % kSfGroup;
+}
+
 // Byte offsets of every buffer inside the caller's workspace (256-B aligned).
 struct WorkspaceLayout {
   size_t err, counts, offsets, pad_off, tile_off, pair_off;

@@ -28,6 +28,19 @@ namespace {
 // outside [0, E) is skipped and reported as MOE_ERR_BAD_ROUTING.
 constexpr int kMaskedSlot = -1;
 
+// The UE8M0 bytes of k-blocks 4g .. 4g+3 of one row of scales (0 past the
+// row's end), as the 32-bit word of group g in the token scale-chunk layout.
+__device__ __forceinline__ uint32_t sf_group_word(const uint8_t* __restrict__ row_sf, int kb_n,
+                                                  int g) {
+  uint32_t w = 0;
+#pragma unroll
+  for (int c = 0; c < kSfGroup; ++c) {
+    const int kb = g * kSfGroup + c;
+    if (kb < kb_n) w |= static_cast<uint32_t>(__ldg(&row_sf[kb])) << (8 * c);
+  }
+  return w;
+}
+
 // Kernel 1: per-block histograms of the block's kRouteChunk slots.
 __global__ void __launch_bounds__(kRouteThreads) route_hist_kernel(
     const int32_t* __restrict__ idx, int S, int E, int32_t* __restrict__ block_hist,
@@ -260,11 +273,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
 // (the e with offsets[e] <= inv[s] < offsets[e+1]) goes to padded row
 // pad_off[e] + inv[s] - offsets[e] (m-tile P / 128, row P % 128), in the
 // pre-swizzled tile layout the FC1 producer bulk-copies.  Its scale bytes go
-// to the tensor-core scale-chunk layout: for k-block kb the 512-byte chunk of
-// the tile holds, at byte (r % 32) * 16 + (r / 32) * 4 + j (j = 0..3), the
-// row's UE8M0 byte, replicated over the four 32-wide K sub-blocks.  Padding
-// rows are left untouched (their results are never stored).  Reading x once
-// per token instead of once per slot matters when x does not fit in L2.
+// to the token scale-chunk layout (sf_byte: one 512-byte chunk per tile and
+// group of four k-blocks, row r's four bytes at (r % 32) * 16 + (r / 32) * 4).
+// Padding rows are left untouched (their results are never stored).  Reading
+// x once per token instead of once per slot matters when x does not fit in L2.
 constexpr int kGatherWarps = 8;
 constexpr int kGatherBatch = 8;   // 16-byte vectors per lane per chunk
 
@@ -329,12 +341,11 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(
       const int P = __shfl_sync(0xffffffffu, prow, jj);
       if (P < 0) continue;
       const int r = P % kTileM;
-      uint8_t* chunk = xg_sf + static_cast<size_t>(P / kTileM) * kb_n * 512 + (r & 31) * 16 +
-                       (r >> 5) * 4;
-      for (int kb = lane; kb < kb_n; kb += 32) {
-        const uint32_t b = __ldg(&xs[static_cast<size_t>(t) * kb_n + kb]);
-        *reinterpret_cast<uint32_t*>(chunk + static_cast<size_t>(kb) * 512) = b * 0x01010101u;
-      }
+      const int groups = sf_groups(kb_n);
+      uint8_t* chunk = xg_sf + static_cast<size_t>(P / kTileM) * groups * 512 + sf_byte(r, 0);
+      for (int g = lane; g < groups; g += 32)
+        *reinterpret_cast<uint32_t*>(chunk + static_cast<size_t>(g) * 512) =
+            sf_group_word(xs + static_cast<size_t>(t) * kb_n, kb_n, g);
     }
   }
 }
@@ -476,10 +487,12 @@ __global__ void __launch_bounds__(kRouteThreads) route_gather_kernel(
     const uint4* __restrict__ src =
         reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * row_bytes);
     uint8_t* __restrict__ dst = xg + static_cast<size_t>(tile) * kb_n * kTileBytes;
-    // Rows of up to 8192 bytes move in one batch of loads; the scale bytes (up
-    // to 64 per row) are loaded with them.
+    // Rows of up to 8192 bytes move in one batch of loads; the scale words of
+    // up to 64 groups (256 k-blocks) are loaded with them.
     constexpr int kBatch = 16;
-    uint8_t* chunk = xg_sf + static_cast<size_t>(tile) * kb_n * 512 + (r & 31) * 16 + (r >> 5) * 4;
+    const int groups = sf_groups(kb_n);
+    uint8_t* chunk = xg_sf + static_cast<size_t>(tile) * groups * 512 + sf_byte(r, 0);
+    const uint8_t* row_sf = scales ? xs + static_cast<size_t>(t) * kb_n : nullptr;
     for (int c0 = lane; c0 < vec; c0 += 32 * kBatch) {
       uint4 xv[kBatch];
 #pragma unroll
@@ -491,8 +504,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_gather_kernel(
       if (scales && c0 == lane) {
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-          const int kb = lane + 32 * u;
-          if (kb < kb_n) sb[u] = __ldg(&xs[static_cast<size_t>(t) * kb_n + kb]);
+          const int g = lane + 32 * u;
+          if (g < groups) sb[u] = sf_group_word(row_sf, kb_n, g);
         }
       }
 #pragma unroll
@@ -505,17 +518,15 @@ __global__ void __launch_bounds__(kRouteThreads) route_gather_kernel(
       if (scales && c0 == lane) {
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-          const int kb = lane + 32 * u;
-          if (kb < kb_n)
-            *reinterpret_cast<uint32_t*>(chunk + static_cast<size_t>(kb) * 512) =
-                sb[u] * 0x01010101u;
+          const int g = lane + 32 * u;
+          if (g < groups)
+            *reinterpret_cast<uint32_t*>(chunk + static_cast<size_t>(g) * 512) = sb[u];
         }
       }
     }
-    for (int kb = lane + 64; scales && kb < kb_n; kb += 32) {   // rows > 8192 bytes
-      const uint32_t b = __ldg(&xs[static_cast<size_t>(t) * kb_n + kb]);
-      *reinterpret_cast<uint32_t*>(chunk + static_cast<size_t>(kb) * 512) = b * 0x01010101u;
-    }
+    for (int g = lane + 64; scales && g < groups; g += 32)   // rows of more than 256 k-blocks
+      *reinterpret_cast<uint32_t*>(chunk + static_cast<size_t>(g) * 512) =
+          sf_group_word(row_sf, kb_n, g);
   }
 }
 
@@ -528,7 +539,7 @@ __global__ void unpack_act_scales_kernel(const uint8_t* __restrict__ chunks, int
   const int b = static_cast<int>(i - r * nb);
   const long long tile = r / kTileM;
   const int rr = static_cast<int>(r - tile * kTileM);
-  dst[i] = chunks[(tile * nb + b) * 512 + (rr & 31) * 16 + (rr >> 5) * 4];
+  dst[i] = chunks[tile * sf_groups(nb) * 512 + sf_byte(rr, b)];
 }
 
 }  // namespace

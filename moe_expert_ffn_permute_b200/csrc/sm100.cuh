@@ -250,8 +250,10 @@ __device__ __forceinline__ uint64_t sf_desc(uint32_t smem_addr) {
 }
 
 // Instruction descriptor of tcgen05.mma.kind::mxf8f6f4.block_scale, M = 128,
-// K-major A and B, UE8M0 scales; sf_id picks the byte of each 32-bit scale
-// word (= which 32-wide K sub-block of a 128-wide stage).
+// K-major A and B, UE8M0 scales.  A scale id picks the byte of each 32-bit
+// scale word that an operand's MMA reads; the kernels pass sf_id = 0 here and
+// OR in each operand's id per instruction (the same id also goes into bits
+// 30-31 of that operand's TMEM scale address).
 //   bits 4-5 B scale id, 7-9 A format, 10-12 B format (0 E4M3, 5 E2M1),
 //   17-22 N >> 3, 23 scale type (1 = UE8M0), 24-28 M >> 4, 29-30 A scale id
 __host__ __device__ constexpr uint32_t mxf8f6f4_idesc(uint32_t b_format, uint32_t n,
