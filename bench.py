@@ -596,6 +596,26 @@ def run_b200(args):
         print(json.dumps(res))
 
 
+def run_forwards(args, wl):
+    """N forwards of one workload in the benchmark's launch configuration
+    (prepared weights, automatic tiles) and nothing else: the launches a
+    profiler captures, without the benchmark's timing around them."""
+    import torch
+
+    from moe_expert_ffn_permute_b200.build import build
+
+    build()
+    dev = torch.device("cuda", 0)
+    lb = LayerBench(wl, args, dev)
+    for _ in range(args.forwards):
+        lb.fwd()
+    torch.cuda.synchronize()
+    if lb.lay.check() != 0:
+        sys.exit(f"bench.py: device error word set after {args.forwards} forwards of {wl.name}")
+    print(f"{wl.name}: {args.forwards} forwards")
+    lb.release()
+
+
 def _oracle_sample(wl, dn, tokens):
     from oracle import layer as L
     sub = dict(dn)
@@ -705,6 +725,9 @@ def main():
     ap.add_argument("--row-major-weights", action="store_true",
                     help="weights as given (row-major, 2-D TMA; MXFP4 scales unchunked) "
                          "instead of prepacked")
+    ap.add_argument("--forwards", type=int, default=0,
+                    help="only run this many forwards of the workload on one GPU, untimed "
+                         "(the launches a profiler captures), and print no JSON line")
     args = ap.parse_args()
     if args.tokens is None and args.workload == HEADLINE[0]:
         args.tokens = HEADLINE[1]
@@ -715,7 +738,9 @@ def main():
         sys.exit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world_env}: launch one rank "
                  f"per GPU (torch.distributed.run --nproc-per-node {args.gpus})")
     wl = workload(args.workload, args.tokens)
-    if args.impl == "reference":
+    if args.forwards > 0:
+        run_forwards(args, wl)
+    elif args.impl == "reference":
         run_reference(args, wl)
     else:
         run_b200(args)

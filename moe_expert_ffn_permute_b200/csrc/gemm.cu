@@ -83,10 +83,10 @@ struct Cfg {
   static constexpr int kStages = kWide ? 3 : 4;
   static constexpr int kARows = kWide ? 2 * BM : BM;        // token rows a stage holds
   static constexpr uint32_t kD1Col = kWide ? 240u : 128u;    // token-major: second half's D
-  // TMEM scale sets (alternating per k-block, so that loading the next
-  // k-block's scales never waits for MMAs still reading the current ones):
-  // token scales (up to 8 columns: two 128-row chunks) and weight scales (8
-  // columns: two 128-row halves).
+  // TMEM scale sets, two of each kind used in turn (so that a copy never
+  // lands in the set that MMAs issued just before it may still read): token
+  // scales (up to 8 columns: two 128-row chunks) and weight scales (8 columns:
+  // two 128-row halves).
   static constexpr uint32_t kSfaCol = kWide ? 480u : 256u;
   static constexpr uint32_t kSfbCol = kWide ? 488u : 264u;
   static constexpr int kSfaBytes = kWide ? 1024 : 512;       // token scale chunk(s) per stage

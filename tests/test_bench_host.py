@@ -99,3 +99,19 @@ def test_gpus_disagreeing_with_world_size_is_refused(monkeypatch):
     with pytest.raises(SystemExit) as ei:
         bench.main()
     assert "WORLD_SIZE=2" in str(ei.value.code)
+
+
+def test_forwards_mode_dispatches_without_timing(monkeypatch):
+    """--forwards N runs only the profiler's launches (run_forwards) on the
+    workload and tokens given, never the timed benchmark or the oracle arm."""
+    import sys
+    bench = _load_bench()
+    seen = []
+    monkeypatch.setattr(bench, "run_forwards", lambda args, wl: seen.append((args.forwards, wl.name)))
+    monkeypatch.setattr(bench, "run_b200", lambda args: pytest.fail("timed run started"))
+    monkeypatch.setattr(bench, "run_reference", lambda args, wl: pytest.fail("oracle arm started"))
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--workload", "mxfp4", "--tokens", "128",
+                                      "--forwards", "4"])
+    bench.main()
+    assert seen == [(4, bench.workload("mxfp4", 128).name)]
